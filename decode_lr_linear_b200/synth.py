@@ -10,13 +10,11 @@ GEMVs, dequantisation inside a product, SwiGLU, softmax, per-token requant)
 lives here; that is written twice, once in ``oracle/`` and once in the CUDA
 kernels, and the two share nothing but the arrays produced below.
 
-Layout convention for stored factors (the library's ABI):
-  * ``At``: the first factor stored output-major, shape [rank, d_in]
-    (row j holds column j of A, A being d_in x rank),
-  * ``Bt``: the second factor stored output-major, shape [d_out, rank]
-    (row k holds column k of B, B being rank x d_out),
-so that y = (x @ A) @ B = (x @ At.T) @ Bt.T.  This is the storage of two
-chained ``nn.Linear`` layers, and the math layout is recovered with ``.T``.
+Layout convention for stored factors (the library's ABI): both factors are
+stored latent-major, one contiguous row per latent component j:
+  * ``At``: [rank, d_in]  -- row j is column j of A (A is d_in x rank),
+  * ``B``:  [rank, d_out] -- row j is row j of B (B is rank x d_out),
+so that y = (x @ A) @ B = sum_j (x . At[j]) B[j].
 
 Random draws: every large Gaussian array is filled in fixed-size chunks, each
 from its own child of ``numpy.random.SeedSequence(seed, spawn_key=key)``, so
@@ -107,10 +105,10 @@ def make_single_linear(seed: int = 0, d: int = 256, rank: int = 32, exact_rank: 
     B = sr[:, None] * V[:, :rank].T
     x = rng.standard_normal((1, d))
     At32 = np.ascontiguousarray(A.T.astype(np.float32))
-    Bt32 = np.ascontiguousarray(B.T.astype(np.float32))
+    B32 = np.ascontiguousarray(B.astype(np.float32))
     return {
         "U": U, "V": V, "sigma": sigma, "W": W, "A": A, "B": B,
-        "At": torch.from_numpy(At32), "Bt": torch.from_numpy(Bt32),
+        "At": torch.from_numpy(At32), "B32": torch.from_numpy(B32),
         "x": torch.from_numpy(x.astype(np.float32)),
         "d_in": d, "d_out": d, "rank": rank,
     }
@@ -199,25 +197,25 @@ def attention_ranks(seed: int = 0, layers: int = 32, hidden: int = 4096,
 def _lr_factors(d_in: int, d_out: int, rank: int, seed: int, key: tuple):
     """Gaussian-column factor pair with a decaying spectrum.
 
-    A = G_A / sqrt(d_in) diag(sigma)^1/2, B = diag(sigma)^1/2 G_B^T / sqrt(d_out),
+    A = G_A / sqrt(d_in) diag(sigma)^1/2, B = diag(sigma)^1/2 G_B / sqrt(d_out),
     sigma_i = c i^-1/2 with c = sqrt(d_out / H_rank), which gives
-    Var(y_k) = 1 for x ~ N(0, I).  Returns (At, Bt) float32, output-major.
+    Var(y_k) = 1 for x ~ N(0, I).  Returns (At [rank, d_in], B [rank, d_out]) float32.
     """
     sig = math.sqrt(d_out / harmonic(rank)) / np.sqrt(np.arange(1, rank + 1, dtype=np.float64))
     sq = np.sqrt(sig).astype(np.float32)
     At = normals((rank, d_in), seed, key + (0,))
     At *= (sq / np.float32(math.sqrt(d_in)))[:, None]
-    Bt = normals((d_out, rank), seed, key + (1,))
-    Bt *= (sq / np.float32(math.sqrt(d_out)))[None, :]
-    return At, Bt
+    B = normals((rank, d_out), seed, key + (1,))
+    B *= (sq / np.float32(math.sqrt(d_out)))[:, None]
+    return At, B
 
 
 def make_attention_layer(layer: int, ranks: np.ndarray, seed: int = 0, hidden: int = 4096) -> dict:
     """bf16 factors of one layer's Q/K/V/O projections (LLaMA-7B shapes)."""
     out = {}
     for p, name in enumerate(ATTN_PROJ):
-        At, Bt = _lr_factors(hidden, hidden, int(ranks[layer, p]), seed, (2, 1, layer, p))
-        out[name] = {"At": to_bf16(At), "Bt": to_bf16(Bt), "rank": int(ranks[layer, p]),
+        At, B = _lr_factors(hidden, hidden, int(ranks[layer, p]), seed, (2, 1, layer, p))
+        out[name] = {"At": to_bf16(At), "B": to_bf16(B), "rank": int(ranks[layer, p]),
                      "d_in": hidden, "d_out": hidden}
     return out
 
@@ -236,7 +234,7 @@ def make_activations(batch: int, dim: int, seed: int, key: tuple, outliers: int 
 # Round-to-nearest int8 weights with per-output-channel scales.
 # --------------------------------------------------------------------------
 def rtn_int8_rows(Wt: np.ndarray, scale_dtype=np.float16):
-    """Symmetric RTN of an output-major weight [n_out, n_in]: one scale per output row.
+    """Symmetric RTN with one scale per row (rows are the output channels).
 
     s = max|w| / 127 rounded to ``scale_dtype``; q = clamp(rint(w / s), -127, 127)
     against the rounded s (ties to even); s == 0 gives q == 0.
@@ -249,6 +247,12 @@ def rtn_int8_rows(Wt: np.ndarray, scale_dtype=np.float16):
     q = np.clip(np.rint(Wt / safe[:, None]), -127, 127)
     q[s64 == 0] = 0
     return q.astype(np.int8), s
+
+
+def rtn_int8_cols(W: np.ndarray, scale_dtype=np.float16):
+    """Symmetric RTN with one scale per column (columns are the output channels)."""
+    q, s = rtn_int8_rows(np.asarray(W).T, scale_dtype)
+    return np.ascontiguousarray(q.T), s
 
 
 def hadamard(n: int) -> np.ndarray:
@@ -284,29 +288,29 @@ def make_hybrid_ffn(seed: int = 0, hidden: int = 4096, inter: int = 11008, n_lr:
     is folded as A' = A R, B' = R^T B, then every stored matrix is RTN int8
     with an fp16 scale per output channel.
 
-    Stored tensors (output-major, int8):
-      A_q  [rank, hidden]        s_A  [rank]
-      B_q  [2*n_lr, rank]        s_B  [2*n_lr]     rows interleaved gate0, up0, gate1, up1, ...
-      D_q  [2*n_dense, hidden]   s_D  [2*n_dense]  rows interleaved likewise
-      Wd_q [hidden, inter]       s_d  [hidden]     columns in [S; D] channel order
+    Stored tensors (int8; every scale belongs to one output channel):
+      A_q  [rank, hidden]        s_A  [rank]       latent-major (row j = latent channel j)
+      B_q  [rank, 2*n_lr]        s_B  [2*n_lr]     latent-major; columns interleaved gate0, up0, gate1, up1, ...
+      D_q  [2*n_dense, hidden]   s_D  [2*n_dense]  output-major; rows interleaved gate0, up0, ...
+      Wd_q [hidden, inter]       s_d  [hidden]     output-major; columns in [S; D] channel order
     """
     n_dense = inter - n_lr
     key = (3,)
     out = {"hidden": hidden, "inter": inter, "n_lr": n_lr, "n_dense": n_dense, "rank": rank}
     if n_lr > 0:
-        At, Bt = _lr_factors(hidden, 2 * n_lr, rank, seed, key + (1,))
+        At, B = _lr_factors(hidden, 2 * n_lr, rank, seed, key + (1,))
         At = At.astype(np.float64)
-        Bt = Bt.astype(np.float64)
+        B = B.astype(np.float64)
         if rotate:
             R = make_rotation(rank, seed)
-            # A' = A R  ->  A'^T = R^T A^T ;  B' = R^T B  ->  B'^T = B^T R
+            # A' = A R  ->  A'^T = R^T A^T ;  B' = R^T B
             At = R.T @ At
-            Bt = Bt @ R
+            B = R.T @ B
         qA, sA = rtn_int8_rows(At)
-        qB, sB = rtn_int8_rows(Bt)
+        qB, sB = rtn_int8_cols(B)
     else:
         qA = np.zeros((rank, hidden), np.int8); sA = np.zeros(rank, np.float16)
-        qB = np.zeros((0, rank), np.int8); sB = np.zeros(0, np.float16)
+        qB = np.zeros((rank, 0), np.int8); sB = np.zeros(0, np.float16)
     Dt = normals((2 * n_dense, hidden), seed, key + (2,)) / np.float32(math.sqrt(hidden))
     qD, sD = rtn_int8_rows(Dt)
     Wd = normals((hidden, inter), seed, key + (3,)) / np.float32(math.sqrt(inter))
@@ -382,10 +386,10 @@ def prefill_ranks(seed: int = 0, layers: int = 40, hidden: int = 5120, inter: in
 
 
 def make_prefill_projection(d_in: int, d_out: int, rank: int, seed: int, key: tuple) -> dict:
-    """int8 factors with fp32 per-output-channel scales: A_q [rank, d_in] s_A [rank],
-    B_q [d_out, rank] s_B [d_out] (output-major)."""
-    At, Bt = _lr_factors(d_in, d_out, rank, seed, (5, 1) + tuple(key))
+    """int8 factors with fp32 per-output-channel scales, latent-major:
+    A_q [rank, d_in] s_A [rank], B_q [rank, d_out] s_B [d_out]."""
+    At, B = _lr_factors(d_in, d_out, rank, seed, (5, 1) + tuple(key))
     qA, sA = rtn_int8_rows(At, np.float32)
-    qB, sB = rtn_int8_rows(Bt, np.float32)
+    qB, sB = rtn_int8_cols(B, np.float32)
     return {"A_q": torch.from_numpy(qA), "s_A": torch.from_numpy(sA), "B_q": torch.from_numpy(qB),
             "s_B": torch.from_numpy(sB), "d_in": d_in, "d_out": d_out, "rank": rank}

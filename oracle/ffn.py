@@ -7,11 +7,11 @@ quantised after an orthogonal rotation is inserted between the SVD factors.
 LASER "System Implementation" fuses the input projection, the latent
 activation, SwiGLU and the (de)quantisation.
 
-Stored layout consumed here (the library's; math layout is the transpose):
-  A_q  [r, hidden]       int8, s_A [r]         -> A' = (A_q * s_A[:,None]).T   hidden x r
-  B_q  [2 n_lr, r]       int8, s_B [2 n_lr]    -> B' rows interleaved gate_c, up_c
-  D_q  [2 n_dense, hidden] int8, s_D           -> dense gate/up, interleaved the same way
-  Wd_q [hidden, inter]   int8, s_d [hidden]    -> down_proj, input channels in [S; D] order
+Stored layout consumed here (the library's), every scale per output channel:
+  A_q  [r, hidden]         int8, s_A [r]        A' = (A_q * s_A[:,None]).T   (hidden x r)
+  B_q  [r, 2 n_lr]         int8, s_B [2 n_lr]   B' = B_q * s_B[None,:]; columns gate_0, up_0, gate_1, ...
+  D_q  [2 n_dense, hidden] int8, s_D            dense gate/up rows, interleaved the same way
+  Wd_q [hidden, inter]     int8, s_d [hidden]   down_proj (transposed), input channels in [S; D] order
 """
 from __future__ import annotations
 
@@ -24,6 +24,12 @@ def dequantize_rows(q, s) -> np.ndarray:
     """w = q * s with one scale per stored row (= per output channel), in float64."""
     q, s = _f64(q), _f64(s)
     return q * s[:, None]
+
+
+def dequantize_cols(q, s) -> np.ndarray:
+    """w = q * s with one scale per column (= per output channel), in float64."""
+    q, s = _f64(q), _f64(s)
+    return q * s[None, :]
 
 
 def silu(t) -> np.ndarray:
@@ -57,7 +63,7 @@ def hybrid_swiglu_ffn(x, A_q, s_A, B_q, s_B, D_q, s_D, Wd_q, s_d, n_lr: int, n_d
     Returns (y, h) with y [batch, hidden] and h [batch, n_lr + n_dense].
     """
     A = dequantize_rows(A_q, s_A).T                   # hidden x r
-    Bs = dequantize_rows(B_q, s_B).T if n_lr else None  # r x 2 n_lr
+    Bs = dequantize_cols(B_q, s_B) if n_lr else None  # r x 2 n_lr
     Ds = dequantize_rows(D_q, s_D).T if n_dense else None  # hidden x 2 n_dense
     Wdown = dequantize_rows(Wd_q, s_d).T              # inter x hidden
     x = _f64(x)

@@ -12,9 +12,9 @@ results and the requantised latent can be compared bit for bit:
   z[t,j]    = fp32( fp32( (float)acc1[t,j] * s_x[t] ) * s_A[j] )
   s_z[t]    = fp32( max_j |z[t,j]| / 127 )   (1 if that is 0, then z_q = 0)
   zq[t,j]   = clamp( rint_even( fp32( z[t,j] / s_z[t] ) ), -127, 127 )
-  acc2[t,k] = sum_j zq[t,j] Bq[k,j]                       (exact integer)
+  acc2[t,k] = sum_j zq[t,j] Bq[j,k]                       (exact integer)
   y[t,k]    = bf16_rn( fp32( fp32( (float)acc2[t,k] * s_z[t] ) * s_B[k] ) )
-Storage is output-major: Aq [r, d_in], Bq [d_out, r].
+Storage is latent-major: Aq [r, d_in] (row j = latent channel j), Bq [r, d_out].
 """
 from __future__ import annotations
 
@@ -78,7 +78,7 @@ def w8a8_lr_linear(xq, s_x, Aq, s_A, Bq, s_B) -> dict:
     """The full W8A8 low-rank pipeline; returns every intermediate."""
     acc1 = int_matmul_nt(xq, Aq)
     z, zq, s_z = requant_latent(acc1, s_x, s_A)
-    acc2 = int_matmul_nt(zq, Bq)
+    acc2 = int_matmul_nt(zq, _np(Bq).T)
     y32 = (acc2.astype(np.float32) * s_z[:, None]).astype(np.float32)
     y32 = (y32 * _np(s_B).astype(np.float32)[None, :]).astype(np.float32)
     return {"acc1": acc1, "z": z, "zq": zq, "s_z": s_z, "acc2": acc2, "y": bf16_round(y32)}
@@ -86,8 +86,8 @@ def w8a8_lr_linear(xq, s_x, Aq, s_A, Bq, s_B) -> dict:
 
 def w8a8_dequant_reference(xq, s_x, Aq, s_A, Bq, s_B) -> np.ndarray:
     """Float64 definition without the latent requant: y = (X A) B with X = xq s_x,
-    A = (Aq s_A)^T, B = (Bq s_B)^T."""
+    A = (Aq s_A)^T, B = Bq s_B (column scales)."""
     X = _np(xq).astype(np.float64) * _np(s_x).astype(np.float64)[:, None]
     A = (_np(Aq).astype(np.float64) * _np(s_A).astype(np.float64)[:, None]).T
-    B = (_np(Bq).astype(np.float64) * _np(s_B).astype(np.float64)[:, None]).T
+    B = _np(Bq).astype(np.float64) * _np(s_B).astype(np.float64)[None, :]
     return (X @ A) @ B

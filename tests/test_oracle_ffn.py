@@ -19,7 +19,7 @@ def _tiny_case(seed=0, hidden=5, n_lr=2, n_dense=3, r=2):
     return dict(
         x=rng.standard_normal((2, hidden)),
         A_q=_rand_q(rng, (r, hidden)), s_A=rng.uniform(0.001, 0.01, r),
-        B_q=_rand_q(rng, (2 * n_lr, r)), s_B=rng.uniform(0.001, 0.01, 2 * n_lr),
+        B_q=_rand_q(rng, (r, 2 * n_lr)), s_B=rng.uniform(0.001, 0.01, 2 * n_lr),
         D_q=_rand_q(rng, (2 * n_dense, hidden)), s_D=rng.uniform(0.001, 0.01, 2 * n_dense),
         Wd_q=_rand_q(rng, (hidden, inter)), s_d=rng.uniform(0.001, 0.01, hidden),
         n_lr=n_lr, n_dense=n_dense,
@@ -37,8 +37,8 @@ def _brute_ffn(c):
         h = []
         z = [sum(x[b, i] * float(c["A_q"][j, i]) * c["s_A"][j] for i in range(hidden)) for j in range(r)]
         for ch in range(n_lr):
-            g = sum(z[j] * float(c["B_q"][2 * ch, j]) * c["s_B"][2 * ch] for j in range(r))
-            u = sum(z[j] * float(c["B_q"][2 * ch + 1, j]) * c["s_B"][2 * ch + 1] for j in range(r))
+            g = sum(z[j] * float(c["B_q"][j, 2 * ch]) * c["s_B"][2 * ch] for j in range(r))
+            u = sum(z[j] * float(c["B_q"][j, 2 * ch + 1]) * c["s_B"][2 * ch + 1] for j in range(r))
             h.append(g / (1 + math.exp(-g)) * u)
         for ch in range(n_dense):
             g = sum(x[b, i] * float(c["D_q"][2 * ch, i]) * c["s_D"][2 * ch] for i in range(hidden))
@@ -87,7 +87,7 @@ def test_integer_preactivations_exact():
         c[k] = np.ones_like(c[k])
     _, h = O.hybrid_swiglu_ffn(**c)
     z = c["x"].astype(np.int64) @ c["A_q"].astype(np.int64).T
-    gu = z @ c["B_q"].astype(np.int64).T
+    gu = z @ c["B_q"].astype(np.int64)
     g, u = gu[:, 0::2].astype(np.float64), gu[:, 1::2].astype(np.float64)
     with np.errstate(over="ignore"):
         ref = g / (1 + np.exp(-g)) * u
@@ -101,7 +101,7 @@ def test_channel_permutation_invariance():
     perm = np.array([2, 0, 3, 1])
     rows = np.stack([2 * perm, 2 * perm + 1], axis=1).reshape(-1)
     c2 = dict(c)
-    c2["B_q"] = c["B_q"][rows]
+    c2["B_q"] = c["B_q"][:, rows]
     c2["s_B"] = c["s_B"][rows]
     cols = np.concatenate([perm, np.arange(4, 6)])
     c2["Wd_q"] = c["Wd_q"][:, cols]
@@ -110,7 +110,7 @@ def test_channel_permutation_invariance():
     # swapping gate and up of one channel changes the result (silu is not symmetric)
     c3 = dict(c)
     sw = np.arange(8); sw[[0, 1]] = [1, 0]
-    c3["B_q"] = c["B_q"][sw]; c3["s_B"] = c["s_B"][sw]
+    c3["B_q"] = c["B_q"][:, sw]; c3["s_B"] = c["s_B"][sw]
     y3, _ = O.hybrid_swiglu_ffn(**c3)
     assert np.abs(y0 - y3).max() > 1e-6
 
@@ -119,7 +119,7 @@ def test_math_layout_matches_stored_layout():
     c = _tiny_case(13, hidden=6, n_lr=2, n_dense=2, r=3)
     y, _ = O.hybrid_swiglu_ffn(**c)
     A = O.dequantize_rows(c["A_q"], c["s_A"]).T
-    Bs = O.dequantize_rows(c["B_q"], c["s_B"]).T
+    Bs = O.dequantize_cols(c["B_q"], c["s_B"])
     Ds = O.dequantize_rows(c["D_q"], c["s_D"]).T
     Wd = O.dequantize_rows(c["Wd_q"], c["s_d"]).T
     y2 = O.swiglu_ffn_math(c["x"], A, Bs[:, 0::2], Bs[:, 1::2], Ds[:, 0::2], Ds[:, 1::2], Wd)

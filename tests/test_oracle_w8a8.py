@@ -64,7 +64,7 @@ def test_pipeline_close_to_fp64_definition():
     ref = O.w8a8_dequant_reference(xq, sx, p["A_q"], p["s_A"], p["B_q"], p["s_B"])
     rel = np.linalg.norm(res["y"] - ref, axis=1) / np.linalg.norm(ref, axis=1)
     assert rel.max() < 1e-2
-    ref2 = np.einsum("tj,kj->tk", res["zq"].astype(np.int64), p["B_q"].numpy().astype(np.int64))
+    ref2 = np.einsum("tj,jk->tk", res["zq"].astype(np.int64), p["B_q"].numpy().astype(np.int64))
     assert np.array_equal(res["acc2"], ref2)
     del rng
 
@@ -74,7 +74,7 @@ def test_unit_scale_integer_pipeline():
     rng = np.random.default_rng(4)
     xq = rng.integers(-5, 6, size=(3, 32)).astype(np.int8)
     Aq = rng.integers(-5, 6, size=(8, 32)).astype(np.int8)
-    Bq = rng.integers(-5, 6, size=(6, 8)).astype(np.int8)
+    Bq = rng.integers(-5, 6, size=(8, 6)).astype(np.int8)
     one = np.ones
     res = O.w8a8_lr_linear(xq, one(3, np.float32), Aq, one(8, np.float32), Bq, one(6, np.float32))
     acc1 = xq.astype(np.int64) @ Aq.astype(np.int64).T

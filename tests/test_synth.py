@@ -84,7 +84,7 @@ def test_latent_factor_spectrum():
 def test_hybrid_ffn_shapes():
     d = synth.make_hybrid_ffn(seed=0, hidden=128, inter=96, n_lr=64, rank=512)
     assert tuple(d["A_q"].shape) == (512, 128)
-    assert tuple(d["B_q"].shape) == (128, 512)
+    assert tuple(d["B_q"].shape) == (512, 128)
     assert tuple(d["D_q"].shape) == (64, 128)
     assert tuple(d["Wd_q"].shape) == (128, 96)
     assert d["s_A"].dtype.itemsize == 2
