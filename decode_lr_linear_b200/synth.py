@@ -292,7 +292,7 @@ def make_hybrid_ffn(seed: int = 0, hidden: int = 4096, inter: int = 11008, n_lr:
       A_q  [rank, hidden]        s_A  [rank]       latent-major (row j = latent channel j)
       B_q  [rank, 2*n_lr]        s_B  [2*n_lr]     latent-major; columns interleaved gate0, up0, gate1, up1, ...
       D_q  [2*n_dense, hidden]   s_D  [2*n_dense]  output-major; rows interleaved gate0, up0, ...
-      Wd_q [hidden, inter]       s_d  [hidden]     output-major; columns in [S; D] channel order
+      Wd_q [inter, hidden]       s_d  [hidden]     input-major; rows in [S; D] channel order
     """
     n_dense = inter - n_lr
     key = (3,)
@@ -313,8 +313,8 @@ def make_hybrid_ffn(seed: int = 0, hidden: int = 4096, inter: int = 11008, n_lr:
         qB = np.zeros((rank, 0), np.int8); sB = np.zeros(0, np.float16)
     Dt = normals((2 * n_dense, hidden), seed, key + (2,)) / np.float32(math.sqrt(hidden))
     qD, sD = rtn_int8_rows(Dt)
-    Wd = normals((hidden, inter), seed, key + (3,)) / np.float32(math.sqrt(inter))
-    qd, sd = rtn_int8_rows(Wd)
+    Wd = normals((inter, hidden), seed, key + (3,)) / np.float32(math.sqrt(inter))
+    qd, sd = rtn_int8_cols(Wd)
     for name, arr in (("A_q", qA), ("s_A", sA), ("B_q", qB), ("s_B", sB), ("D_q", qD), ("s_D", sD),
                       ("Wd_q", qd), ("s_d", sd)):
         out[name] = torch.from_numpy(np.ascontiguousarray(arr))

@@ -11,7 +11,7 @@ Stored layout consumed here (the library's), every scale per output channel:
   A_q  [r, hidden]         int8, s_A [r]        A' = (A_q * s_A[:,None]).T   (hidden x r)
   B_q  [r, 2 n_lr]         int8, s_B [2 n_lr]   B' = B_q * s_B[None,:]; columns gate_0, up_0, gate_1, ...
   D_q  [2 n_dense, hidden] int8, s_D            dense gate/up rows, interleaved the same way
-  Wd_q [hidden, inter]     int8, s_d [hidden]   down_proj (transposed), input channels in [S; D] order
+  Wd_q [inter, hidden]     int8, s_d [hidden]   down_proj W_down = Wd_q * s_d[None,:]; rows in [S; D] order
 """
 from __future__ import annotations
 
@@ -65,7 +65,7 @@ def hybrid_swiglu_ffn(x, A_q, s_A, B_q, s_B, D_q, s_D, Wd_q, s_d, n_lr: int, n_d
     A = dequantize_rows(A_q, s_A).T                   # hidden x r
     Bs = dequantize_cols(B_q, s_B) if n_lr else None  # r x 2 n_lr
     Ds = dequantize_rows(D_q, s_D).T if n_dense else None  # hidden x 2 n_dense
-    Wdown = dequantize_rows(Wd_q, s_d).T              # inter x hidden
+    Wdown = dequantize_cols(Wd_q, s_d)                # inter x hidden
     x = _f64(x)
     parts = []
     if n_lr:

@@ -21,7 +21,7 @@ def _tiny_case(seed=0, hidden=5, n_lr=2, n_dense=3, r=2):
         A_q=_rand_q(rng, (r, hidden)), s_A=rng.uniform(0.001, 0.01, r),
         B_q=_rand_q(rng, (r, 2 * n_lr)), s_B=rng.uniform(0.001, 0.01, 2 * n_lr),
         D_q=_rand_q(rng, (2 * n_dense, hidden)), s_D=rng.uniform(0.001, 0.01, 2 * n_dense),
-        Wd_q=_rand_q(rng, (hidden, inter)), s_d=rng.uniform(0.001, 0.01, hidden),
+        Wd_q=_rand_q(rng, (inter, hidden)), s_d=rng.uniform(0.001, 0.01, hidden),
         n_lr=n_lr, n_dense=n_dense,
     )
 
@@ -45,7 +45,7 @@ def _brute_ffn(c):
             u = sum(x[b, i] * float(c["D_q"][2 * ch + 1, i]) * c["s_D"][2 * ch + 1] for i in range(hidden))
             h.append(g / (1 + math.exp(-g)) * u)
         for k in range(hidden):
-            y[b, k] = sum(h[c2] * float(c["Wd_q"][k, c2]) * c["s_d"][k] for c2 in range(len(h)))
+            y[b, k] = sum(h[c2] * float(c["Wd_q"][c2, k]) * c["s_d"][k] for c2 in range(len(h)))
     return y
 
 
@@ -72,7 +72,7 @@ def test_no_lowrank_channels_is_dense_swiglu():
                                d["Wd_q"], d["s_d"], 0, 48)
     Dq = d["D_q"].double() * d["s_D"].double()[:, None]      # [2*48, 64]
     Wg, Wu = Dq[0::2].T, Dq[1::2].T                           # 64 x 48 each
-    Wdown = (d["Wd_q"].double() * d["s_d"].double()[:, None]).T  # 48 x 64
+    Wdown = d["Wd_q"].double() * d["s_d"].double()[None, :]  # 48 x 64
     xt = torch.from_numpy(x)
     ref = (F.silu(xt @ Wg) * (xt @ Wu)) @ Wdown
     assert np.abs(y - ref.numpy()).max() < 1e-12
@@ -104,7 +104,7 @@ def test_channel_permutation_invariance():
     c2["B_q"] = c["B_q"][:, rows]
     c2["s_B"] = c["s_B"][rows]
     cols = np.concatenate([perm, np.arange(4, 6)])
-    c2["Wd_q"] = c["Wd_q"][:, cols]
+    c2["Wd_q"] = c["Wd_q"][cols, :]
     y1, _ = O.hybrid_swiglu_ffn(**c2)
     assert np.abs(y0 - y1).max() < 1e-12
     # swapping gate and up of one channel changes the result (silu is not symmetric)
@@ -121,6 +121,6 @@ def test_math_layout_matches_stored_layout():
     A = O.dequantize_rows(c["A_q"], c["s_A"]).T
     Bs = O.dequantize_cols(c["B_q"], c["s_B"])
     Ds = O.dequantize_rows(c["D_q"], c["s_D"]).T
-    Wd = O.dequantize_rows(c["Wd_q"], c["s_d"]).T
+    Wd = O.dequantize_cols(c["Wd_q"], c["s_d"])
     y2 = O.swiglu_ffn_math(c["x"], A, Bs[:, 0::2], Bs[:, 1::2], Ds[:, 0::2], Ds[:, 1::2], Wd)
     assert np.abs(y - y2).max() < 1e-12

@@ -86,7 +86,7 @@ def test_hybrid_ffn_shapes():
     assert tuple(d["A_q"].shape) == (512, 128)
     assert tuple(d["B_q"].shape) == (512, 128)
     assert tuple(d["D_q"].shape) == (64, 128)
-    assert tuple(d["Wd_q"].shape) == (128, 96)
+    assert tuple(d["Wd_q"].shape) == (96, 128)
     assert d["s_A"].dtype.itemsize == 2
 
 
