@@ -1,0 +1,16 @@
+"""B200 (sm_100a) low-rank decode library: Python binding of include/lr.h.
+
+The compute path is the CUDA shared library ``liblr_decode.so`` (built by
+``python -m decode_lr_linear_b200.build``); this package only marshals
+arguments.  ``synth`` holds the seeded synthetic-input generators.
+"""
+from .ops import (  # noqa: F401
+    Factor, FfnWeights, LatentKv, workspace,
+    lr_linear, lr_linear_workspace_size, lr_linear_grouped, lr_linear_grouped_workspace_size,
+    lr_swiglu_ffn, lr_swiglu_ffn_workspace_size, lr_latent_kv_decode, lr_latent_kv_workspace_size,
+    lr_quantize_per_token, lr_workspace_init, lr_check_device_error,
+)
+from ._lib import LrError, load  # noqa: F401
+
+__all__ = [n for n in dir() if n.startswith("lr_")] + ["Factor", "FfnWeights", "LatentKv", "workspace", "LrError",
+                                                       "load"]

@@ -1,0 +1,357 @@
+// C ABI of the low-rank decode library: argument validation, workspace sizing
+// and dispatch to the sm_100a kernels.  Nothing here computes on the host.
+#include <algorithm>
+#include <cstdint>
+#include <cstring>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace lr {
+
+// The library's device error word: set by kernels whose bounded waits give up.
+__device__ int g_device_error = 0;
+
+int* device_error_word() {
+  static int* cache[64] = {nullptr};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  if (!cache[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) return nullptr;
+    cache[dev] = reinterpret_cast<int*>(p);
+  }
+  return cache[dev];
+}
+
+}  // namespace lr
+
+namespace {
+
+using namespace lr;
+
+constexpr int kMaxDevices = 64;
+
+int sm_count_current() {
+  static int cache[kMaxDevices] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;
+  if (cache[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    cache[dev] = n;
+  }
+  return cache[dev];
+}
+
+inline bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+inline lr_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? LR_OK : LR_ERR_CUDA; }
+
+
+// Shape/pointer checks common to every factor descriptor.
+lr_status_t check_factor(const lr_factor_desc_t* d) {
+  if (!d || !d->A || !d->B) return LR_ERR_INVALID_ARG;
+  if (d->d_in <= 0 || d->d_out <= 0 || d->rank <= 0) return LR_ERR_INVALID_ARG;
+  if (d->active_rank < 0 || d->active_rank > d->rank) return LR_ERR_INVALID_ARG;
+  if (d->w_dtype != LR_F32 && d->w_dtype != LR_BF16 && d->w_dtype != LR_I8) return LR_ERR_UNSUPPORTED;
+  if (d->w_dtype == LR_I8) {
+    if (!d->scale_A || !d->scale_B) return LR_ERR_INVALID_ARG;
+    if (d->scale_dtype != LR_F16 && d->scale_dtype != LR_F32) return LR_ERR_UNSUPPORTED;
+    if (!al16(d->scale_A) || !al16(d->scale_B)) return LR_ERR_MISALIGNED;
+  }
+  if ((d->d_in % 8) != 0 || (d->d_out % 8) != 0) return LR_ERR_UNSUPPORTED;
+  if (!al16(d->A) || !al16(d->B)) return LR_ERR_MISALIGNED;
+  return LR_OK;
+}
+
+inline int active(const lr_factor_desc_t* d) { return d->active_rank ? d->active_rank : d->rank; }
+
+size_t rank1_ws_bytes(const lr_factor_desc_t* descs, int n, int batch) {
+  const int chunk = std::min(batch, kMaxDecodeChunk);
+  size_t b = kTicketBytes;
+  for (int p = 0; p < n; ++p) b += round_up(size_t(chunk) * descs[p].d_out * 4, 256);
+  return b;
+}
+
+lr_status_t run_rank1(const lr_factor_desc_t* descs, int n, const void* x, int batch, void* const* ys, void* ws,
+                      size_t ws_bytes, cudaStream_t stream) {
+  const lr_dtype_t wt = descs[0].w_dtype;
+  const size_t xs = (wt == LR_F32) ? 4 : 2;
+  const size_t ysz = (wt == LR_F32) ? 4 : 2;
+  if (!ws) return LR_ERR_WORKSPACE;
+  if (ws_bytes < rank1_ws_bytes(descs, n, batch)) return LR_ERR_WORKSPACE;
+  if (!al16(ws)) return LR_ERR_MISALIGNED;
+  Rank1Params P;
+  std::memset(&P, 0, sizeof(P));
+  P.n_proj = n;
+  P.d_in = descs[0].d_in;
+  P.scale_f16 = descs[0].scale_dtype == LR_F16 ? 1 : 0;
+  P.ticket = reinterpret_cast<unsigned int*>(ws);
+  const int chunk = std::min(batch, kMaxDecodeChunk);
+  char* accp = reinterpret_cast<char*>(ws) + kTicketBytes;
+  int row = 0;
+  for (int p = 0; p < n; ++p) {
+    Rank1Proj& pr = P.proj[p];
+    pr.A = descs[p].A;
+    pr.B = descs[p].B;
+    pr.sA = wt == LR_I8 ? descs[p].scale_A : nullptr;
+    pr.sB = wt == LR_I8 ? descs[p].scale_B : nullptr;
+    pr.acc = reinterpret_cast<float*>(accp);
+    accp += round_up(size_t(chunk) * descs[p].d_out * 4, 256);
+    pr.d_out = descs[p].d_out;
+    pr.rows = active(&descs[p]);
+    pr.row_begin = row;
+    row += pr.rows;
+  }
+  P.total_rows = row;
+  const int sms = sm_count_current();
+  for (int b0 = 0; b0 < batch; b0 += kMaxDecodeChunk) {
+    P.nb = std::min(kMaxDecodeChunk, batch - b0);
+    P.x = reinterpret_cast<const char*>(x) + size_t(b0) * P.d_in * xs;
+    for (int p = 0; p < n; ++p)
+      P.proj[p].y = reinterpret_cast<char*>(ys[p]) + size_t(b0) * descs[p].d_out * ysz;
+    cudaError_t e = launch_lr_rank1(P, wt, sms, stream);
+    if (e != cudaSuccess) return LR_ERR_CUDA;
+  }
+  return LR_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+lr_status_t lr_linear_workspace_size(const lr_factor_desc_t* desc, int batch, int w8a8, size_t* bytes) {
+  if (!bytes) return LR_ERR_INVALID_ARG;
+  lr_status_t st = check_factor(desc);
+  if (st != LR_OK) return st;
+  if (batch < 1) return LR_ERR_INVALID_ARG;
+  if (w8a8) {
+    if (desc->w_dtype != LR_I8) return LR_ERR_UNSUPPORTED;
+    *bytes = w8a8_workspace_bytes(batch, active(desc));
+  } else {
+    *bytes = rank1_ws_bytes(desc, 1, batch);
+  }
+  return LR_OK;
+}
+
+lr_status_t lr_linear(const lr_factor_desc_t* desc, const void* x, const float* x_scale, int batch, void* y,
+                      void* ws, size_t ws_bytes, lr_stream_t stream) {
+  lr_status_t st = check_factor(desc);
+  if (st != LR_OK) return st;
+  if (!x || !y || batch < 1) return LR_ERR_INVALID_ARG;
+  if (!al16(x) || !al16(y)) return LR_ERR_MISALIGNED;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (x_scale) {
+    if (desc->w_dtype != LR_I8 || desc->scale_dtype != LR_F32) return LR_ERR_UNSUPPORTED;
+    if (!al16(x_scale)) return LR_ERR_MISALIGNED;
+    if ((desc->d_in % 16) != 0 || (desc->d_out % 16) != 0) return LR_ERR_UNSUPPORTED;
+    if (!ws) return LR_ERR_WORKSPACE;
+    const int r = active(desc);
+    if (ws_bytes < w8a8_workspace_bytes(batch, r)) return LR_ERR_WORKSPACE;
+    if (!al16(ws)) return LR_ERR_MISALIGNED;
+    W8A8Params P;
+    std::memset(&P, 0, sizeof(P));
+    P.T = batch; P.d_in = desc->d_in; P.d_out = desc->d_out; P.rank = r;
+    P.xq = reinterpret_cast<const int8_t*>(x); P.sx = x_scale;
+    P.Aq = reinterpret_cast<const int8_t*>(desc->A); P.sA = reinterpret_cast<const float*>(desc->scale_A);
+    P.Bq = reinterpret_cast<const int8_t*>(desc->B); P.sB = reinterpret_cast<const float*>(desc->scale_B);
+    P.y = y;
+    char* w = reinterpret_cast<char*>(ws);
+    P.rank_pad = int(round_up(size_t(r), 128));
+    P.z = reinterpret_cast<float*>(w);
+    w += round_up(size_t(batch) * r * 4, 256);
+    P.zq = reinterpret_cast<int8_t*>(w);
+    w += round_up(size_t(round_up(batch, 128)) * P.rank_pad, 256);
+    P.sz = reinterpret_cast<float*>(w);
+    P.err = device_error_word();
+    return from_cuda(launch_w8a8(P, sm_count_current(), s));
+  }
+  void* ys[1] = {y};
+  return run_rank1(desc, 1, x, batch, ys, ws, ws_bytes, s);
+}
+
+lr_status_t lr_linear_grouped_workspace_size(const lr_factor_desc_t* descs, int n, int batch, size_t* bytes) {
+  if (!bytes || !descs || n < 1 || n > LR_MAX_GROUP || batch < 1) return LR_ERR_INVALID_ARG;
+  for (int p = 0; p < n; ++p) {
+    lr_status_t st = check_factor(&descs[p]);
+    if (st != LR_OK) return st;
+  }
+  *bytes = rank1_ws_bytes(descs, n, batch);
+  return LR_OK;
+}
+
+lr_status_t lr_linear_grouped(const lr_factor_desc_t* descs, int n, const void* x, int batch, void* const* ys,
+                              void* ws, size_t ws_bytes, lr_stream_t stream) {
+  if (!descs || n < 1 || n > LR_MAX_GROUP || !x || !ys || batch < 1) return LR_ERR_INVALID_ARG;
+  for (int p = 0; p < n; ++p) {
+    lr_status_t st = check_factor(&descs[p]);
+    if (st != LR_OK) return st;
+    if (!ys[p]) return LR_ERR_INVALID_ARG;
+    if (!al16(ys[p])) return LR_ERR_MISALIGNED;
+    if (descs[p].d_in != descs[0].d_in || descs[p].w_dtype != descs[0].w_dtype) return LR_ERR_INVALID_ARG;
+    if (descs[0].w_dtype == LR_I8 && descs[p].scale_dtype != descs[0].scale_dtype) return LR_ERR_INVALID_ARG;
+  }
+  if (!al16(x)) return LR_ERR_MISALIGNED;
+  return run_rank1(descs, n, x, batch, ys, ws, ws_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+// --------------------------------------------------------------------------
+
+static lr_status_t check_ffn(const lr_ffn_desc_t* d) {
+  if (!d) return LR_ERR_INVALID_ARG;
+  if (d->hidden <= 0 || d->inter <= 0 || d->n_lr < 0 || d->n_lr > d->inter) return LR_ERR_INVALID_ARG;
+  if (d->n_lr > 0 && (d->rank <= 0 || !d->A || !d->s_A || !d->B || !d->s_B)) return LR_ERR_INVALID_ARG;
+  if (d->inter > d->n_lr && (!d->D || !d->s_D)) return LR_ERR_INVALID_ARG;
+  if (!d->W_down || !d->s_down) return LR_ERR_INVALID_ARG;
+  if (d->scale_dtype != LR_F16 && d->scale_dtype != LR_F32) return LR_ERR_UNSUPPORTED;
+  if ((d->hidden % 16) != 0 || (d->n_lr % 4) != 0) return LR_ERR_UNSUPPORTED;
+  const void* ptrs[] = {d->A, d->s_A, d->B, d->s_B, d->D, d->s_D, d->W_down, d->s_down};
+  for (const void* p : ptrs)
+    if (p && !al16(p)) return LR_ERR_MISALIGNED;
+  return LR_OK;
+}
+
+static size_t ffn_ws_bytes(const lr_ffn_desc_t* d, int batch) {
+  const int chunk = std::min(batch, kMaxDecodeChunk);
+  const int n_dense = d->inter - d->n_lr;
+  return kTicketBytes + round_up(size_t(chunk) * 2 * d->n_lr * 4, 256) + round_up(size_t(chunk) * n_dense * 4, 256) +
+         round_up(size_t(chunk) * d->hidden * 4, 256);
+}
+
+lr_status_t lr_swiglu_ffn_workspace_size(const lr_ffn_desc_t* desc, int batch, size_t* bytes) {
+  if (!bytes || batch < 1) return LR_ERR_INVALID_ARG;
+  lr_status_t st = check_ffn(desc);
+  if (st != LR_OK) return st;
+  *bytes = ffn_ws_bytes(desc, batch);
+  return LR_OK;
+}
+
+lr_status_t lr_swiglu_ffn(const lr_ffn_desc_t* d, const void* x, int batch, void* y, void* ws, size_t ws_bytes,
+                          lr_stream_t stream) {
+  lr_status_t st = check_ffn(d);
+  if (st != LR_OK) return st;
+  if (!x || !y || batch < 1) return LR_ERR_INVALID_ARG;
+  if (!al16(x) || !al16(y)) return LR_ERR_MISALIGNED;
+  if (!ws || ws_bytes < ffn_ws_bytes(d, batch)) return LR_ERR_WORKSPACE;
+  if (!al16(ws)) return LR_ERR_MISALIGNED;
+  const int chunk = std::min(batch, kMaxDecodeChunk);
+  FfnParams P;
+  std::memset(&P, 0, sizeof(P));
+  P.hidden = d->hidden; P.inter = d->inter; P.n_lr = d->n_lr; P.n_dense = d->inter - d->n_lr; P.rank = d->rank;
+  P.scale_f16 = d->scale_dtype == LR_F16 ? 1 : 0;
+  P.A = d->A; P.sA = d->s_A; P.B = d->B; P.sB = d->s_B; P.D = d->D; P.sD = d->s_D; P.Wd = d->W_down; P.sd = d->s_down;
+  char* w = reinterpret_cast<char*>(ws);
+  P.ticket = reinterpret_cast<unsigned int*>(w);
+  w += kTicketBytes;
+  P.gu_acc = reinterpret_cast<float*>(w);
+  w += round_up(size_t(chunk) * 2 * d->n_lr * 4, 256);
+  P.h_dense = reinterpret_cast<float*>(w);
+  w += round_up(size_t(chunk) * P.n_dense * 4, 256);
+  P.y_acc = reinterpret_cast<float*>(w);
+  const int sms = sm_count_current();
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  for (int b0 = 0; b0 < batch; b0 += kMaxDecodeChunk) {
+    P.nb = std::min(kMaxDecodeChunk, batch - b0);
+    P.x = reinterpret_cast<const char*>(x) + size_t(b0) * d->hidden * 2;
+    P.y = reinterpret_cast<char*>(y) + size_t(b0) * d->hidden * 2;
+    if (launch_ffn(P, sms, s) != cudaSuccess) return LR_ERR_CUDA;
+  }
+  return LR_OK;
+}
+
+// --------------------------------------------------------------------------
+
+static lr_status_t check_kv(const lr_latent_kv_desc_t* d, int* split) {
+  if (!d || !d->B_K || !d->B_V) return LR_ERR_INVALID_ARG;
+  if (d->batch <= 0 || d->heads <= 0 || d->max_ctx <= 0 || d->rank <= 0 || d->head_dim <= 0) return LR_ERR_INVALID_ARG;
+  if (d->rank != 32 || d->head_dim != 128) return LR_ERR_UNSUPPORTED;
+  if (d->mode != LR_KV_ABSORBED) return LR_ERR_UNSUPPORTED;
+  if (d->split_tokens < 0 || (d->split_tokens % 64) != 0 || d->split_tokens > 1024) return LR_ERR_INVALID_ARG;
+  if (d->heads > 65535 || d->batch > 65535) return LR_ERR_UNSUPPORTED;
+  if (!al16(d->B_K) || !al16(d->B_V)) return LR_ERR_MISALIGNED;
+  int t = d->split_tokens;
+  if (t == 0) t = d->max_ctx > 8192 ? 512 : 256;
+  *split = t;
+  return LR_OK;
+}
+
+lr_status_t lr_latent_kv_workspace_size(const lr_latent_kv_desc_t* d, size_t* bytes) {
+  int t = 0;
+  if (!bytes) return LR_ERR_INVALID_ARG;
+  lr_status_t st = check_kv(d, &t);
+  if (st != LR_OK) return st;
+  const size_t ns = (size_t(d->max_ctx) + t - 1) / t;
+  *bytes = size_t(d->batch) * d->heads * ns * (d->rank + 2) * 4;
+  return LR_OK;
+}
+
+lr_status_t lr_latent_kv_decode(const lr_latent_kv_desc_t* d, const void* q, const void* C_K, const void* C_V,
+                                const int* seq_lens, void* out, void* ws, size_t ws_bytes, lr_stream_t stream) {
+  int t = 0;
+  lr_status_t st = check_kv(d, &t);
+  if (st != LR_OK) return st;
+  if (!q || !C_K || !C_V || !seq_lens || !out) return LR_ERR_INVALID_ARG;
+  if (!al16(q) || !al16(C_K) || !al16(C_V) || !al16(seq_lens) || !al16(out)) return LR_ERR_MISALIGNED;
+  size_t need = 0;
+  lr_latent_kv_workspace_size(d, &need);
+  if (!ws || ws_bytes < need) return LR_ERR_WORKSPACE;
+  if (!al16(ws)) return LR_ERR_MISALIGNED;
+  LatentKvParams P;
+  std::memset(&P, 0, sizeof(P));
+  P.batch = d->batch; P.heads = d->heads; P.head_dim = d->head_dim; P.rank = d->rank; P.max_ctx = d->max_ctx;
+  P.split_tokens = t; P.n_splits = (d->max_ctx + t - 1) / t; P.scale = d->scale;
+  P.q = q; P.CK = C_K; P.CV = C_V; P.BK = d->B_K; P.BV = d->B_V; P.seq_lens = seq_lens; P.out = out;
+  P.partial = reinterpret_cast<float*>(ws);
+  P.mode = d->mode;
+  P.err = device_error_word();
+  return from_cuda(launch_latent_kv(P, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+// --------------------------------------------------------------------------
+
+lr_status_t lr_quantize_per_token(const void* x, int rows, int cols, int8_t* x_q, float* s, lr_stream_t stream) {
+  if (!x || !x_q || !s || rows < 1 || cols < 1) return LR_ERR_INVALID_ARG;
+  if ((cols % 16) != 0 || cols > 49152) return LR_ERR_UNSUPPORTED;
+  if (!al16(x) || !al16(x_q) || !al16(s)) return LR_ERR_MISALIGNED;
+  return from_cuda(launch_quantize_per_token(x, rows, cols, x_q, s, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+lr_status_t lr_workspace_init(void* ws, size_t ws_bytes, lr_stream_t stream) {
+  if (!ws) return LR_ERR_INVALID_ARG;
+  if (!al16(ws)) return LR_ERR_MISALIGNED;
+  return from_cuda(cudaMemsetAsync(ws, 0, ws_bytes, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+lr_status_t lr_check_device_error(lr_stream_t stream, int* err) {
+  if (!err) return LR_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return LR_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, lr::g_device_error, sizeof(int)) != cudaSuccess) return LR_ERR_CUDA;
+  *err = v;
+  if (v != 0) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(lr::g_device_error, &zero, sizeof(int)) != cudaSuccess) return LR_ERR_CUDA;
+    return LR_ERR_DEVICE_TIMEOUT;
+  }
+  return LR_OK;
+}
+
+const char* lr_status_string(lr_status_t s) {
+  switch (s) {
+    case LR_OK: return "ok";
+    case LR_ERR_INVALID_ARG: return "invalid argument";
+    case LR_ERR_UNSUPPORTED: return "unsupported dtype or shape";
+    case LR_ERR_MISALIGNED: return "device pointer not 16-byte aligned";
+    case LR_ERR_WORKSPACE: return "workspace missing or too small";
+    case LR_ERR_CUDA: return "CUDA error";
+    case LR_ERR_DEVICE_TIMEOUT: return "a kernel gave up a bounded wait";
+  }
+  return "unknown status";
+}
+
+int lr_version(void) { return 100; }
+
+}  // extern "C"

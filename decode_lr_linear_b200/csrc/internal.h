@@ -1,0 +1,102 @@
+// Internal launch interface between the C ABI (api.cu) and the kernel files.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/lr.h"
+
+namespace lr {
+
+// Device address of the library's error word on the current device.
+int* device_error_word();
+
+constexpr int kMaxGroup = LR_MAX_GROUP;
+
+// Workspace element shared by the split-reduction kernels: one arrival counter
+// padded to 256 bytes, followed by fp32 accumulators.
+constexpr size_t kTicketBytes = 256;
+
+// Batch rows handled by one launch of the CUDA-core decode kernels.
+constexpr int kMaxDecodeChunk = 8;
+
+struct Rank1Proj {
+  const void* A;      // [rank, d_in]
+  const void* B;      // [rank, d_out]
+  const void* sA;     // int8: [rank]
+  const void* sB;     // int8: [d_out]
+  float* acc;         // [chunk, d_out] fp32 accumulator (zero on entry and exit)
+  void* y;            // [batch, d_out] output (f32 or bf16), already offset to the chunk
+  int d_out;
+  int rows;           // active latent rows
+  int row_begin;      // first global latent index of this projection
+};
+
+struct Rank1Params {
+  Rank1Proj proj[kMaxGroup];
+  int n_proj;
+  int d_in;
+  int nb;             // batch rows in this launch (<= kMaxDecodeChunk)
+  int total_rows;
+  const void* x;      // [nb, d_in], already offset to the chunk
+  unsigned int* ticket;
+  int scale_f16;
+};
+
+// y = (x A) B for up to kMaxGroup projections sharing x; weight-only paths.
+cudaError_t launch_lr_rank1(const Rank1Params& p, lr_dtype_t w_dtype, int sm_count, cudaStream_t s);
+
+struct FfnParams {
+  int hidden, inter, n_lr, n_dense, rank;
+  int nb;
+  int scale_f16;
+  const int8_t* A; const void* sA;
+  const int8_t* B; const void* sB;
+  const int8_t* D; const void* sD;
+  const int8_t* Wd; const void* sd;
+  const void* x;      // bf16 [nb, hidden]
+  void* y;            // bf16 [nb, hidden]
+  float* gu_acc;      // [nb, 2*n_lr]  (zero on entry and exit)
+  float* h_dense;     // [nb, n_dense]
+  float* y_acc;       // [nb, hidden]  (zero on entry and exit)
+  unsigned int* ticket;
+};
+
+cudaError_t launch_ffn(const FfnParams& p, int sm_count, cudaStream_t s);
+
+struct LatentKvParams {
+  int batch, heads, head_dim, rank, max_ctx;
+  int split_tokens, n_splits;
+  float scale;
+  const void* q; const void* CK; const void* CV;
+  const void* BK; const void* BV;
+  const int* seq_lens;
+  void* out;
+  float* partial;     // [batch, heads, n_splits, rank + 2]
+  int mode;
+  int* err;           // device error word
+};
+
+cudaError_t launch_latent_kv(const LatentKvParams& p, cudaStream_t s);
+
+cudaError_t launch_quantize_per_token(const void* x, int rows, int cols, int8_t* xq, float* s,
+                                      cudaStream_t st);
+
+struct W8A8Params {
+  int T, d_in, d_out, rank;
+  const int8_t* xq; const float* sx;
+  const int8_t* Aq; const float* sA;
+  const int8_t* Bq; const float* sB;
+  void* y;            // bf16 [T, d_out]
+  float* z;           // [T, rank] fp32 workspace
+  int8_t* zq;         // [T, rank_pad] int8 workspace
+  float* sz;          // [T]
+  int rank_pad;
+  int* err;           // device error word
+};
+
+size_t w8a8_workspace_bytes(int T, int rank);
+cudaError_t launch_w8a8(const W8A8Params& p, int sm_count, cudaStream_t s);
+
+}  // namespace lr

@@ -1,0 +1,288 @@
+/*
+ * lr.h -- C ABI of the B200 (sm_100a) low-rank decode library.
+ *
+ * The library executes truncated-SVD-factorised layers at decode time without
+ * ever forming the full weight: a weight W (d_in x d_out, y = x W) is replaced
+ * by factors A (d_in x r) and B (r x d_out) and the layer computes
+ * y = (x A) B.  Three families of calls are provided:
+ *   - lr_linear / lr_linear_grouped: factorised linears (Q/K/V/O projections;
+ *     the grouped form shares one input between several projections),
+ *   - lr_swiglu_ffn: the hybrid SwiGLU FFN whose gate/up channels are split
+ *     into SVD-compressed channels (sharing one latent) and dense channels,
+ *     int8 round-to-nearest weights with per-output-channel scales,
+ *   - lr_latent_kv_decode: single-query flash-decoding attention over
+ *     per-head rank-r latent K/V caches,
+ * plus per-token int8 quantisation for the W8A8 prefill path.
+ *
+ * Conventions shared by every call
+ *   - All tensor pointers are DEVICE pointers unless a parameter says "host".
+ *     The caller owns every buffer, including the workspace; the library never
+ *     allocates, frees or synchronises (except lr_check_device_error, whose job
+ *     is to synchronise).  Descriptors are read during the call and not kept.
+ *   - Tensors are dense and row-major; every device pointer must be 16-byte
+ *     aligned (LR_ERR_MISALIGNED otherwise).
+ *   - Every call is asynchronous on the given stream (NULL = legacy default).
+ *   - Arguments are validated before any launch; nothing is launched when a
+ *     call returns an error.  A failed kernel launch returns LR_ERR_CUDA.
+ *   - There is no host fallback: every step runs in this library's kernels.
+ *   - Workspaces: a call that takes one needs at least the bytes reported by
+ *     its *_workspace_size function.  A workspace must be zero-filled once
+ *     (lr_workspace_init) before its first use; every call leaves it zeroed
+ *     again on completion.  Two calls that may run concurrently must not share
+ *     a workspace.
+ *
+ * Factor storage ("latent-major"): both factors hold one contiguous row per
+ * latent component j,
+ *     A_store [rank, d_in]   row j = column j of A,
+ *     B_store [rank, d_out]  row j = row j of B,
+ * so y = sum_j (x . A_store[j]) B_store[j].  The leading rows are the leading
+ * singular components, so a shorter active rank uses a prefix of both.
+ */
+#ifndef LR_DECODE_H
+#define LR_DECODE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define LR_API __attribute__((visibility("default")))
+#else
+#define LR_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t. */
+typedef struct CUstream_st* lr_stream_t;
+
+typedef enum {
+  LR_OK = 0,
+  LR_ERR_INVALID_ARG = 1,    /* null pointer, non-positive size, inconsistent shape */
+  LR_ERR_UNSUPPORTED = 2,    /* valid but not implemented combination (dtype, shape) */
+  LR_ERR_MISALIGNED = 3,     /* a device pointer is not 16-byte aligned */
+  LR_ERR_WORKSPACE = 4,      /* workspace missing or smaller than required */
+  LR_ERR_CUDA = 5,           /* a CUDA runtime call or kernel launch failed */
+  LR_ERR_DEVICE_TIMEOUT = 6  /* a kernel gave up a bounded wait (see lr_check_device_error) */
+} lr_status_t;
+
+typedef enum { LR_F32 = 0, LR_BF16 = 1, LR_F16 = 2, LR_I8 = 3, LR_I32 = 4 } lr_dtype_t;
+
+/* ------------------------------------------------------------------------ */
+/* Factorised linear                                                        */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * One truncated-SVD factor pair.  The factor pair replaces the weight
+ * (SAES-SVD technical summary, CEALC: the local term || A_l B_l X_l - W_l X_l ||;
+ * WSVD "Fine-Grained Per-Head SVD": W_Kh = A_Kh B_Kh); per-projection ranks are
+ * free (LASER "Loss-Aware Cross-Layer Rank Allocation", FLRC "Fisher-based
+ * layer-wise rank allocation": non-uniform ranks across layers and projections).
+ *
+ *   A            [rank, d_in]  latent-major first factor (see file header)
+ *   B            [rank, d_out] latent-major second factor
+ *   rank         stored rank (rows of A and B), >= 1
+ *   active_rank  0 (or rank): use every component; 1..rank-1: use only the
+ *                first active_rank components (FLRC "progressive low-rank
+ *                decoding", r(t) <= r); bytes read scale with it
+ *   w_dtype      LR_F32, LR_BF16 or LR_I8
+ *   scale_A      LR_I8 only: [rank] scale of row j of A (per latent channel)
+ *   scale_B      LR_I8 only: [d_out] scale of column k of B (per output channel)
+ *   scale_dtype  LR_I8 only: LR_F16 or LR_F32
+ * An int8 factor dequantises as A[i][j] = A_store[j][i] * scale_A[j] and
+ * B[j][k] = B_store[j][k] * scale_B[k] (LASER "Hybrid SVD-Quantization for
+ * FFNs": RTN quantisation of the factors).
+ */
+typedef struct lr_factor_desc {
+  const void* A;
+  const void* B;
+  int d_in;
+  int d_out;
+  int rank;
+  int active_rank;
+  lr_dtype_t w_dtype;
+  lr_dtype_t scale_dtype;
+  const void* scale_A;
+  const void* scale_B;
+} lr_factor_desc_t;
+
+/*
+ * y = (x A) B for `batch` tokens (rows of x).
+ *
+ * Weight-only paths (x_scale == NULL):
+ *   w_dtype LR_F32:  x f32 [batch, d_in]  -> y f32 [batch, d_out]
+ *   w_dtype LR_BF16: x bf16 [batch, d_in] -> y bf16 [batch, d_out]
+ *   w_dtype LR_I8:   x bf16 [batch, d_in] -> y bf16 [batch, d_out]
+ *   accumulation in fp32; the r-dim latent z = x A stays on chip in fp32.
+ * W8A8 path (x_scale != NULL; w_dtype LR_I8, scale_dtype LR_F32):
+ *   x int8 [batch, d_in] with per-token scales x_scale f32 [batch] (from
+ *   lr_quantize_per_token), y bf16 [batch, d_out]; int8 x int8 -> int32 tensor
+ *   core products; the latent is requantised per token in between:
+ *     acc1 = x_q A_q (int32);  z = fp32(fp32(acc1 * x_scale[t]) * scale_A[j])
+ *     s_z  = max_j |z| / 127;  z_q = clamp(rint(z / s_z), -127, 127)
+ *     acc2 = z_q B_q (int32);  y = bf16(fp32(fp32(acc2 * s_z[t]) * scale_B[k]))
+ *   (LASER results, W8A8 setting; WSVD "Quantization-Aware Training",
+ *   weights and activations quantised, e.g. W8A8).
+ * ws: workspace of at least lr_linear_workspace_size(...) bytes.
+ * Errors: LR_ERR_INVALID_ARG (null pointers, batch < 1, bad shape or rank),
+ * LR_ERR_UNSUPPORTED (dtype combination), LR_ERR_MISALIGNED,
+ * LR_ERR_WORKSPACE, LR_ERR_CUDA.
+ */
+LR_API lr_status_t lr_linear(const lr_factor_desc_t* desc, const void* x, const float* x_scale, int batch,
+                      void* y, void* ws, size_t ws_bytes, lr_stream_t stream);
+
+LR_API lr_status_t lr_linear_workspace_size(const lr_factor_desc_t* desc, int batch, int w8a8,
+                                     size_t* bytes);
+
+/*
+ * Several factorised linears that share one input x (e.g. Q, K and V), in one
+ * launch: y_p = (x A_p) B_p for p < n (1 <= n <= LR_MAX_GROUP).  All
+ * descriptors must have the same d_in, w_dtype and scale_dtype; ranks and
+ * d_out may differ.  `descs` is a host array of n descriptors and `ys` a host
+ * array of n device output pointers.  Weight-only paths only (batch 1..8).
+ * LASER "System Implementation" fuses the input projection with the latent
+ * activation; sharing x across Q/K/V reads it once.
+ */
+#define LR_MAX_GROUP 4
+LR_API lr_status_t lr_linear_grouped(const lr_factor_desc_t* descs, int n, const void* x, int batch,
+                              void* const* ys, void* ws, size_t ws_bytes, lr_stream_t stream);
+
+LR_API lr_status_t lr_linear_grouped_workspace_size(const lr_factor_desc_t* descs, int n, int batch,
+                                             size_t* bytes);
+
+/* ------------------------------------------------------------------------ */
+/* Hybrid SwiGLU FFN                                                        */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * LASER "Hybrid SVD-Quantization for FFNs": the first n_lr hidden channels are
+ * low-rank through one latent of width `rank` shared by gate and up; the other
+ * n_dense = inter - n_lr channels are dense; every matrix is int8 RTN with one
+ * scale per output channel; an orthogonal rotation between the factors is
+ * folded offline (A' = A R, B' = R^T B), so the kernels never see it.
+ *
+ *   A      [rank, hidden]        int8, s_A [rank]        latent-major A'
+ *   B      [rank, 2*n_lr]        int8, s_B [2*n_lr]      latent-major B'; columns
+ *                                                        gate_0, up_0, gate_1, up_1, ...
+ *   D      [2*n_dense, hidden]   int8, s_D [2*n_dense]   dense gate/up, output-major,
+ *                                                        rows gate_0, up_0, gate_1, ...
+ *   W_down [inter, hidden]       int8, s_down [hidden]   input-major down projection,
+ *                                                        rows in [S; D] channel order
+ *   scale_dtype  LR_F16 or LR_F32 for all scales.
+ * Computes, per token (LASER "System Implementation": fused input projection,
+ * latent activation, SwiGLU and dequantisation):
+ *   z = x A';  [g_S, u_S] = z B';  [g_D, u_D] = x D';
+ *   h = [silu(g_S) u_S, silu(g_D) u_D];  y = h W_down;  silu(t) = t / (1 + e^-t).
+ */
+typedef struct lr_ffn_desc {
+  int hidden;
+  int inter;
+  int n_lr;
+  int rank;
+  lr_dtype_t scale_dtype;
+  const int8_t* A;
+  const void* s_A;
+  const int8_t* B;
+  const void* s_B;
+  const int8_t* D;
+  const void* s_D;
+  const int8_t* W_down;
+  const void* s_down;
+} lr_ffn_desc_t;
+
+/* x bf16 [batch, hidden] -> y bf16 [batch, hidden]; batch 1..8.
+ * Errors as lr_linear. */
+LR_API lr_status_t lr_swiglu_ffn(const lr_ffn_desc_t* desc, const void* x, int batch, void* y, void* ws,
+                          size_t ws_bytes, lr_stream_t stream);
+
+LR_API lr_status_t lr_swiglu_ffn_workspace_size(const lr_ffn_desc_t* desc, int batch, size_t* bytes);
+
+/* ------------------------------------------------------------------------ */
+/* Per-head latent K/V decode attention                                     */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * WSVD "Fine-Grained Per-Head SVD": the key projection of head h is factored
+ * W_Kh = A_Kh B_Kh at rank r and the cache keeps the per-head latent C_K,h
+ * (likewise for values); WSVD "Quantization-Aware Training (QAT) en Fused
+ * Kernel": K and V are reconstructed inside the flash-decoding pipeline and
+ * never written to global memory.
+ *
+ *   B_K, B_V  [heads, rank, head_dim] bf16: key t of head h is
+ *             K_t = C_K[b,h,t,:] B_K[h], value V_t = C_V[b,h,t,:] B_V[h]
+ *   scale     softmax scale (1/sqrt(head_dim) for standard attention)
+ *   mode      LR_KV_ABSORBED: scores s_t = C_K[t] (B_K q) * scale, latent
+ *             values accumulated and reconstructed once per split;
+ *             LR_KV_RECONSTRUCT: each tile K_tile = C_K_tile B_K is built on
+ *             chip (tensor cores) and scored against q
+ *   split_tokens  tokens per split-K chunk (multiple of 64), 0 = library choice
+ * Supported: rank 32, head_dim 128.
+ */
+#define LR_KV_ABSORBED 0
+#define LR_KV_RECONSTRUCT 1
+typedef struct lr_latent_kv_desc {
+  int batch;
+  int heads;
+  int head_dim;
+  int rank;
+  int max_ctx;
+  float scale;
+  const void* B_K;
+  const void* B_V;
+  int mode;
+  int split_tokens;
+} lr_latent_kv_desc_t;
+
+/*
+ * q bf16 [batch, heads, head_dim]; C_K, C_V bf16 [batch, heads, max_ctx, rank];
+ * seq_lens int32 [batch] (device) with 0 <= seq_lens[b] <= max_ctx (values are
+ * clamped into that range; a length of 0 yields a zero output row);
+ * out bf16 [batch, heads, head_dim].  The single query of each sequence attends
+ * to cached positions 0 .. seq_lens[b]-1.
+ */
+LR_API lr_status_t lr_latent_kv_decode(const lr_latent_kv_desc_t* desc, const void* q, const void* C_K,
+                                const void* C_V, const int* seq_lens, void* out, void* ws,
+                                size_t ws_bytes, lr_stream_t stream);
+
+LR_API lr_status_t lr_latent_kv_workspace_size(const lr_latent_kv_desc_t* desc, size_t* bytes);
+
+/* ------------------------------------------------------------------------ */
+/* W8A8 helpers                                                             */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * Per-token symmetric int8 quantisation (LASER results, W8A8 setting):
+ * s[t] = fp32(max_i |x[t,i]| / 127) (1 when the row is all zero),
+ * x_q[t,i] = clamp(rint(x[t,i] / s[t]), -127, 127), division in IEEE fp32,
+ * rint ties to even.  x bf16 [rows, cols] -> x_q int8 [rows, cols], s f32 [rows].
+ */
+LR_API lr_status_t lr_quantize_per_token(const void* x, int rows, int cols, int8_t* x_q, float* s,
+                                  lr_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* Utilities                                                                */
+/* ------------------------------------------------------------------------ */
+
+/* Zero-fill a workspace (cudaMemsetAsync on `stream`). */
+LR_API lr_status_t lr_workspace_init(void* ws, size_t ws_bytes, lr_stream_t stream);
+
+/*
+ * Synchronise `stream`, then read and clear the library's device error word on
+ * the current device.  *err = 0 when no kernel gave up a bounded wait since the
+ * last check; otherwise a nonzero code naming the wait.  Returns
+ * LR_ERR_DEVICE_TIMEOUT when *err != 0, LR_ERR_CUDA if synchronisation failed.
+ */
+LR_API lr_status_t lr_check_device_error(lr_stream_t stream, int* err);
+
+/* Static string for a status code. */
+LR_API const char* lr_status_string(lr_status_t status);
+
+/* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
+LR_API int lr_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LR_DECODE_H */

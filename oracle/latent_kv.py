@@ -25,23 +25,34 @@ def _softmax(s: np.ndarray) -> np.ndarray:
 
 
 def decode_head(q, CK, CV, BK, BV, n: int, scale: float) -> np.ndarray:
-    """One (batch, head): reconstruct K, V for the first n positions, then softmax attention."""
+    """One (batch, head): reconstruct K, V for the first n positions, then softmax attention.
+
+    An empty context (n = 0) has no softmax; the library's reading is a zero output.
+    """
+    if n <= 0:
+        return np.zeros(_f64(BV).shape[1])
     K = _f64(CK)[:n] @ _f64(BK)          # n x head_dim
     V = _f64(CV)[:n] @ _f64(BV)          # n x head_dim
     p = _softmax((K @ _f64(q)) * scale)  # n
     return p @ V
 
 
+def _pairs_and_lens(q, seq_lens, pairs):
+    seq_lens = np.asarray(seq_lens.cpu() if hasattr(seq_lens, "cpu") else seq_lens).astype(np.int64)
+    nb, nh = q.shape[0], q.shape[1]
+    todo = pairs if pairs is not None else [(b, h) for b in range(nb) for h in range(nh)]
+    return seq_lens, todo
+
+
 def latent_kv_decode(q, C_K, C_V, B_K, B_V, seq_lens, scale: float, pairs=None) -> np.ndarray:
     """o [batch, heads, head_dim] in float64 (reconstruct-then-attend form).
 
     ``pairs``: optional list of (b, h) to evaluate; other entries stay NaN.
+    Inputs are converted to float64 one (batch, head) at a time.
     """
-    q, C_K, C_V, B_K, B_V = _f64(q), _f64(C_K), _f64(C_V), _f64(B_K), _f64(B_V)
-    seq_lens = np.asarray(seq_lens.cpu() if hasattr(seq_lens, "cpu") else seq_lens).astype(np.int64)
+    seq_lens, todo = _pairs_and_lens(q, seq_lens, pairs)
     nb, nh, hd = q.shape
     out = np.full((nb, nh, hd), np.nan)
-    todo = pairs if pairs is not None else [(b, h) for b in range(nb) for h in range(nh)]
     for b, h in todo:
         out[b, h] = decode_head(q[b, h], C_K[b, h], C_V[b, h], B_K[h], B_V[h], int(seq_lens[b]), scale)
     return out
@@ -50,17 +61,17 @@ def latent_kv_decode(q, C_K, C_V, B_K, B_V, seq_lens, scale: float, pairs=None) 
 def decode_head_absorbed(q, CK, CV, BK, BV, n: int, scale: float) -> np.ndarray:
     """Same result with the factors moved onto the query and the output:
     s_t = C_K[t] (B_K q) * scale, acc = sum_t p_t C_V[t] (r-vector), o = acc B_V."""
+    if n <= 0:
+        return np.zeros(_f64(BV).shape[1])
     qt = _f64(BK) @ _f64(q)              # r
     p = _softmax((_f64(CK)[:n] @ qt) * scale)
     return (p @ _f64(CV)[:n]) @ _f64(BV)
 
 
 def latent_kv_decode_absorbed(q, C_K, C_V, B_K, B_V, seq_lens, scale: float, pairs=None) -> np.ndarray:
-    q, C_K, C_V, B_K, B_V = _f64(q), _f64(C_K), _f64(C_V), _f64(B_K), _f64(B_V)
-    seq_lens = np.asarray(seq_lens.cpu() if hasattr(seq_lens, "cpu") else seq_lens).astype(np.int64)
+    seq_lens, todo = _pairs_and_lens(q, seq_lens, pairs)
     nb, nh, hd = q.shape
     out = np.full((nb, nh, hd), np.nan)
-    todo = pairs if pairs is not None else [(b, h) for b in range(nb) for h in range(nh)]
     for b, h in todo:
         out[b, h] = decode_head_absorbed(q[b, h], C_K[b, h], C_V[b, h], B_K[h], B_V[h],
                                          int(seq_lens[b]), scale)

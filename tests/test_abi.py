@@ -1,0 +1,133 @@
+"""The C-ABI library loads, exports what include/lr.h declares, and validates
+arguments on the host (CPU only: no call here reaches a kernel launch)."""
+import ctypes
+
+import pytest
+
+from decode_lr_linear_b200 import _lib as L
+
+FAKE = 0x10000          # a 16-byte aligned non-null address (never dereferenced on the host)
+MIS = 0x10001           # a misaligned address
+
+
+@pytest.fixture(scope="module")
+def lib():
+    return L.load()
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = L.header_functions()
+    assert len(names) >= 13
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_status_strings(lib):
+    for s in range(7):
+        assert lib.lr_status_string(s)
+    assert lib.lr_version() >= 100
+
+
+def _desc(**kw):
+    d = dict(A=FAKE, B=FAKE, d_in=4096, d_out=4096, rank=1024, active_rank=0, w_dtype=L.LR_BF16,
+             scale_dtype=L.LR_F32, scale_A=None, scale_B=None)
+    d.update(kw)
+    return L.FactorDesc(**d)
+
+
+def _ws(lib, d, batch, w8a8=0):
+    n = ctypes.c_size_t(0)
+    st = lib.lr_linear_workspace_size(ctypes.byref(d), batch, w8a8, ctypes.byref(n))
+    return st, n.value
+
+
+def test_linear_workspace_sizes(lib):
+    st, n = _ws(lib, _desc(), 1)
+    assert st == L.LR_OK and n == 256 + 4096 * 4
+    st, n8 = _ws(lib, _desc(), 16)
+    assert st == L.LR_OK and n8 == 256 + 8 * 4096 * 4
+    st, _ = _ws(lib, _desc(w_dtype=L.LR_I8), 1)
+    assert st == L.LR_ERR_INVALID_ARG  # int8 needs scales
+    st, n = _ws(lib, _desc(w_dtype=L.LR_I8, scale_A=FAKE, scale_B=FAKE), 2048, 1)
+    assert st == L.LR_OK and n > 2048 * 1024
+
+
+def test_linear_validation(lib):
+    call = lambda d, x=FAKE, xs=None, b=1, y=FAKE, ws=FAKE, wsb=1 << 20: lib.lr_linear(  # noqa: E731
+        ctypes.byref(d) if d is not None else None, x, xs, b, y, ws, wsb, None)
+    assert call(None) == L.LR_ERR_INVALID_ARG
+    assert call(_desc(A=None)) == L.LR_ERR_INVALID_ARG
+    assert call(_desc(rank=0)) == L.LR_ERR_INVALID_ARG
+    assert call(_desc(active_rank=2000)) == L.LR_ERR_INVALID_ARG
+    assert call(_desc(d_in=4100)) == L.LR_ERR_UNSUPPORTED
+    assert call(_desc(w_dtype=L.LR_F16)) == L.LR_ERR_UNSUPPORTED
+    assert call(_desc(A=MIS)) == L.LR_ERR_MISALIGNED
+    assert call(_desc(), x=MIS) == L.LR_ERR_MISALIGNED
+    assert call(_desc(), b=0) == L.LR_ERR_INVALID_ARG
+    assert call(_desc(), wsb=16) == L.LR_ERR_WORKSPACE
+    assert call(_desc(), ws=None) == L.LR_ERR_WORKSPACE
+    assert call(_desc(), xs=FAKE) == L.LR_ERR_UNSUPPORTED  # W8A8 needs int8 weights
+    d8 = _desc(w_dtype=L.LR_I8, scale_A=FAKE, scale_B=FAKE, scale_dtype=L.LR_F16)
+    assert call(d8, xs=FAKE) == L.LR_ERR_UNSUPPORTED  # W8A8 needs fp32 scales
+
+
+def test_grouped_validation(lib):
+    arr = (L.FactorDesc * 3)(_desc(), _desc(d_in=2048), _desc())
+    ys = (ctypes.c_void_p * 3)(FAKE, FAKE, FAKE)
+    assert lib.lr_linear_grouped(arr, 3, FAKE, 1, ys, FAKE, 1 << 20, None) == L.LR_ERR_INVALID_ARG
+    arr = (L.FactorDesc * 5)(*[_desc()] * 5)
+    assert lib.lr_linear_grouped(arr, 5, FAKE, 1, ys, FAKE, 1 << 20, None) == L.LR_ERR_INVALID_ARG
+    arr = (L.FactorDesc * 3)(_desc(), _desc(d_out=1024), _desc(rank=512))
+    n = ctypes.c_size_t(0)
+    assert lib.lr_linear_grouped_workspace_size(arr, 3, 1, ctypes.byref(n)) == L.LR_OK
+    assert n.value == 256 + 4096 * 4 + 1024 * 4 + 4096 * 4
+
+
+def _ffn(**kw):
+    d = dict(hidden=4096, inter=11008, n_lr=8192, rank=1536, scale_dtype=L.LR_F16, A=FAKE, s_A=FAKE, B=FAKE,
+             s_B=FAKE, D=FAKE, s_D=FAKE, W_down=FAKE, s_down=FAKE)
+    d.update(kw)
+    return L.FfnDesc(**d)
+
+
+def test_ffn_validation_and_workspace(lib):
+    n = ctypes.c_size_t(0)
+    d = _ffn()
+    assert lib.lr_swiglu_ffn_workspace_size(ctypes.byref(d), 1, ctypes.byref(n)) == L.LR_OK
+    assert n.value == 256 + 16384 * 4 + 2816 * 4 + 4096 * 4
+    bad = _ffn(n_lr=12000)
+    assert lib.lr_swiglu_ffn(ctypes.byref(bad), FAKE, 1, FAKE, FAKE, 1 << 20, None) == L.LR_ERR_INVALID_ARG
+    bad = _ffn(hidden=4100)
+    assert lib.lr_swiglu_ffn(ctypes.byref(bad), FAKE, 1, FAKE, FAKE, 1 << 20, None) == L.LR_ERR_UNSUPPORTED
+    bad = _ffn(D=MIS)
+    assert lib.lr_swiglu_ffn(ctypes.byref(bad), FAKE, 1, FAKE, FAKE, 1 << 20, None) == L.LR_ERR_MISALIGNED
+    assert lib.lr_swiglu_ffn(ctypes.byref(d), FAKE, 1, FAKE, FAKE, 64, None) == L.LR_ERR_WORKSPACE
+    dense_only = _ffn(n_lr=0, A=None, s_A=None, B=None, s_B=None)
+    assert lib.lr_swiglu_ffn_workspace_size(ctypes.byref(dense_only), 1, ctypes.byref(n)) == L.LR_OK
+
+
+def _kv(**kw):
+    d = dict(batch=8, heads=32, head_dim=128, rank=32, max_ctx=4096, scale=128 ** -0.5, B_K=FAKE, B_V=FAKE,
+             mode=L.LR_KV_ABSORBED, split_tokens=0)
+    d.update(kw)
+    return L.LatentKvDesc(**d)
+
+
+def test_latent_kv_validation_and_workspace(lib):
+    n = ctypes.c_size_t(0)
+    d = _kv()
+    assert lib.lr_latent_kv_workspace_size(ctypes.byref(d), ctypes.byref(n)) == L.LR_OK
+    assert n.value == 8 * 32 * (4096 // 256) * 34 * 4
+    for bad, code in ((_kv(rank=16), L.LR_ERR_UNSUPPORTED), (_kv(head_dim=64), L.LR_ERR_UNSUPPORTED),
+                      (_kv(split_tokens=100), L.LR_ERR_INVALID_ARG), (_kv(batch=0), L.LR_ERR_INVALID_ARG),
+                      (_kv(B_K=MIS), L.LR_ERR_MISALIGNED)):
+        assert lib.lr_latent_kv_decode(ctypes.byref(bad), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1 << 30,
+                                       None) == code
+    assert lib.lr_latent_kv_decode(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 16,
+                                   None) == L.LR_ERR_WORKSPACE
+
+
+def test_quantize_validation(lib):
+    assert lib.lr_quantize_per_token(FAKE, 4, 100, FAKE, FAKE, None) == L.LR_ERR_UNSUPPORTED
+    assert lib.lr_quantize_per_token(None, 4, 128, FAKE, FAKE, None) == L.LR_ERR_INVALID_ARG
+    assert lib.lr_quantize_per_token(MIS, 4, 128, FAKE, FAKE, None) == L.LR_ERR_MISALIGNED
