@@ -1,5 +1,4 @@
 """GPU parity: hybrid SwiGLU FFN, latent-KV decode attention and per-token quantisation."""
-import math
 
 import numpy as np
 import pytest
@@ -113,4 +112,4 @@ def test_quantize_zero_row_and_ties(cuda_device):
     q_ref, s_ref = ow8.quantize_per_token(x)
     assert np.array_equal(xq.cpu().numpy(), q_ref) and np.array_equal(s.cpu().numpy(), s_ref)
     assert s[0].item() == 1.0 and int(xq[0].abs().max()) == 0
-    del math
+
