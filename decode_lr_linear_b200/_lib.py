@@ -20,6 +20,7 @@ LR_OK, LR_ERR_INVALID_ARG, LR_ERR_UNSUPPORTED, LR_ERR_MISALIGNED, LR_ERR_WORKSPA
 LR_F32, LR_BF16, LR_F16, LR_I8, LR_I32 = range(5)
 LR_MAX_GROUP = 4
 LR_KV_ABSORBED, LR_KV_RECONSTRUCT = 0, 1
+LR_NOALLOC_SCRATCH_BYTES = 1 << 20
 
 c_int, c_void_p, c_size_t, c_float = ctypes.c_int, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_float
 
@@ -46,6 +47,7 @@ P = ctypes.POINTER
 _SIGNATURES = {
     "lr_linear": (c_int, [P(FactorDesc), c_void_p, c_void_p, c_int, c_void_p, c_void_p, c_size_t, c_void_p]),
     "lr_linear_workspace_size": (c_int, [P(FactorDesc), c_int, c_int, P(c_size_t)]),
+    "lr_linear_noalloc": (c_int, [P(FactorDesc), c_void_p, c_int, c_void_p, c_void_p]),
     "lr_linear_grouped": (c_int, [P(FactorDesc), c_int, c_void_p, c_int, P(c_void_p), c_void_p, c_size_t,
                                   c_void_p]),
     "lr_linear_grouped_workspace_size": (c_int, [P(FactorDesc), c_int, c_int, P(c_size_t)]),

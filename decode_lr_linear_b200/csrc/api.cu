@@ -3,6 +3,7 @@
 #include <algorithm>
 #include <cstdint>
 #include <cstring>
+#include <mutex>
 
 #include "common.cuh"
 #include "internal.h"
@@ -118,9 +119,53 @@ lr_status_t run_rank1(const lr_factor_desc_t* descs, int n, const void* x, int b
   return LR_OK;
 }
 
+// ---------------------------------------------------------------------------
+// Scratch for lr_linear_noalloc: a fixed-size device array that belongs to the
+// library, so that callers who cannot allocate device memory still have the
+// split-reduction accumulators and arrival counter that lr_linear needs.  Host
+// code never uses the symbol itself as a pointer: its device address is looked
+// up once per device and cached.
+// ---------------------------------------------------------------------------
+__device__ __align__(256) unsigned char g_noalloc_scratch[LR_NOALLOC_SCRATCH_BYTES];
+
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kMaxDevices] = {nullptr};
+
+// Device address of the scratch on the current device; the first call on a
+// device looks it up and zero-fills it on `s` (the kernels leave it zeroed).
+lr_status_t noalloc_scratch(cudaStream_t s, void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return LR_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return LR_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return LR_ERR_CUDA;
+    if (cudaMemsetAsync(p, 0, LR_NOALLOC_SCRATCH_BYTES, s) != cudaSuccess) return LR_ERR_CUDA;
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return LR_OK;
+}
+
 }  // namespace
 
 extern "C" {
+
+lr_status_t lr_linear_noalloc(const lr_factor_desc_t* desc, const void* x, int batch, void* y,
+                              lr_stream_t stream) {
+  lr_status_t st = check_factor(desc);
+  if (st != LR_OK) return st;
+  if (!x || !y || batch < 1) return LR_ERR_INVALID_ARG;
+  if (!al16(x) || !al16(y)) return LR_ERR_MISALIGNED;
+  if (rank1_ws_bytes(desc, 1, batch) > size_t(LR_NOALLOC_SCRATCH_BYTES)) return LR_ERR_WORKSPACE;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  void* ws = nullptr;
+  st = noalloc_scratch(s, &ws);
+  if (st != LR_OK) return st;
+  void* ys[1] = {y};
+  return run_rank1(desc, 1, x, batch, ys, ws, LR_NOALLOC_SCRATCH_BYTES, s);
+}
 
 lr_status_t lr_linear_workspace_size(const lr_factor_desc_t* desc, int batch, int w8a8, size_t* bytes) {
   if (!bytes) return LR_ERR_INVALID_ARG;

@@ -151,6 +151,34 @@ LR_API lr_status_t lr_linear_grouped(const lr_factor_desc_t* descs, int n, const
 LR_API lr_status_t lr_linear_grouped_workspace_size(const lr_factor_desc_t* descs, int n, int batch,
                                              size_t* bytes);
 
+/*
+ * lr_linear without a caller-provided workspace (the pages have no
+ * counterpart to this call; it exists for integration).
+ *
+ * Some callers cannot allocate device memory at all: a plugin running inside
+ * a host framework that owns every device allocation, or a serving loop that
+ * has to stay allocation-free after start-up because cudaMalloc can
+ * synchronise the device and stall other work.  This call does what lr_linear
+ * does on its weight-only paths (x_scale must be absent: f32, bf16 and int8
+ * weights) but takes its scratch from a fixed array inside the library of
+ * LR_NOALLOC_SCRATCH_BYTES bytes per device, which every GPU that loads the
+ * library keeps until the process exits.  The caller still passes x and y.
+ *
+ *   - The scratch a call needs is 256 + 256-rounded(min(batch, 8) * d_out * 4)
+ *     bytes; a call that needs more returns LR_ERR_WORKSPACE and launches
+ *     nothing.
+ *   - The first call on a device looks the array up and zero-fills it on
+ *     `stream`; make that first call before any stream capture.  Every call
+ *     leaves the array zeroed again.
+ *   - All calls on one device share the array: calls that may overlap on the
+ *     GPU (different streams without ordering between them) race and give
+ *     wrong results.  Serialise them, or use lr_linear with your own workspace.
+ * It allocates nothing: no cudaMalloc, no cudaFree, no allocating library call.
+ */
+#define LR_NOALLOC_SCRATCH_BYTES (1u << 20)
+LR_API lr_status_t lr_linear_noalloc(const lr_factor_desc_t* desc, const void* x, int batch, void* y,
+                                     lr_stream_t stream);
+
 /* ------------------------------------------------------------------------ */
 /* Hybrid SwiGLU FFN                                                        */
 /* ------------------------------------------------------------------------ */
