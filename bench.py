@@ -6,8 +6,9 @@ Workload (one "step"): one decode token through a LLaMA-7B-shaped stack of
 hidden 4096, seeded non-uniform ranks in [512, 1536] at 40 % parameter
 reduction, batch 1).  Per layer: one grouped call computes Q, K, V from the
 layer input x; the O projection reads the V output (single-token attention
-returns V exactly) and its output is the next layer's input.  Every
-projection is one launch of the library's fused factorised-linear kernel.
+returns V exactly) and its output is the next layer's input.  The
+whole stack is one lr_linear_chain call: one launch per step, with one
+grid-wide barrier per dependent projection inside it.
 
 The 32 layers hold 2.58 GB of factors, far above the 126 MB L2, so every
 step streams them from HBM (no L2 flush needed).  Timing: W untimed warm-up
@@ -47,6 +48,8 @@ def parse(argv=None):
     ap.add_argument("--batch", type=int, default=1)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--layers", type=int, default=LAYERS,
+                    help="layers in the stack (default 32; fewer only for profiling small cases)")
     return ap.parse_args(argv)
 
 
@@ -100,7 +103,7 @@ def host_cores() -> int:
 # ---------------------------------------------------------------------------
 def algorithmic_bytes_per_step(ranks, batch: int) -> int:
     """Factor bytes (bf16) of all 128 projections plus activation reads/writes."""
-    factor = int(sum(int(r) * (HIDDEN + HIDDEN) * 2 for r in ranks.reshape(-1)))
+    factor = int(sum(int(r) * (HIDDEN + HIDDEN) * 2 for r in ranks[:LAYERS].reshape(-1)))
     act = LAYERS * batch * HIDDEN * 2 * (2 + 4)  # reads: x (shared by Q/K/V), v; writes: q, k, v, o
     return factor + act
 
@@ -205,6 +208,8 @@ def measured_hbm_peak():
 
 
 def run_ours(args) -> None:
+    global LAYERS
+    LAYERS = args.layers
     import torch
 
     import decode_lr_linear_b200 as lr
@@ -221,17 +226,18 @@ def run_ours(args) -> None:
     x0 = synth.make_activations(batch, HIDDEN, seed=0, key=(90,)).to(device)
     qkv = [[torch.empty(batch, HIDDEN, dtype=torch.bfloat16, device=device) for _ in range(3)] for _ in range(LAYERS)]
     outs = [torch.empty(batch, HIDDEN, dtype=torch.bfloat16, device=device) for _ in range(LAYERS)]
-    ws = lr.workspace(lr.lr_linear_grouped_workspace_size([layers[0][n] for n in "qkv"], batch), device)
+    # the whole stack as one chain: step 2l = Q/K/V of layer l (input: the previous O), step 2l+1 = O (input: V)
+    steps = []
+    for l in range(LAYERS):
+        L = layers[l]
+        steps.append(lr.ChainStep([L["q"], L["k"], L["v"]], -1 if l == 0 else 2 * l - 1, 0, qkv[l]))
+        steps.append(lr.ChainStep([L["o"]], 2 * l, 2, [outs[l]]))
+    ws = lr.workspace(lr.lr_linear_chain_workspace_size(steps, batch), device)
 
     def step():
-        x = x0
-        for l in range(LAYERS):
-            L = layers[l]
-            lr.lr_linear_grouped([L["q"], L["k"], L["v"]], x, ys=qkv[l], ws=ws)
-            lr.lr_linear(L["o"], qkv[l][2], y=outs[l], ws=ws)
-            x = outs[l]
+        lr.lr_linear_chain(steps, x0, ws=ws)
 
-    launches_per_step = 2 * LAYERS * ((batch + 7) // 8)
+    launches_per_step = (batch + 7) // 8
     step()
     torch.cuda.synchronize()
     g = torch.cuda.CUDAGraph()
@@ -300,9 +306,10 @@ def run_ours(args) -> None:
         "layer_us": ms_step * 1e3 / LAYERS,
         "hbm_gbs": achieved,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                     "traffic": None, "peak_source": peak_kind, "kernel": "lr_rank1_kernel (bf16, batch 1)",
-                     "note": "the step is launches of this one kernel only, so its mean launch duration is the "
-                             "event-timed step time over the launch count"},
+                     "traffic": None, "peak_source": peak_kind,
+                     "kernel": "chain_kernel<bf16, batch 1> (factorised-linear chain)",
+                     "note": "the step is one launch of this kernel only, so its launch duration is the "
+                             "event-timed step time"},
         "gpu_launches": launches_per_step * args.steps,
         "e2e": {"value": world * batch / (ms_e2e * 1e-3), "unit": "tokens/s",
                 "h2d_bytes_per_step": int(x_host.numel() * x_host.element_size()),

@@ -5,12 +5,13 @@ The compute path is the CUDA shared library ``liblr_decode.so`` (built by
 arguments.  ``synth`` holds the seeded synthetic-input generators.
 """
 from .ops import (  # noqa: F401
-    Factor, FfnWeights, LatentKv, workspace,
+    Factor, FfnWeights, LatentKv, ChainStep, workspace, lr_linear_chain, lr_linear_chain_workspace_size,
     lr_linear, lr_linear_workspace_size, lr_linear_grouped, lr_linear_grouped_workspace_size,
     lr_swiglu_ffn, lr_swiglu_ffn_workspace_size, lr_latent_kv_decode, lr_latent_kv_workspace_size,
-    lr_quantize_per_token, lr_workspace_init, lr_check_device_error,
+    lr_quantize_per_token, lr_gemm_s8s32, lr_workspace_init, lr_check_device_error,
 )
 from ._lib import LrError, load  # noqa: F401
 
-__all__ = [n for n in dir() if n.startswith("lr_")] + ["Factor", "FfnWeights", "LatentKv", "workspace", "LrError",
+__all__ = [n for n in dir() if n.startswith("lr_")] + ["Factor", "FfnWeights", "LatentKv", "ChainStep", "workspace",
+                                                       "LrError",
                                                        "load"]

@@ -19,6 +19,7 @@ LR_OK, LR_ERR_INVALID_ARG, LR_ERR_UNSUPPORTED, LR_ERR_MISALIGNED, LR_ERR_WORKSPA
 # lr_dtype_t
 LR_F32, LR_BF16, LR_F16, LR_I8, LR_I32 = range(5)
 LR_MAX_GROUP = 4
+LR_MAX_CHAIN = 64
 LR_KV_ABSORBED, LR_KV_RECONSTRUCT = 0, 1
 LR_NOALLOC_SCRATCH_BYTES = 1 << 20
 
@@ -29,6 +30,11 @@ class FactorDesc(ctypes.Structure):
     _fields_ = [("A", c_void_p), ("B", c_void_p), ("d_in", c_int), ("d_out", c_int), ("rank", c_int),
                 ("active_rank", c_int), ("w_dtype", c_int), ("scale_dtype", c_int),
                 ("scale_A", c_void_p), ("scale_B", c_void_p)]
+
+
+class ChainStep(ctypes.Structure):
+    _fields_ = [("n", c_int), ("input_step", c_int), ("input_proj", c_int),
+                ("proj", FactorDesc * 4), ("y", c_void_p * 4)]
 
 
 class FfnDesc(ctypes.Structure):
@@ -48,6 +54,8 @@ _SIGNATURES = {
     "lr_linear": (c_int, [P(FactorDesc), c_void_p, c_void_p, c_int, c_void_p, c_void_p, c_size_t, c_void_p]),
     "lr_linear_workspace_size": (c_int, [P(FactorDesc), c_int, c_int, P(c_size_t)]),
     "lr_linear_noalloc": (c_int, [P(FactorDesc), c_void_p, c_int, c_void_p, c_void_p]),
+    "lr_linear_chain": (c_int, [P(ChainStep), c_int, c_void_p, c_int, c_void_p, c_size_t, c_void_p]),
+    "lr_linear_chain_workspace_size": (c_int, [P(ChainStep), c_int, c_int, P(c_size_t)]),
     "lr_linear_grouped": (c_int, [P(FactorDesc), c_int, c_void_p, c_int, P(c_void_p), c_void_p, c_size_t,
                                   c_void_p]),
     "lr_linear_grouped_workspace_size": (c_int, [P(FactorDesc), c_int, c_int, P(c_size_t)]),
@@ -57,6 +65,7 @@ _SIGNATURES = {
                                     c_size_t, c_void_p]),
     "lr_latent_kv_workspace_size": (c_int, [P(LatentKvDesc), P(c_size_t)]),
     "lr_quantize_per_token": (c_int, [c_void_p, c_int, c_int, c_void_p, c_void_p, c_void_p]),
+    "lr_gemm_s8s32": (c_int, [c_void_p, c_void_p, c_int, c_int, c_int, c_int, c_void_p, c_void_p]),
     "lr_workspace_init": (c_int, [c_void_p, c_size_t, c_void_p]),
     "lr_check_device_error": (c_int, [c_void_p, P(c_int)]),
     "lr_status_string": (ctypes.c_char_p, [c_int]),

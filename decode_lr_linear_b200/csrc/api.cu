@@ -69,54 +69,132 @@ lr_status_t check_factor(const lr_factor_desc_t* d) {
 
 inline int active(const lr_factor_desc_t* d) { return d->active_rank ? d->active_rank : d->rank; }
 
-size_t rank1_ws_bytes(const lr_factor_desc_t* descs, int n, int batch) {
+// Limits of the streaming decode kernels: rows are moved by bulk copies, so a
+// row must be 16-byte aligned and fit one 32 KiB shared-memory stage.
+lr_status_t check_rank1_limits(const lr_factor_desc_t* d) {
+  const size_t es = d->w_dtype == LR_F32 ? 4 : (d->w_dtype == LR_BF16 ? 2 : 1);
+  if ((size_t(d->d_in) * es) % 16 != 0 || (size_t(d->d_out) * es) % 16 != 0) return LR_ERR_UNSUPPORTED;
+  if (size_t(d->d_in) * es > 32768 || size_t(d->d_out) * es > 32768) return LR_ERR_UNSUPPORTED;
+  return LR_OK;
+}
+
+// One step of a chain as the host sees it.
+struct HostStep {
+  const lr_factor_desc_t* d;
+  int n;
+  int input_step;
+  int input_proj;
+  void* const* y;
+};
+
+// Floats of one accumulator set: the largest step's outputs for one batch chunk.
+size_t chain_acc_set(const HostStep* steps, int n_steps, int batch) {
   const int chunk = std::min(batch, kMaxDecodeChunk);
-  size_t b = kTicketBytes;
-  for (int p = 0; p < n; ++p) b += round_up(size_t(chunk) * descs[p].d_out * 4, 256);
-  return b;
+  size_t m = 0;
+  for (int s = 0; s < n_steps; ++s) {
+    size_t t = 0;
+    for (int p = 0; p < steps[s].n; ++p) t += size_t(chunk) * steps[s].d[p].d_out;
+    m = std::max(m, t);
+  }
+  return round_up(m, 64);
+}
+
+size_t chain_ws_bytes(const HostStep* steps, int n_steps, int batch) {
+  return kTicketBytes + 3 * chain_acc_set(steps, n_steps, batch) * 4;
+}
+
+size_t rank1_ws_bytes(const lr_factor_desc_t* descs, int n, int batch) {
+  HostStep h{descs, n, -1, 0, nullptr};
+  return chain_ws_bytes(&h, 1, batch);
+}
+
+lr_status_t check_chain(const HostStep* steps, int n_steps) {
+  if (n_steps < 1 || n_steps > LR_MAX_CHAIN) return LR_ERR_INVALID_ARG;
+  const lr_factor_desc_t& d0 = steps[0].d[0];
+  int x_width = -1;
+  for (int s = 0; s < n_steps; ++s) {
+    const HostStep& h = steps[s];
+    if (h.n < 1 || h.n > LR_MAX_GROUP || !h.d || !h.y) return LR_ERR_INVALID_ARG;
+    for (int p = 0; p < h.n; ++p) {
+      lr_status_t st = check_factor(&h.d[p]);
+      if (st != LR_OK) return st;
+      st = check_rank1_limits(&h.d[p]);
+      if (st != LR_OK) return st;
+      if (h.d[p].d_in != h.d[0].d_in || h.d[p].w_dtype != d0.w_dtype) return LR_ERR_INVALID_ARG;
+      if (d0.w_dtype == LR_I8 && h.d[p].scale_dtype != d0.scale_dtype) return LR_ERR_INVALID_ARG;
+      if (!h.y[p]) return LR_ERR_INVALID_ARG;
+      if (!al16(h.y[p])) return LR_ERR_MISALIGNED;
+    }
+    if (h.input_step < 0) {
+      if (x_width >= 0 && x_width != h.d[0].d_in) return LR_ERR_INVALID_ARG;
+      x_width = h.d[0].d_in;
+    } else {
+      if (h.input_step >= s) return LR_ERR_INVALID_ARG;
+      const HostStep& src = steps[h.input_step];
+      if (h.input_proj < 0 || h.input_proj >= src.n) return LR_ERR_INVALID_ARG;
+      if (src.d[h.input_proj].d_out != h.d[0].d_in) return LR_ERR_INVALID_ARG;
+    }
+  }
+  return LR_OK;
+}
+
+lr_status_t run_chain(const HostStep* steps, int n_steps, const void* x, int batch, void* ws, size_t ws_bytes,
+                      cudaStream_t stream) {
+  lr_status_t st = check_chain(steps, n_steps);
+  if (st != LR_OK) return st;
+  if (!x || batch < 1) return LR_ERR_INVALID_ARG;
+  if (!al16(x)) return LR_ERR_MISALIGNED;
+  if (!ws || ws_bytes < chain_ws_bytes(steps, n_steps, batch)) return LR_ERR_WORKSPACE;
+  if (!al16(ws)) return LR_ERR_MISALIGNED;
+  const lr_dtype_t wt = steps[0].d[0].w_dtype;
+  const size_t es = (wt == LR_F32) ? 4 : 2;  // activation / output element size
+  static ChainParams P;                      // large (kernel parameters); filled under a lock
+  static std::mutex mu;
+  std::lock_guard<std::mutex> lock(mu);
+  std::memset(&P, 0, sizeof(P));
+  P.n_steps = n_steps;
+  P.scale_f16 = steps[0].d[0].scale_dtype == LR_F16 ? 1 : 0;
+  P.bar = reinterpret_cast<unsigned int*>(ws);
+  P.acc = reinterpret_cast<float*>(reinterpret_cast<char*>(ws) + kTicketBytes);
+  P.acc_set = int(chain_acc_set(steps, n_steps, batch));
+  P.err = device_error_word();
+  int x_width = 0;
+  for (int s = 0; s < n_steps; ++s) {
+    ChainStep& c = P.step[s];
+    c.n = steps[s].n;
+    c.d_in = steps[s].d[0].d_in;
+    c.input_step = steps[s].input_step < 0 ? -1 : steps[s].input_step;
+    c.input_proj = steps[s].input_proj;
+    if (c.input_step < 0) x_width = c.d_in;
+    int rows = 0;
+    for (int p = 0; p < c.n; ++p) {
+      const lr_factor_desc_t& d = steps[s].d[p];
+      c.p[p].A = d.A;
+      c.p[p].B = d.B;
+      c.p[p].sA = wt == LR_I8 ? d.scale_A : nullptr;
+      c.p[p].sB = wt == LR_I8 ? d.scale_B : nullptr;
+      c.p[p].d_out = d.d_out;
+      c.p[p].rows = active(&d);
+      rows += c.p[p].rows;
+    }
+    c.total_rows = rows;
+  }
+  const int sms = sm_count_current();
+  for (int b0 = 0; b0 < batch; b0 += kMaxDecodeChunk) {
+    P.nb = std::min(kMaxDecodeChunk, batch - b0);
+    P.x = reinterpret_cast<const char*>(x) + size_t(b0) * x_width * es;
+    for (int s = 0; s < n_steps; ++s)
+      for (int p = 0; p < P.step[s].n; ++p)
+        P.step[s].p[p].y = reinterpret_cast<char*>(steps[s].y[p]) + size_t(b0) * steps[s].d[p].d_out * es;
+    if (launch_chain(P, wt, sms, stream) != cudaSuccess) return LR_ERR_CUDA;
+  }
+  return LR_OK;
 }
 
 lr_status_t run_rank1(const lr_factor_desc_t* descs, int n, const void* x, int batch, void* const* ys, void* ws,
                       size_t ws_bytes, cudaStream_t stream) {
-  const lr_dtype_t wt = descs[0].w_dtype;
-  const size_t xs = (wt == LR_F32) ? 4 : 2;
-  const size_t ysz = (wt == LR_F32) ? 4 : 2;
-  if (!ws) return LR_ERR_WORKSPACE;
-  if (ws_bytes < rank1_ws_bytes(descs, n, batch)) return LR_ERR_WORKSPACE;
-  if (!al16(ws)) return LR_ERR_MISALIGNED;
-  Rank1Params P;
-  std::memset(&P, 0, sizeof(P));
-  P.n_proj = n;
-  P.d_in = descs[0].d_in;
-  P.scale_f16 = descs[0].scale_dtype == LR_F16 ? 1 : 0;
-  P.ticket = reinterpret_cast<unsigned int*>(ws);
-  const int chunk = std::min(batch, kMaxDecodeChunk);
-  char* accp = reinterpret_cast<char*>(ws) + kTicketBytes;
-  int row = 0;
-  for (int p = 0; p < n; ++p) {
-    Rank1Proj& pr = P.proj[p];
-    pr.A = descs[p].A;
-    pr.B = descs[p].B;
-    pr.sA = wt == LR_I8 ? descs[p].scale_A : nullptr;
-    pr.sB = wt == LR_I8 ? descs[p].scale_B : nullptr;
-    pr.acc = reinterpret_cast<float*>(accp);
-    accp += round_up(size_t(chunk) * descs[p].d_out * 4, 256);
-    pr.d_out = descs[p].d_out;
-    pr.rows = active(&descs[p]);
-    pr.row_begin = row;
-    row += pr.rows;
-  }
-  P.total_rows = row;
-  const int sms = sm_count_current();
-  for (int b0 = 0; b0 < batch; b0 += kMaxDecodeChunk) {
-    P.nb = std::min(kMaxDecodeChunk, batch - b0);
-    P.x = reinterpret_cast<const char*>(x) + size_t(b0) * P.d_in * xs;
-    for (int p = 0; p < n; ++p)
-      P.proj[p].y = reinterpret_cast<char*>(ys[p]) + size_t(b0) * descs[p].d_out * ysz;
-    cudaError_t e = launch_lr_rank1(P, wt, sms, stream);
-    if (e != cudaSuccess) return LR_ERR_CUDA;
-  }
-  return LR_OK;
+  HostStep h{descs, n, -1, 0, ys};
+  return run_chain(&h, 1, x, batch, ws, ws_bytes, stream);
 }
 
 // ---------------------------------------------------------------------------
@@ -210,6 +288,8 @@ lr_status_t lr_linear(const lr_factor_desc_t* desc, const void* x, const float* 
     P.zq = reinterpret_cast<int8_t*>(w);
     w += round_up(size_t(round_up(batch, 128)) * P.rank_pad, 256);
     P.sz = reinterpret_cast<float*>(w);
+    w += round_up(size_t(round_up(batch, 128)) * 4, 256);
+    P.amax = reinterpret_cast<unsigned int*>(w);
     P.err = device_error_word();
     return from_cuda(launch_w8a8(P, sm_count_current(), s));
   }
@@ -242,6 +322,24 @@ lr_status_t lr_linear_grouped(const lr_factor_desc_t* descs, int n, const void* 
   return run_rank1(descs, n, x, batch, ys, ws, ws_bytes, reinterpret_cast<cudaStream_t>(stream));
 }
 
+lr_status_t lr_linear_chain_workspace_size(const lr_chain_step_t* steps, int n_steps, int batch, size_t* bytes) {
+  if (!bytes || !steps || n_steps < 1 || n_steps > LR_MAX_CHAIN || batch < 1) return LR_ERR_INVALID_ARG;
+  HostStep h[LR_MAX_CHAIN];
+  for (int s = 0; s < n_steps; ++s) h[s] = HostStep{steps[s].proj, steps[s].n, steps[s].input_step, steps[s].input_proj, steps[s].y};
+  lr_status_t st = check_chain(h, n_steps);
+  if (st != LR_OK) return st;
+  *bytes = chain_ws_bytes(h, n_steps, batch);
+  return LR_OK;
+}
+
+lr_status_t lr_linear_chain(const lr_chain_step_t* steps, int n_steps, const void* x, int batch, void* ws,
+                            size_t ws_bytes, lr_stream_t stream) {
+  if (!steps || n_steps < 1 || n_steps > LR_MAX_CHAIN) return LR_ERR_INVALID_ARG;
+  HostStep h[LR_MAX_CHAIN];
+  for (int s = 0; s < n_steps; ++s) h[s] = HostStep{steps[s].proj, steps[s].n, steps[s].input_step, steps[s].input_proj, steps[s].y};
+  return run_chain(h, n_steps, x, batch, ws, ws_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
 // --------------------------------------------------------------------------
 
 static lr_status_t check_ffn(const lr_ffn_desc_t* d) {
@@ -251,7 +349,8 @@ static lr_status_t check_ffn(const lr_ffn_desc_t* d) {
   if (d->inter > d->n_lr && (!d->D || !d->s_D)) return LR_ERR_INVALID_ARG;
   if (!d->W_down || !d->s_down) return LR_ERR_INVALID_ARG;
   if (d->scale_dtype != LR_F16 && d->scale_dtype != LR_F32) return LR_ERR_UNSUPPORTED;
-  if ((d->hidden % 16) != 0 || (d->n_lr % 4) != 0) return LR_ERR_UNSUPPORTED;
+  if ((d->hidden % 16) != 0 || (d->n_lr % 8) != 0) return LR_ERR_UNSUPPORTED;
+  if (d->hidden > 32768 || 2 * d->n_lr > 32768) return LR_ERR_UNSUPPORTED;
   const void* ptrs[] = {d->A, d->s_A, d->B, d->s_B, d->D, d->s_D, d->W_down, d->s_down};
   for (const void* p : ptrs)
     if (p && !al16(p)) return LR_ERR_MISALIGNED;
@@ -361,6 +460,16 @@ lr_status_t lr_quantize_per_token(const void* x, int rows, int cols, int8_t* x_q
   if ((cols % 16) != 0 || cols > 49152) return LR_ERR_UNSUPPORTED;
   if (!al16(x) || !al16(x_q) || !al16(s)) return LR_ERR_MISALIGNED;
   return from_cuda(launch_quantize_per_token(x, rows, cols, x_q, s, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+lr_status_t lr_gemm_s8s32(const int8_t* A, const int8_t* B, int b_layout, int M, int N, int K, int32_t* C,
+                          lr_stream_t stream) {
+  if (!A || !B || !C || M < 1 || N < 1 || K < 1) return LR_ERR_INVALID_ARG;
+  if (b_layout != 0 && b_layout != 1) return LR_ERR_INVALID_ARG;
+  if ((K % 16) != 0 || (N % 16) != 0 || K >= 133144) return LR_ERR_UNSUPPORTED;
+  if (!al16(A) || !al16(B) || !al16(C)) return LR_ERR_MISALIGNED;
+  return from_cuda(launch_gemm_s8s32(A, B, b_layout, M, N, K, C, device_error_word(),
+                                     reinterpret_cast<cudaStream_t>(stream)));
 }
 
 lr_status_t lr_workspace_init(void* ws, size_t ws_bytes, lr_stream_t stream) {

@@ -11,6 +11,7 @@
 #include <utility>
 
 #define LR_DEV __device__ __forceinline__
+#define LR_HD_INLINE __host__ __device__ __forceinline__
 
 namespace lr {
 
@@ -20,6 +21,7 @@ enum DeviceErrorCode : int {
   kErrNone = 0,
   kErrMbarTimeout = 1,   // an mbarrier wait gave up
   kErrTmemTimeout = 2,   // a TMEM allocation could not be obtained
+  kErrGridBarrier = 3,   // a grid-wide barrier wait gave up
 };
 
 LR_DEV void set_device_error(int* err, int code) {
@@ -55,6 +57,11 @@ LR_DEV float4 ld_cg_f4(const float* p) {
   float4 v;
   asm volatile("ld.global.cg.v4.f32 {%0,%1,%2,%3}, [%4];"
                : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "l"(p) : "memory");
+  return v;
+}
+LR_DEV unsigned int ld_acquire_u32(const unsigned int* p) {
+  unsigned int v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
   return v;
 }
 LR_DEV void st_cg_f4(float* p, float4 v) {

@@ -3,467 +3,1128 @@
 //
 // A factorised linear y = (x A) B is evaluated as a sum of rank-1 terms,
 // y = sum_j z_j b_j with z_j = x . a_j, where a_j / b_j are the latent-major
-// rows of the two factors.  Each CTA owns a contiguous block of latent rows:
-// it streams its rows of A (phase A, z_j kept in shared memory), then its rows
-// of B (phase B), and adds its partial y into an fp32 accumulator in L2 with
-// vector reductions.  The last CTA to arrive (atomic ticket, no waiting)
-// converts the accumulator to the output type and zeroes it again.  Both
-// factor streams are read exactly once, coalesced, 8 elements per lane.
+// rows of the two factors.  Each CTA owns a contiguous block of latent rows.
+// One producer warp streams the CTA's rows of A and then of B through a ring
+// of shared-memory stages with bulk asynchronous copies (cp.async.bulk,
+// completing on mbarriers); sixteen consumer warps compute from shared memory:
+//   phase A: z_j = a_j . x for the CTA's rows (x staged in shared memory),
+//   phase B: partial y += z_j b_j, added into an fp32 accumulator in L2 with
+//            vector reductions (red.global.add.v4.f32).
+// The last CTA to arrive (atomic ticket, no waiting) converts the accumulator
+// to the output type and zeroes it again.  Each factor byte is read once;
+// the weight copies are issued before the programmatic-dependent-launch wait,
+// so they overlap the tail of the preceding kernel.
 //
-// The same building blocks evaluate the hybrid FFN of LASER ("Hybrid
-// SVD-Quantization for FFNs", "System Implementation") in two launches:
+// The same engine evaluates the hybrid FFN of LASER ("Hybrid SVD-Quantization
+// for FFNs", "System Implementation") in two launches:
 //   phase 1: low-rank branch  z = x A', [g_S,u_S] += z_j b'_j  (reduction)
 //            dense branch     [g_D,u_D] = x D' row dots, SwiGLU in the epilogue
 //   phase 2: h = [silu(g_S) u_S, h_D]; y += h_c w_c over input channels of
 //            W_down (reduction), last CTA applies the output scales.
+#include <algorithm>
+#include <cstring>
+#include <type_traits>
+
 #include "common.cuh"
 #include "internal.h"
 
 namespace lr {
-
 namespace {
 
-constexpr int kThreads = 512;
-constexpr int kWarps = kThreads / 32;
-constexpr int kLine = 256;          // elements covered by one warp-wide chunk load
-constexpr int kMaxRowsCta = 96;     // latent rows owned by one CTA, at most
-// independent chunk loads in flight per lane (fewer for wide batches: registers)
-template <int NB> constexpr int unroll_for() { return NB >= 8 ? 2 : (NB >= 4 ? 4 : 8); }
+constexpr int kConsumerWarps = 16;
+constexpr int kConsumers = kConsumerWarps * 32;
+constexpr int kThreads = kConsumers + 32;  // + one producer warp
+constexpr int kLineElems = 256;            // elements of one warp-wide chunk (8 per lane)
+constexpr int kStageBytes = 32 * 1024;
+constexpr int kMaxStages = 4;
+// A CTA that fits in this much shared memory can share its SM with the next
+// kernel's CTA, whose producer then streams while this one drains.
+constexpr size_t kCoResidentSmem = 108 * 1024;
+constexpr int kRowGroup = 4;               // rows reduced together in phase A (ILP)
+constexpr int kMaxSegs = 2 * kMaxGroup;
+constexpr size_t kSmemLimit = 227 * 1024;
 
-struct SmemLayout {
-  // part [rows][kWarps][NB] fp32, z [rows][NB] fp32, row pointers, row projections
-  static size_t bytes(int rows, int nb) {
-    return size_t(rows) * kWarps * nb * 4 + size_t(rows) * nb * 4 + size_t(rows) * 8 + size_t(rows) * 4 + 64;
-  }
+enum Mode : int { kLinear = 0, kFfn1 = 1, kFfn2 = 2 };
+enum SegKind : int { kDot = 0, kRank1 = 1 };
+
+struct Seg {
+  const unsigned char* src;  // first byte of the segment's first row
+  int row_bytes;
+  int rows;
+  int rps;                   // rows per ring stage
+  int kind;                  // kDot: row . x ; kRank1: acc += z_row * row
+  int zrow0;                 // CTA-local index of the first row (into part / z)
+  int proj;                  // projection (kLinear)
 };
 
-// Phase A: part[r][warp][b] = sum over this warp's lines of a_r . x_b.
-template <typename WT, typename XT, int NB, int kUnroll = unroll_for<NB>()>
-LR_DEV void phase_dot(const WT* const* arow, int nr, int d_in, const XT* x, int nb, float* part) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  for (int i = lane; i < nr * NB; i += 32) part[(i / NB) * kWarps * NB + warp * NB + (i % NB)] = 0.f;
-  __syncwarp();
-  const int nlines = (d_in + kLine - 1) / kLine;
-  for (int l = warp; l < nlines; l += kWarps) {
-    const int col = l * kLine + lane * 8;
-    const bool cv = col < d_in;
-    float xr[NB][8];
+struct Plan {
+  Seg seg[kMaxSegs];
+  int nseg;
+  int nrows;
+  int row_base;              // first global row of the CTA (scales, channel ids)
+  int role;                  // kFfn1: 0 low-rank branch, 1 dense branch
+};
+
+struct KParams {
+  Rank1Params r;
+  FfnParams f;
+  int g_lr;                  // kFfn1: CTAs of the low-rank branch
+  int stages;                // ring stages in use
+  int rows_cap;              // rows per CTA the shared-memory layout holds
+  int x_elems;               // elements of one staged activation row (0: none)
+  int* err;
+};
+
+struct Layout {
+  size_t ring, x, part, z, total;
+};
+
+LR_HD_INLINE size_t round16(size_t v) { return (v + 15) & ~size_t(15); }
+
+template <int NB>
+LR_HD_INLINE Layout layout_for(int stages, int x_elems, int x_esize, int rows_cap) {
+  Layout L;
+  L.ring = 0;
+  L.x = size_t(stages) * kStageBytes;
+  L.part = L.x + round16(size_t(NB) * x_elems * x_esize);
+  L.z = L.part + round16(size_t(rows_cap) * kConsumerWarps * NB * 4);
+  L.total = L.z + round16(size_t(rows_cap) * NB * 4);
+  return L;
+}
+
+// ---- shared-memory chunk loads (8 elements) --------------------------------
+template <typename T> struct SChunk;
+template <> struct SChunk<float> {
+  LR_DEV static void load(const unsigned char* p, float* f) {
+    const float4 a = *reinterpret_cast<const float4*>(p), b = *reinterpret_cast<const float4*>(p + 16);
+    f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w; f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
+  }
+};
+template <> struct SChunk<__nv_bfloat16> {
+  LR_DEV static void load(const unsigned char* p, float* f) { bf16x8_to_f32(*reinterpret_cast<const uint4*>(p), f); }
+};
+template <> struct SChunk<int8_t> {
+  LR_DEV static void load(const unsigned char* p, float* f) { i8x8_to_f32(*reinterpret_cast<const uint2*>(p), f); }
+};
+
+LR_DEV void consumer_sync() { asm volatile("bar.sync 1, %0;" :: "r"(kConsumers) : "memory"); }
+
+// Sum of four per-lane values over the warp for each of the four, with six
+// shuffles: after the two exchange steps lane l holds a partial of value
+// ((l >> 3) & 3) over lanes {l, l^8, l^16, l^24}; three more steps finish it.
+// Lanes 0, 8, 16 and 24 return the totals of values 0, 1, 2 and 3.
+LR_DEV float warp_sum4(float v0, float v1, float v2, float v3, int lane) {
+  const bool hi = (lane & 16) != 0, mid = (lane & 8) != 0;
+  const float r0 = __shfl_xor_sync(0xffffffffu, hi ? v0 : v2, 16);
+  const float r1 = __shfl_xor_sync(0xffffffffu, hi ? v1 : v3, 16);
+  const float k0 = (hi ? v2 : v0) + r0, k1 = (hi ? v3 : v1) + r1;
+  const float r = __shfl_xor_sync(0xffffffffu, mid ? k0 : k1, 8);
+  float t = (mid ? k1 : k0) + r;
+  t += __shfl_xor_sync(0xffffffffu, t, 4);
+  t += __shfl_xor_sync(0xffffffffu, t, 2);
+  t += __shfl_xor_sync(0xffffffffu, t, 1);
+  return t;
+}
+
+// ---- phase A: part[row][warp][b] = sum over this warp's lines of row . x_b --
+// Every (row, warp) slot is written exactly once (a row lives in one stage and
+// all of a warp's lines of that row are summed here), so part needs no zeroing.
+// When a row has at most kConsumerWarps lines, warp w only ever touches line w
+// and its x chunk comes from registers (xr), loaded once per kernel.
+template <typename WT, typename XT, int NB>
+LR_DEV void consume_dot(const unsigned char* stage, int k, int d_in, const XT* xs, const float (&xr)[NB][8],
+                        bool x_in_regs, float* part, int zrow, int cw, int lane) {
+  const int lines = (d_in + kLineElems - 1) / kLineElems;
+  for (int r0 = 0; r0 < k; r0 += kRowGroup) {
+    float s[kRowGroup][NB];
+#pragma unroll
+    for (int u = 0; u < kRowGroup; ++u)
+#pragma unroll
+      for (int b = 0; b < NB; ++b) s[u][b] = 0.f;
+    for (int line = cw; line < lines; line += kConsumerWarps) {
+      const int col = line * kLineElems + lane * 8;
+      if (col < d_in) {
+        float xv[NB][8];
+#pragma unroll
+        for (int b = 0; b < NB; ++b) {
+          if (NB <= 2 && x_in_regs) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) xv[b][e] = xr[b][e];
+          } else {
+            SChunk<XT>::load(reinterpret_cast<const unsigned char*>(xs + size_t(b) * d_in + col), xv[b]);
+          }
+        }
+        float w[kRowGroup][8];
+#pragma unroll
+        for (int u = 0; u < kRowGroup; ++u) {
+          const int rr = min(r0 + u, k - 1);  // rows past k load a valid row, masked below
+          SChunk<WT>::load(stage + (size_t(rr) * d_in + col) * sizeof(WT), w[u]);
+        }
+#pragma unroll
+        for (int u = 0; u < kRowGroup; ++u) {
+          const float m = (r0 + u < k) ? 1.f : 0.f;
+#pragma unroll
+          for (int b = 0; b < NB; ++b) {
+            float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+            for (int e = 0; e < 8; e += 2) {
+              a0 = fmaf(w[u][e], xv[b][e], a0);
+              a1 = fmaf(w[u][e + 1], xv[b][e + 1], a1);
+            }
+            s[u][b] = fmaf(m, a0 + a1, s[u][b]);
+          }
+        }
+      }
+    }
 #pragma unroll
     for (int b = 0; b < NB; ++b) {
-      if (cv && b < nb) load_act8(x + size_t(b) * d_in + col, xr[b]);
-      else {
-#pragma unroll
-        for (int e = 0; e < 8; ++e) xr[b][e] = 0.f;
-      }
-    }
-    for (int r = 0; r < nr; r += kUnroll) {
-      float w[kUnroll][8];
-#pragma unroll
-      for (int u = 0; u < kUnroll; ++u) {
-        if (cv && r + u < nr) Chunk<WT>::load(arow[r + u] + col, w[u]);
-        else {
-#pragma unroll
-          for (int e = 0; e < 8; ++e) w[u][e] = 0.f;
-        }
-      }
-#pragma unroll
-      for (int u = 0; u < kUnroll; ++u) {
-#pragma unroll
-        for (int b = 0; b < NB; ++b) {
-          float s = 0.f;
-#pragma unroll
-          for (int e = 0; e < 8; ++e) s = fmaf(w[u][e], xr[b][e], s);
-          s = warp_sum(s);
-          if (lane == 0 && r + u < nr) part[(r + u) * kWarps * NB + warp * NB + b] += s;
-        }
-      }
+      const float t = warp_sum4(s[0][b], s[1][b], s[2][b], s[3][b], lane);
+      const int u = lane >> 3;
+      if ((lane & 7) == 0 && r0 + u < k) part[(size_t(zrow + r0 + u) * kConsumerWarps + cw) * NB + b] = t;
     }
   }
 }
 
-// z[r][b] = sum_w part[r][w][b] (fixed order) times an optional row scale.
-template <int NB>
-LR_DEV void reduce_parts(const float* part, int nr, float* zs, const void* sA, const int* srow, bool f16) {
-  for (int i = threadIdx.x; i < nr * NB; i += kThreads) {
-    const int r = i / NB, b = i % NB;
-    float s = 0.f;
+// ---- phase B: acc[li][b][e] += z[row][b] * row[col+e] ----------------------
+template <typename WT, int NB, int LPW>
+LR_DEV void consume_rank1(const unsigned char* stage, int k, int d_out, const float* z, int zrow,
+                          float (&acc)[LPW][NB][8], int cw, int lane) {
+  const int lines = (d_out + kLineElems - 1) / kLineElems;
+#pragma unroll
+  for (int li = 0; li < LPW; ++li) {
+    const int line = cw + li * kConsumerWarps;
+    const int col = line * kLineElems + lane * 8;
+    if (line < lines && col < d_out) {
 #pragma unroll 4
-    for (int w = 0; w < kWarps; ++w) s += part[r * kWarps * NB + w * NB + b];
-    if (sA) s *= load_scale(sA, srow[r], f16);
-    zs[r * NB + b] = s;
-  }
-}
-
-// Phase B: acc[b][k] += sum_r z[r][b] * B0[r][k] over nr consecutive rows of B.
-template <typename WT, int NB, int kUnroll = unroll_for<NB>()>
-LR_DEV void phase_rank1(const WT* B0, int d_out, int nr, const float* zs, float* acc, int nb) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int nlines = (d_out + kLine - 1) / kLine;
-  for (int l = warp; l < nlines; l += kWarps) {
-    const int col = l * kLine + lane * 8;
-    const bool cv = col < d_out;
-    float a[NB][8];
-#pragma unroll
-    for (int b = 0; b < NB; ++b)
-#pragma unroll
-      for (int e = 0; e < 8; ++e) a[b][e] = 0.f;
-    for (int r = 0; r < nr; r += kUnroll) {
-      float w[kUnroll][8];
-#pragma unroll
-      for (int u = 0; u < kUnroll; ++u) {
-        if (cv && r + u < nr) Chunk<WT>::load(B0 + size_t(r + u) * d_out + col, w[u]);
-        else {
-#pragma unroll
-          for (int e = 0; e < 8; ++e) w[u][e] = 0.f;
-        }
-      }
-#pragma unroll
-      for (int u = 0; u < kUnroll; ++u) {
-        const int rr = (r + u < nr) ? (r + u) : r;  // w is zero when out of range
+      for (int i = 0; i < k; ++i) {
+        float w[8];
+        SChunk<WT>::load(stage + (size_t(i) * d_out + col) * sizeof(WT), w);
+        const float* zr = z + size_t(zrow + i) * NB;
 #pragma unroll
         for (int b = 0; b < NB; ++b) {
-          const float zb = zs[rr * NB + b];
+          const float zb = zr[b];
 #pragma unroll
-          for (int e = 0; e < 8; ++e) a[b][e] = fmaf(zb, w[u][e], a[b][e]);
+          for (int e = 0; e < 8; ++e) acc[li][b][e] = fmaf(zb, w[e], acc[li][b][e]);
         }
       }
     }
-    if (cv) {
+  }
+}
+
+template <int NB, int LPW>
+LR_DEV void flush_rank1(float (&acc)[LPW][NB][8], float* dst, int d_out, int nb, int cw, int lane) {
+  const int lines = (d_out + kLineElems - 1) / kLineElems;
+#pragma unroll
+  for (int li = 0; li < LPW; ++li) {
+    const int line = cw + li * kConsumerWarps;
+    const int col = line * kLineElems + lane * 8;
+    if (line < lines && col < d_out) {
 #pragma unroll
       for (int b = 0; b < NB; ++b) {
         if (b < nb) {
-          float* p = acc + size_t(b) * d_out + col;
-          red_add_f4(p, a[b][0], a[b][1], a[b][2], a[b][3]);
-          red_add_f4(p + 4, a[b][4], a[b][5], a[b][6], a[b][7]);
+          float* p = dst + size_t(b) * d_out + col;
+          red_add_f4(p, acc[li][b][0], acc[li][b][1], acc[li][b][2], acc[li][b][3]);
+          red_add_f4(p + 4, acc[li][b][4], acc[li][b][5], acc[li][b][6], acc[li][b][7]);
         }
+      }
+    }
+#pragma unroll
+    for (int b = 0; b < NB; ++b)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[li][b][e] = 0.f;
+  }
+}
+
+// ---- producer: stream every segment's rows through the ring ---------------
+LR_DEV void produce(const Plan& pl, unsigned char* ring, uint64_t* full, uint64_t* empty, int stages, int* err) {
+  // Start the DRAM reads of the CTA's whole working set at once (into L2); the
+  // ring copies below then mostly hit L2, and DRAM streaming does not wait for
+  // consumer progress or for the preceding kernel.
+  for (int s = 0; s < pl.nseg; ++s) {
+    const Seg& g = pl.seg[s];
+    const size_t total = size_t(g.rows) * g.row_bytes;
+    for (size_t off = 0; off < total; off += kStageBytes)
+      prefetch_l2_bulk(g.src + off, uint32_t(total - off < size_t(kStageBytes) ? total - off : kStageBytes));
+  }
+  int st = 0;
+  for (int s = 0; s < pl.nseg; ++s) {
+    const Seg& g = pl.seg[s];
+    for (int r = 0; r < g.rows; r += g.rps) {
+      const int k = min(g.rps, g.rows - r);
+      const int slot = st % stages, round = st / stages;
+      if (round > 0 && !mbar_wait_bounded(&empty[slot], uint32_t(round - 1) & 1u, err)) return;
+      const uint32_t bytes = uint32_t(k) * uint32_t(g.row_bytes);
+      mbar_arrive_expect_tx(&full[slot], bytes);
+      bulk_g2s(ring + size_t(slot) * kStageBytes, g.src + size_t(r) * g.row_bytes, bytes, &full[slot]);
+      ++st;
+    }
+  }
+}
+
+// Barrier over the CTAs of one launch.  The grid never exceeds the CTAs that
+// can be resident at once (one per SM at most), so every CTA gets to arrive.
+// words[0] counts arrivals, words[1] is a generation number: the last CTA to
+// arrive resets the count and bumps the generation; the others wait (bounded:
+// after ~2^22 polls the wait gives up and sets the device error word) until
+// the generation changes.  All threads of the CTA call it; on return every
+// CTA's earlier global writes and reductions are visible.
+LR_DEV void grid_barrier(unsigned int* words, int* err) {
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const unsigned gen = ld_acquire_u32(words + 1);
+    const unsigned prev = atomicAdd(words, 1u);
+    if (prev == gridDim.x - 1) {
+      atomicExch(words, 0u);
+      __threadfence();
+      atomicAdd(words + 1, 1u);
+    } else {
+      uint32_t i = 0;
+      while (ld_acquire_u32(words + 1) == gen) {
+        if (++i > (1u << 22)) {
+          set_device_error(err, kErrGridBarrier);
+          break;
+        }
+        __nanosleep(32);
+      }
+    }
+  }
+  __syncthreads();
+  __threadfence();
+}
+
+// One output of a split reduction: y[b][k] = acc[b][k] * scale[k] (optional).
+struct FinalTarget {
+  float* acc;
+  void* y;
+  const void* scale;
+  int n;       // nb * d_out
+  int d_out;
+};
+
+template <typename YT>
+LR_DEV void finalize_chunk(const FinalTarget& t, int i, bool f16) {
+  const float4 v0 = ld_cg_f4(t.acc + i), v1 = ld_cg_f4(t.acc + i + 4);
+  const int k = i % t.d_out;
+  float v[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+  if (t.scale) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) v[e] *= load_scale(t.scale, k + e, f16);
+  }
+  YT* y = reinterpret_cast<YT*>(t.y);
+  if constexpr (sizeof(YT) == 2) {
+    uint4 o;
+    uint32_t* ow = reinterpret_cast<uint32_t*>(&o);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * e], v[2 * e + 1]);
+      ow[e] = *reinterpret_cast<uint32_t*>(&h);
+    }
+    *reinterpret_cast<uint4*>(y + i) = o;
+  } else {
+    *reinterpret_cast<float4*>(y + i) = make_float4(v[0], v[1], v[2], v[3]);
+    *reinterpret_cast<float4*>(y + i + 4) = make_float4(v[4], v[5], v[6], v[7]);
+  }
+  const float4 zero = make_float4(0.f, 0.f, 0.f, 0.f);
+  st_cg_f4(t.acc + i, zero);
+  st_cg_f4(t.acc + i + 4, zero);
+}
+
+// After the grid barrier: this CTA converts its 1/gridDim share of all the
+// targets' 8-element chunks (targets concatenated) and zeroes them in acc.
+template <typename YT, int NT>
+LR_DEV void finalize_slice(const FinalTarget (&t)[NT], int nt, bool f16) {
+  int total = 0;
+#pragma unroll
+  for (int q = 0; q < NT; ++q)
+    if (q < nt) total += t[q].n / 8;
+  const int c0 = int((long long)total * blockIdx.x / gridDim.x);
+  const int c1 = int((long long)total * (blockIdx.x + 1) / gridDim.x);
+  for (int c = c0 + int(threadIdx.x); c < c1; c += kThreads) {
+    int off = c;
+#pragma unroll
+    for (int q = 0; q < NT; ++q) {
+      if (q < nt) {
+        const int nq = t[q].n / 8;
+        if (off >= 0 && off < nq) finalize_chunk<YT>(t[q], off * 8, f16);
+        off -= nq;
       }
     }
   }
 }
 
-// Arrival ticket: returns true in exactly one CTA, the last one to arrive,
-// after every CTA's reductions are visible to it.
-LR_DEV bool last_cta_arrives(unsigned int* ticket) {
-  __shared__ int s_last;
-  __threadfence();
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    const unsigned prev = atomicAdd(ticket, 1u);
-    s_last = (prev == gridDim.x - 1) ? 1 : 0;
-  }
-  __syncthreads();
-  if (!s_last) return false;
-  __threadfence();
-  return true;
+LR_DEV void split_range(long long total, int part, int parts, int* a, int* b) {
+  *a = int(total * part / parts);
+  *b = int(total * (part + 1) / parts);
 }
 
-// y[b][k] = acc[b][k] * scale[k] (optional) in the output type; acc := 0.
-template <typename YT>
-LR_DEV void finalize(float* acc, YT* y, int nb, int d_out, const void* scale, bool f16) {
-  const int n = nb * d_out;
-  for (int i = threadIdx.x * 8; i < n; i += kThreads * 8) {
-    const int k = i % d_out;
-    float4 v0 = ld_cg_f4(acc + i), v1 = ld_cg_f4(acc + i + 4);
-    float v[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-    if (scale) {
-#pragma unroll
-      for (int e = 0; e < 8; ++e) v[e] *= load_scale(scale, k + e, f16);
+LR_DEV int rows_per_stage(int row_bytes) { return max(1, kStageBytes / row_bytes); }
+
+// Build this CTA's segment list (thread 0 only).
+template <typename WT, int MODE>
+LR_DEV void build_plan(const KParams& K, Plan& pl) {
+  pl.nseg = 0;
+  pl.role = 0;
+  auto add = [&](const void* base, size_t row0, int row_bytes, int rows, int kind, int zrow0, int proj) {
+    if (rows <= 0) return;
+    Seg& g = pl.seg[pl.nseg++];
+    g.src = reinterpret_cast<const unsigned char*>(base) + row0 * size_t(row_bytes);
+    g.row_bytes = row_bytes;
+    g.rows = rows;
+    g.rps = rows_per_stage(row_bytes);
+    g.kind = kind;
+    g.zrow0 = zrow0;
+    g.proj = proj;
+  };
+  if constexpr (MODE == kLinear) {
+    const Rank1Params& P = K.r;
+    int r0, r1;
+    split_range(P.total_rows, blockIdx.x, gridDim.x, &r0, &r1);
+    pl.nrows = r1 - r0;
+    pl.row_base = r0;
+    for (int kind = kDot; kind <= kRank1; ++kind) {
+      for (int p = 0; p < P.n_proj; ++p) {
+        const Rank1Proj& pr = P.proj[p];
+        const int a = max(r0, pr.row_begin), b = min(r1, pr.row_begin + pr.rows);
+        if (a >= b) continue;
+        if (kind == kDot)
+          add(pr.A, size_t(a - pr.row_begin), P.d_in * int(sizeof(WT)), b - a, kDot, a - r0, p);
+        else
+          add(pr.B, size_t(a - pr.row_begin), pr.d_out * int(sizeof(WT)), b - a, kRank1, a - r0, p);
+      }
     }
-    if constexpr (sizeof(YT) == 2) {
-      uint4 o;
-      __nv_bfloat162 h[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) h[e] = __floats2bfloat162_rn(v[2 * e], v[2 * e + 1]);
-      o.x = *reinterpret_cast<uint32_t*>(&h[0]); o.y = *reinterpret_cast<uint32_t*>(&h[1]);
-      o.z = *reinterpret_cast<uint32_t*>(&h[2]); o.w = *reinterpret_cast<uint32_t*>(&h[3]);
-      *reinterpret_cast<uint4*>(y + i) = o;
+  } else if constexpr (MODE == kFfn1) {
+    const FfnParams& F = K.f;
+    if (int(blockIdx.x) < K.g_lr) {
+      int r0, r1;
+      split_range(F.rank, blockIdx.x, K.g_lr, &r0, &r1);
+      pl.nrows = r1 - r0;
+      pl.row_base = r0;
+      add(F.A, size_t(r0), F.hidden, r1 - r0, kDot, 0, 0);
+      add(F.B, size_t(r0), 2 * F.n_lr, r1 - r0, kRank1, 0, 0);
     } else {
-      *reinterpret_cast<float4*>(y + i) = make_float4(v[0], v[1], v[2], v[3]);
-      *reinterpret_cast<float4*>(y + i + 4) = make_float4(v[4], v[5], v[6], v[7]);
+      int p0, p1;
+      split_range(F.n_dense, blockIdx.x - K.g_lr, gridDim.x - K.g_lr, &p0, &p1);
+      pl.role = 1;
+      pl.nrows = 2 * (p1 - p0);
+      pl.row_base = 2 * p0;
+      add(F.D, size_t(2 * p0), F.hidden, 2 * (p1 - p0), kDot, 0, 0);
     }
-    const float4 zero = make_float4(0.f, 0.f, 0.f, 0.f);
-    st_cg_f4(acc + i, zero);
-    st_cg_f4(acc + i + 4, zero);
+  } else {
+    const FfnParams& F = K.f;
+    int c0, c1;
+    split_range(F.inter, blockIdx.x, gridDim.x, &c0, &c1);
+    pl.nrows = c1 - c0;
+    pl.row_base = c0;
+    add(F.Wd, size_t(c0), F.hidden, c1 - c0, kRank1, 0, 0);
   }
 }
 
-LR_DEV void block_rows(int total, int* r0, int* r1) {
-  *r0 = int((long long)total * blockIdx.x / gridDim.x);
-  *r1 = int((long long)total * (blockIdx.x + 1) / gridDim.x);
+// Scale of CTA-local row r after phase A (per latent / output channel).
+template <int MODE>
+LR_DEV float row_scale(const KParams& K, const Plan& pl, int r) {
+  const bool f16 = (MODE == kLinear ? K.r.scale_f16 : K.f.scale_f16) != 0;
+  if constexpr (MODE == kLinear) {
+    for (int s = 0; s < pl.nseg; ++s) {
+      const Seg& g = pl.seg[s];
+      if (g.kind == kDot && r >= g.zrow0 && r < g.zrow0 + g.rows) {
+        const Rank1Proj& pr = K.r.proj[g.proj];
+        return pr.sA ? load_scale(pr.sA, pl.row_base + r - pr.row_begin, f16) : 1.f;
+      }
+    }
+    return 1.f;
+  } else {
+    if (pl.role == 0) return load_scale(K.f.sA, pl.row_base + r, f16);
+    return load_scale(K.f.sD, pl.row_base + r, f16);
+  }
 }
 
-// ---------------------------------------------------------------------------
-// Factorised linear (grouped): one launch for up to kMaxGroup projections.
-// ---------------------------------------------------------------------------
-template <typename WT, typename XT, typename YT, int NB>
-__global__ void __launch_bounds__(kThreads, 1) lr_rank1_kernel(const __grid_constant__ Rank1Params P) {
-  extern __shared__ __align__(16) unsigned char smem_raw[];
-  int r0, r1;
-  block_rows(P.total_rows, &r0, &r1);
-  const int nr = r1 - r0;
-  float* part = reinterpret_cast<float*>(smem_raw);
-  float* zs = part + size_t(nr) * kWarps * NB;
-  const WT** arow = reinterpret_cast<const WT**>(zs + size_t(nr) * NB + (nr & 1) * NB);
-  int* srow = reinterpret_cast<int*>(arow + nr);
-  __shared__ int s_proj_of_row[kMaxRowsCta];
+template <typename WT, typename XT, typename YT, int NB, int LPW, int MODE>
+__global__ void __launch_bounds__(kThreads, (NB <= 1 && LPW <= 2 ? 2 : 1)) stream_kernel(const __grid_constant__ KParams K) {
+  extern __shared__ __align__(128) unsigned char smem[];
+  __shared__ Plan pl;
+  __shared__ __align__(8) uint64_t full[kMaxStages];
+  __shared__ __align__(8) uint64_t empty[kMaxStages];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const Layout L = layout_for<NB>(K.stages, K.x_elems, int(sizeof(XT)), K.rows_cap);
+  unsigned char* ring = smem;
+  XT* xs = reinterpret_cast<XT*>(smem + L.x);
+  float* part = reinterpret_cast<float*>(smem + L.part);
+  float* zs = reinterpret_cast<float*>(smem + L.z);
 
   pdl_launch_dependents();
-  for (int i = threadIdx.x; i < nr; i += kThreads) {
-    const int g = r0 + i;
-    int p = 0;
+  if (threadIdx.x == 0) {
+    build_plan<WT, MODE>(K, pl);
+    for (int s = 0; s < K.stages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], kConsumerWarps);
+    }
+    fence_mbar_init();
+  }
+  __syncthreads();
+
+  if (warp == kConsumerWarps) {
+    // weights are never written by an earlier kernel: no dependency wait here
+    if (lane == 0) produce(pl, ring, full, empty, K.stages, K.err);
+  } else {
+    const int cw = warp;
+    const int nb = (MODE == kLinear) ? K.r.nb : K.f.nb;
+    pdl_wait();
+    if constexpr (MODE != kFfn2) {
+      const uint4* xg = reinterpret_cast<const uint4*>(MODE == kLinear ? K.r.x : K.f.x);
+      const int n16 = int(size_t(NB) * K.x_elems * sizeof(XT) / 16);
+      const int valid16 = int(size_t(nb) * K.x_elems * sizeof(XT) / 16);
+      for (int i = threadIdx.x; i < n16; i += kConsumers)
+        reinterpret_cast<uint4*>(xs)[i] = i < valid16 ? xg[i] : make_uint4(0u, 0u, 0u, 0u);
+    } else {
+      const FfnParams& F = K.f;
+      const bool f16 = F.scale_f16 != 0;
+      const int two_n = 2 * F.n_lr;
+      for (int i = threadIdx.x; i < pl.nrows * NB; i += kConsumers) {
+        const int r = i / NB, b = i % NB, ch = pl.row_base + r;
+        float h = 0.f;
+        if (b < nb) {
+          if (ch < F.n_lr) {
+            float* gp = F.gu_acc + size_t(b) * two_n + 2 * ch;
+            float g, u;
+            asm volatile("ld.global.cg.f32 %0, [%1];" : "=f"(g) : "l"(gp) : "memory");
+            asm volatile("ld.global.cg.f32 %0, [%1];" : "=f"(u) : "l"(gp + 1) : "memory");
+            g *= load_scale(F.sB, 2 * ch, f16);
+            u *= load_scale(F.sB, 2 * ch + 1, f16);
+            h = silu(g) * u;
+            asm volatile("st.global.cg.f32 [%0], %1;" :: "l"(gp), "f"(0.f) : "memory");
+            asm volatile("st.global.cg.f32 [%0], %1;" :: "l"(gp + 1), "f"(0.f) : "memory");
+          } else {
+            h = F.h_dense[size_t(b) * F.n_dense + (ch - F.n_lr)];
+          }
+        }
+        zs[r * NB + b] = h;
+      }
+    }
+    consumer_sync();
+
+    // this warp's x chunk, when each warp owns a single line of every row
+    float xr[NB][8];
+    const bool x_in_regs = NB <= 2 && MODE != kFfn2 && (K.x_elems + kLineElems - 1) / kLineElems <= kConsumerWarps;
 #pragma unroll
-    for (int q = 1; q < kMaxGroup; ++q)
-      if (q < P.n_proj && g >= P.proj[q].row_begin) p = q;
-    const int j = g - P.proj[p].row_begin;
-    arow[i] = reinterpret_cast<const WT*>(P.proj[p].A) + size_t(j) * P.d_in;
-    srow[i] = j;
-    s_proj_of_row[i] = p;
-  }
-  __syncthreads();
-  // Weights are never written by an earlier kernel: start their DRAM reads
-  // before waiting for the producer of x.
-  if (threadIdx.x < nr) {
-    const size_t bytes = size_t(P.d_in) * sizeof(WT);
-    if ((bytes & 15) == 0) prefetch_l2_bulk(arow[threadIdx.x], uint32_t(bytes));
-  }
-  pdl_wait();
+    for (int b = 0; b < NB; ++b)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) xr[b][e] = 0.f;
+    if constexpr (MODE != kFfn2) {
+      const int col = cw * kLineElems + lane * 8;
+      if (x_in_regs && col < K.x_elems) {
+#pragma unroll
+        for (int b = 0; b < NB; ++b)
+          SChunk<XT>::load(reinterpret_cast<const unsigned char*>(xs + size_t(b) * K.x_elems + col), xr[b]);
+      }
+    }
 
-  phase_dot<WT, XT, NB>(arow, nr, P.d_in, reinterpret_cast<const XT*>(P.x), P.nb, part);
-  __syncthreads();
-  // scale of A depends on the row's projection; all projections share scale dtype
-  for (int i = threadIdx.x; i < nr * NB; i += kThreads) {
-    const int r = i / NB, b = i % NB;
-    float s = 0.f;
+    float acc[LPW][NB][8];
+#pragma unroll
+    for (int li = 0; li < LPW; ++li)
+#pragma unroll
+      for (int b = 0; b < NB; ++b)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[li][b][e] = 0.f;
+    bool zready = (MODE == kFfn2), failed = false;
+    int st = 0;
+    for (int s = 0; s < pl.nseg; ++s) {
+      const Seg& g = pl.seg[s];
+      if (g.kind == kRank1 && !zready) {
+        consumer_sync();
+        for (int i = threadIdx.x; i < pl.nrows * NB; i += kConsumers) {
+          const int r = i / NB, b = i % NB;
+          float v = 0.f;
 #pragma unroll 4
-    for (int w = 0; w < kWarps; ++w) s += part[r * kWarps * NB + w * NB + b];
-    const void* sA = P.proj[s_proj_of_row[r]].sA;
-    if (sA) s *= load_scale(sA, srow[r], P.scale_f16 != 0);
-    zs[r * NB + b] = s;
+          for (int w = 0; w < kConsumerWarps; ++w) v += part[(r * kConsumerWarps + w) * NB + b];
+          zs[r * NB + b] = v * row_scale<MODE>(K, pl, r);
+        }
+        consumer_sync();
+        zready = true;
+      }
+      const int elems = g.row_bytes / int(sizeof(WT));
+      for (int r = 0; r < g.rows; r += g.rps) {
+        const int k = min(g.rps, g.rows - r);
+        const int slot = st % K.stages, round = st / K.stages;
+        if (!failed && !mbar_wait_bounded(&full[slot], uint32_t(round) & 1u, K.err)) failed = true;
+        if (!failed) {
+          const unsigned char* stage = ring + size_t(slot) * kStageBytes;
+          if (g.kind == kDot)
+            consume_dot<WT, XT, NB>(stage, k, elems, xs, xr, x_in_regs, part, g.zrow0 + r, cw, lane);
+          else consume_rank1<WT, NB, LPW>(stage, k, elems, zs, g.zrow0 + r, acc, cw, lane);
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[slot]);
+        ++st;
+      }
+      if (g.kind == kRank1 && !failed) {
+        float* dst;
+        if constexpr (MODE == kLinear) dst = K.r.proj[g.proj].acc;
+        else if constexpr (MODE == kFfn1) dst = K.f.gu_acc;
+        else dst = K.f.y_acc;
+        flush_rank1<NB, LPW>(acc, dst, elems, nb, cw, lane);
+      }
+    }
+    if constexpr (MODE == kFfn1) {
+      if (pl.role == 1) {
+        // dense branch: g, u of each channel pair, SwiGLU, h_D
+        consumer_sync();
+        for (int i = threadIdx.x; i < pl.nrows * NB; i += kConsumers) {
+          const int r = i / NB, b = i % NB;
+          float v = 0.f;
+#pragma unroll 4
+          for (int w = 0; w < kConsumerWarps; ++w) v += part[(r * kConsumerWarps + w) * NB + b];
+          zs[r * NB + b] = v * row_scale<MODE>(K, pl, r);
+        }
+        consumer_sync();
+        const FfnParams& F = K.f;
+        for (int i = threadIdx.x; i < (pl.nrows / 2) * NB; i += kConsumers) {
+          const int pp = i / NB, b = i % NB;
+          if (b < nb) {
+            const float g = zs[(2 * pp) * NB + b], u = zs[(2 * pp + 1) * NB + b];
+            F.h_dense[size_t(b) * F.n_dense + pl.row_base / 2 + pp] = silu(g) * u;
+          }
+        }
+      }
+    }
   }
-  __syncthreads();
 
-  // phase B over the segments of rows that belong to one projection
-  int sa = 0;
-  while (sa < nr) {
-    const int p = s_proj_of_row[sa];
-    int sb = sa + 1;
-    while (sb < nr && s_proj_of_row[sb] == p) ++sb;
-    const Rank1Proj& pr = P.proj[p];
-    const WT* B0 = reinterpret_cast<const WT*>(pr.B) + size_t(srow[sa]) * pr.d_out;
-    phase_rank1<WT, NB>(B0, pr.d_out, sb - sa, zs + sa * NB, pr.acc, P.nb);
-    sa = sb;
+  if constexpr (MODE == kFfn1) {
+    return;
+  } else {
+    unsigned int* words = (MODE == kLinear) ? K.r.ticket : K.f.ticket;
+    grid_barrier(words, K.err);
+    if constexpr (MODE == kLinear) {
+      FinalTarget t[kMaxGroup];
+#pragma unroll
+      for (int p = 0; p < kMaxGroup; ++p)
+        t[p] = FinalTarget{K.r.proj[p].acc, K.r.proj[p].y, K.r.proj[p].sB, K.r.nb * K.r.proj[p].d_out,
+                           K.r.proj[p].d_out};
+      finalize_slice<YT, kMaxGroup>(t, K.r.n_proj, K.r.scale_f16 != 0);
+    } else {
+      FinalTarget t[1] = {FinalTarget{K.f.y_acc, K.f.y, K.f.sd, K.f.nb * K.f.hidden, K.f.hidden}};
+      finalize_slice<__nv_bfloat16, 1>(t, 1, K.f.scale_f16 != 0);
+    }
   }
-
-  if (!last_cta_arrives(P.ticket)) return;
-  for (int p = 0; p < P.n_proj; ++p)
-    finalize<YT>(P.proj[p].acc, reinterpret_cast<YT*>(P.proj[p].y), P.nb, P.proj[p].d_out, P.proj[p].sB,
-                 P.scale_f16 != 0);
-  if (threadIdx.x == 0) *P.ticket = 0u;
 }
 
-template <typename WT, typename XT, typename YT, int NB>
-cudaError_t launch_rank1_t(const Rank1Params& p, int sm_count, cudaStream_t s) {
-  int grid = sm_count;
-  if (grid > p.total_rows) grid = p.total_rows;
-  const int need = (p.total_rows + kMaxRowsCta - 1) / kMaxRowsCta;
-  if (grid < need) grid = need;
-  const int rows_max = (p.total_rows + grid - 1) / grid;
-  const size_t smem = SmemLayout::bytes(rows_max, NB);
-  auto kern = lr_rank1_kernel<WT, XT, YT, NB>;
-  cudaError_t e = ensure_smem(kern, smem);
+// ---------------------------------------------------------------------------
+// Chains of grouped factorised linears: one persistent CTA per SM.
+//
+// The producer warp streams the factor rows of every step back to back; it
+// never waits for a step boundary, so the loads of step s+1 are in flight
+// while step s finishes.  Consumers, per step: stage the step's input x (fp32)
+// in shared memory, run phase A and phase B on the CTA's latent rows, add the
+// partial outputs into accumulator set s % 3, then meet at a grid barrier
+// (bounded spin; the grid is one CTA per SM, all resident).  After it each
+// CTA writes its slice of the step's outputs and zeroes its slice of set
+// (s-1) % 3, which step s read as its input and nobody reads again.
+// ---------------------------------------------------------------------------
+constexpr int kChainStagesMax = 6;
+int lpw_for(int d_out);
+
+struct ChainLayout {
+  size_t x, part, z, total;
+};
+
+template <int NB>
+LR_HD_INLINE ChainLayout chain_layout(int stages, int x_elems, int rows_cap) {
+  ChainLayout L;
+  L.x = size_t(stages) * kStageBytes;
+  L.part = L.x + round16(size_t(NB) * x_elems * 4);
+  L.z = L.part + round16(size_t(rows_cap) * kConsumerWarps * NB * 4);
+  L.total = L.z + round16(size_t(rows_cap) * NB * 4);
+  return L;
+}
+
+// Segments of step `st` owned by this CTA, in streaming order: all A rows
+// (kind kDot) then all B rows (kind kRank1).
+// f(proj, kind, src, row_bytes, rows, zrow0, j0)
+template <typename WT, class F>
+LR_DEV void for_each_segment(const ChainStep& st, F&& f) {
+  int r0, r1;
+  split_range(st.total_rows, blockIdx.x, gridDim.x, &r0, &r1);
+  for (int kind = kDot; kind <= kRank1; ++kind) {
+    int begin = 0;
+    for (int p = 0; p < st.n; ++p) {
+      const ChainProj& pr = st.p[p];
+      const int a = max(r0, begin), b = min(r1, begin + pr.rows);
+      if (a < b) {
+        const int j0 = a - begin;
+        if (kind == kDot)
+          f(p, kDot, reinterpret_cast<const unsigned char*>(pr.A) + size_t(j0) * st.d_in * sizeof(WT),
+            st.d_in * int(sizeof(WT)), b - a, a - r0, j0);
+        else
+          f(p, kRank1, reinterpret_cast<const unsigned char*>(pr.B) + size_t(j0) * pr.d_out * sizeof(WT),
+            pr.d_out * int(sizeof(WT)), b - a, a - r0, j0);
+      }
+      begin += pr.rows;
+    }
+  }
+}
+
+LR_DEV int step_rows(const ChainStep& st) {
+  int r0, r1;
+  split_range(st.total_rows, blockIdx.x, gridDim.x, &r0, &r1);
+  return r1 - r0;
+}
+
+LR_DEV int acc_offset(const ChainStep& st, int p, int nb) {
+  int o = 0;
+  for (int q = 0; q < p; ++q) o += nb * st.p[q].d_out;
+  return o;
+}
+
+LR_DEV int acc_used(const ChainStep& st, int nb) { return acc_offset(st, st.n, nb); }
+
+template <typename WT>
+LR_DEV void chain_produce(const ChainParams& P, unsigned char* ring, uint64_t* full, uint64_t* empty, int stages) {
+  int st = 0;
+  bool ok = true;
+  for (int s = 0; s < P.n_steps && ok; ++s) {
+    for_each_segment<WT>(P.step[s], [&](int, int, const unsigned char* src, int row_bytes, int rows, int, int) {
+      const int rps = rows_per_stage(row_bytes);
+      for (int r = 0; r < rows && ok; r += rps) {
+        const int k = min(rps, rows - r);
+        const int slot = st % stages, round = st / stages;
+        if (round > 0 && !mbar_wait_bounded(&empty[slot], uint32_t(round - 1) & 1u, P.err)) {
+          ok = false;
+          return;
+        }
+        const uint32_t bytes = uint32_t(k) * uint32_t(row_bytes);
+        mbar_arrive_expect_tx(&full[slot], bytes);
+        bulk_g2s(ring + size_t(slot) * kStageBytes, src + size_t(r) * row_bytes, bytes, &full[slot]);
+        ++st;
+      }
+    });
+  }
+}
+
+// Grid barrier among the consumer threads of every CTA.  words[0] counts
+// arrivals over the whole launch; barrier k is passed once it reaches
+// gridDim.x * (k + 1).  Bounded: gives up after ~2^22 polls, setting the
+// device error word.
+LR_DEV void consumer_grid_barrier(unsigned int* words, unsigned int target, int* err) {
+  __threadfence();
+  consumer_sync();
+  if (threadIdx.x == 0) {
+    atomicAdd(words, 1u);
+    uint32_t i = 0;
+    while (ld_acquire_u32(words) < target) {
+      if (++i > (1u << 22)) {
+        set_device_error(err, kErrGridBarrier);
+        break;
+      }
+      __nanosleep(20);
+    }
+  }
+  consumer_sync();
+  __threadfence();
+}
+
+template <typename WT, int NB, int LPW>
+__global__ void __launch_bounds__(kThreads, 1) chain_kernel(const __grid_constant__ ChainParams P, int stages,
+                                                            int rows_cap, int x_elems_max) {
+  using XT = typename std::conditional<sizeof(WT) == 4, float, __nv_bfloat16>::type;
+  using YT = XT;
+  extern __shared__ __align__(128) unsigned char smem[];
+  __shared__ __align__(8) uint64_t full[kChainStagesMax];
+  __shared__ __align__(8) uint64_t empty[kChainStagesMax];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const ChainLayout L = chain_layout<NB>(stages, x_elems_max, rows_cap);
+  unsigned char* ring = smem;
+  float* xs = reinterpret_cast<float*>(smem + L.x);
+  float* part = reinterpret_cast<float*>(smem + L.part);
+  float* zs = reinterpret_cast<float*>(smem + L.z);
+  const bool f16 = P.scale_f16 != 0;
+  const int nb = P.nb;
+
+  pdl_launch_dependents();
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < stages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], kConsumerWarps);
+    }
+    fence_mbar_init();
+  }
+  __syncthreads();
+
+  if (warp == kConsumerWarps) {
+    if (lane == 0) chain_produce<WT>(P, ring, full, empty, stages);
+  } else {
+    const int cw = warp;
+    pdl_wait();
+    int st = 0;
+    bool failed = false;
+    for (int s = 0; s < P.n_steps; ++s) {
+      const ChainStep& S = P.step[s];
+      // ---- stage this step's input (fp32) ----
+      {
+        const int n = nb * S.d_in;
+        const int set_prev = (s + 2) % 3;
+        for (int i = threadIdx.x * 4; i < NB * S.d_in; i += kConsumers * 4) {
+          float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+          if (i < n) {
+            if (S.input_step < 0) {
+              const XT* xg = reinterpret_cast<const XT*>(P.x) + i;
+              if constexpr (sizeof(XT) == 4) {
+                v = *reinterpret_cast<const float4*>(xg);
+              } else {
+                const uint2 u = *reinterpret_cast<const uint2*>(xg);
+                v = make_float4(__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xffff0000u),
+                                __uint_as_float(u.y << 16), __uint_as_float(u.y & 0xffff0000u));
+              }
+            } else if (S.input_step == s - 1) {
+              const ChainStep& I = P.step[S.input_step];
+              const float* a = P.acc + size_t(set_prev) * P.acc_set + acc_offset(I, S.input_proj, nb) + i;
+              v = ld_cg_f4(a);
+              const void* sB = I.p[S.input_proj].sB;
+              if (sB) {
+                const int k = i % S.d_in;
+                v.x *= load_scale(sB, k, f16); v.y *= load_scale(sB, k + 1, f16);
+                v.z *= load_scale(sB, k + 2, f16); v.w *= load_scale(sB, k + 3, f16);
+              }
+            } else {
+              const YT* yg = reinterpret_cast<const YT*>(P.step[S.input_step].p[S.input_proj].y) + i;
+              if constexpr (sizeof(YT) == 4) {
+                v = ld_cg_f4(reinterpret_cast<const float*>(yg));
+              } else {
+                uint2 u;
+                asm volatile("ld.global.cg.v2.u32 {%0,%1}, [%2];" : "=r"(u.x), "=r"(u.y) : "l"(yg) : "memory");
+                v = make_float4(__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xffff0000u),
+                                __uint_as_float(u.y << 16), __uint_as_float(u.y & 0xffff0000u));
+              }
+            }
+          }
+          *reinterpret_cast<float4*>(xs + i) = v;
+        }
+      }
+      consumer_sync();
+      float xr[NB][8];
+      const bool x_in_regs = NB <= 2 && (S.d_in + kLineElems - 1) / kLineElems <= kConsumerWarps;
+#pragma unroll
+      for (int b = 0; b < NB; ++b)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) xr[b][e] = 0.f;
+      {
+        const int col = cw * kLineElems + lane * 8;
+        if (x_in_regs && col < S.d_in) {
+#pragma unroll
+          for (int b = 0; b < NB; ++b)
+            SChunk<float>::load(reinterpret_cast<const unsigned char*>(xs + size_t(b) * S.d_in + col), xr[b]);
+        }
+      }
+      // ---- phase A then phase B over this CTA's rows of the step ----
+      float acc[LPW][NB][8];
+#pragma unroll
+      for (int li = 0; li < LPW; ++li)
+#pragma unroll
+        for (int b = 0; b < NB; ++b)
+#pragma unroll
+          for (int e = 0; e < 8; ++e) acc[li][b][e] = 0.f;
+      bool zready = false;
+      const int nrows = step_rows(S);
+      float* acc_set = P.acc + size_t(s % 3) * P.acc_set;
+      for_each_segment<WT>(S, [&](int p, int kind, const unsigned char*, int row_bytes, int rows, int zrow0, int) {
+        if (kind == kRank1 && !zready) {
+          consumer_sync();
+          for (int i = threadIdx.x; i < nrows * NB; i += kConsumers) {
+            const int r = i / NB, b = i % NB;
+            float v = 0.f;
+#pragma unroll 4
+            for (int w = 0; w < kConsumerWarps; ++w) v += part[(r * kConsumerWarps + w) * NB + b];
+            // scale of A for local row r: find its A segment
+            float sc = 1.f;
+            for_each_segment<WT>(S, [&](int q, int kq, const unsigned char*, int, int rq, int z0, int j0) {
+              if (kq == kDot && r >= z0 && r < z0 + rq && S.p[q].sA) sc = load_scale(S.p[q].sA, j0 + (r - z0), f16);
+            });
+            zs[r * NB + b] = v * sc;
+          }
+          consumer_sync();
+          zready = true;
+        }
+        const int elems = row_bytes / int(sizeof(WT));
+        const int rps = rows_per_stage(row_bytes);
+        for (int r = 0; r < rows; r += rps) {
+          const int k = min(rps, rows - r);
+          const int slot = st % stages, round = st / stages;
+          if (!failed && !mbar_wait_bounded(&full[slot], uint32_t(round) & 1u, P.err)) failed = true;
+          if (!failed) {
+            const unsigned char* stage = ring + size_t(slot) * kStageBytes;
+            if (kind == kDot)
+              consume_dot<WT, float, NB>(stage, k, elems, xs, xr, x_in_regs, part, zrow0 + r, cw, lane);
+            else
+              consume_rank1<WT, NB, LPW>(stage, k, elems, zs, zrow0 + r, acc, cw, lane);
+          }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&empty[slot]);
+          ++st;
+        }
+        if (kind == kRank1 && !failed) flush_rank1<NB, LPW>(acc, acc_set + acc_offset(S, p, nb), elems, nb, cw, lane);
+      });
+      // ---- all partial outputs of step s are in: write them, retire set s-1 ----
+      consumer_grid_barrier(P.bar, gridDim.x * unsigned(s + 1), P.err);
+      {
+        const int total = acc_used(S, nb) / 8;
+        const int c0 = int((long long)total * blockIdx.x / gridDim.x);
+        const int c1 = int((long long)total * (blockIdx.x + 1) / gridDim.x);
+        const bool last = s == P.n_steps - 1;
+        for (int c = c0 + int(threadIdx.x); c < c1; c += kConsumers) {
+          int off = c * 8, p = 0;
+          while (p < S.n - 1 && off >= nb * S.p[p].d_out) { off -= nb * S.p[p].d_out; ++p; }
+          const ChainProj& pr = S.p[p];
+          float* a = acc_set + acc_offset(S, p, nb) + off;
+          const float4 v0 = ld_cg_f4(a), v1 = ld_cg_f4(a + 4);
+          float v[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+          if (pr.sB) {
+            const int k = off % pr.d_out;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) v[e] *= load_scale(pr.sB, k + e, f16);
+          }
+          YT* y = reinterpret_cast<YT*>(pr.y) + off;
+          if constexpr (sizeof(YT) == 2) {
+            uint4 o;
+            uint32_t* ow = reinterpret_cast<uint32_t*>(&o);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * e], v[2 * e + 1]);
+              ow[e] = *reinterpret_cast<uint32_t*>(&h);
+            }
+            *reinterpret_cast<uint4*>(y) = o;
+          } else {
+            *reinterpret_cast<float4*>(y) = make_float4(v[0], v[1], v[2], v[3]);
+            *reinterpret_cast<float4*>(y + 4) = make_float4(v[4], v[5], v[6], v[7]);
+          }
+          if (last) {
+            st_cg_f4(a, make_float4(0.f, 0.f, 0.f, 0.f));
+            st_cg_f4(a + 4, make_float4(0.f, 0.f, 0.f, 0.f));
+          }
+        }
+        if (s >= 1) {
+          const ChainStep& Sp = P.step[s - 1];
+          float* prev = P.acc + size_t((s + 2) % 3) * P.acc_set;
+          const int tp = acc_used(Sp, nb) / 8;
+          const int d0 = int((long long)tp * blockIdx.x / gridDim.x);
+          const int d1 = int((long long)tp * (blockIdx.x + 1) / gridDim.x);
+          for (int c = d0 + int(threadIdx.x); c < d1; c += kConsumers) {
+            st_cg_f4(prev + c * 8, make_float4(0.f, 0.f, 0.f, 0.f));
+            st_cg_f4(prev + c * 8 + 4, make_float4(0.f, 0.f, 0.f, 0.f));
+          }
+        }
+      }
+    }
+  }
+  // ---- leave the barrier counters at zero for the next launch ----
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    const unsigned prev = atomicAdd(P.bar + 1, 1u);
+    if (prev == gridDim.x - 1) {
+      atomicExch(P.bar, 0u);
+      atomicExch(P.bar + 1, 0u);
+    }
+  }
+}
+
+template <typename WT, int NB, int LPW>
+cudaError_t launch_chain_t(const ChainParams& p, int grid, int rows_cap, int x_elems_max, cudaStream_t s) {
+  int stages = kChainStagesMax;
+  size_t bytes = 0;
+  for (; stages >= 2; --stages) {
+    bytes = chain_layout<NB>(stages, x_elems_max, rows_cap).total;
+    if (bytes <= kSmemLimit - 2048) break;
+  }
+  if (bytes > kSmemLimit - 2048) return cudaErrorInvalidValue;
+  auto kern = chain_kernel<WT, NB, LPW>;
+  cudaError_t e = ensure_smem(kern, bytes);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = smem;
+  cfg.dynamicSmemBytes = bytes;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, p);
+  return cudaLaunchKernelEx(&cfg, kern, p, stages, rows_cap, x_elems_max);
 }
 
-template <typename WT, typename XT, typename YT>
-cudaError_t launch_rank1_nb(const Rank1Params& p, int sm_count, cudaStream_t s) {
-  if (p.nb <= 1) return launch_rank1_t<WT, XT, YT, 1>(p, sm_count, s);
-  if (p.nb <= 2) return launch_rank1_t<WT, XT, YT, 2>(p, sm_count, s);
-  if (p.nb <= 4) return launch_rank1_t<WT, XT, YT, 4>(p, sm_count, s);
-  return launch_rank1_t<WT, XT, YT, 8>(p, sm_count, s);
+template <typename WT>
+cudaError_t launch_chain_w(const ChainParams& p, int sm_count, cudaStream_t s) {
+  int max_dout = 0, x_max = 0, max_rows = 0;
+  for (int i = 0; i < p.n_steps; ++i) {
+    const ChainStep& st = p.step[i];
+    x_max = std::max(x_max, st.d_in);
+    max_rows = std::max(max_rows, st.total_rows);
+    for (int q = 0; q < st.n; ++q) max_dout = std::max(max_dout, st.p[q].d_out);
+    if (size_t(st.d_in) * sizeof(WT) > size_t(kStageBytes)) return cudaErrorInvalidValue;
+  }
+  if (size_t(max_dout) * sizeof(WT) > size_t(kStageBytes)) return cudaErrorInvalidValue;
+  const int lpw = lpw_for(max_dout);
+  const int grid = std::min(sm_count, std::max(max_rows, 1));
+  const int rows_cap = (max_rows + grid - 1) / grid;
+  const int nb = p.nb;
+#define LR_CCASE(NB_, LPW_) \
+  if (lpw == LPW_ && nb <= NB_) return launch_chain_t<WT, NB_, LPW_>(p, grid, rows_cap, x_max, s);
+  LR_CCASE(1, 1) LR_CCASE(2, 1) LR_CCASE(4, 1) LR_CCASE(8, 1)
+  LR_CCASE(1, 2) LR_CCASE(2, 2) LR_CCASE(4, 2)
+  LR_CCASE(1, 4) LR_CCASE(2, 4)
+  LR_CCASE(1, 8)
+#undef LR_CCASE
+  return cudaErrorInvalidValue;
 }
 
 // ---------------------------------------------------------------------------
-// Hybrid SwiGLU FFN.
+// Launch helpers
 // ---------------------------------------------------------------------------
-template <int NB>
-__global__ void __launch_bounds__(kThreads, 1) ffn_phase1_kernel(const __grid_constant__ FfnParams P, int g_lr) {
-  extern __shared__ __align__(16) unsigned char smem_raw[];
-  const bool f16 = P.scale_f16 != 0;
-  const __nv_bfloat16* x = reinterpret_cast<const __nv_bfloat16*>(P.x);
-  pdl_launch_dependents();
-  if (int(blockIdx.x) < g_lr) {
-    // low-rank branch: rows of A' (latent channels) then rows of B'
-    const int r0 = int((long long)P.rank * blockIdx.x / g_lr), r1 = int((long long)P.rank * (blockIdx.x + 1) / g_lr);
-    const int nr = r1 - r0;
-    float* part = reinterpret_cast<float*>(smem_raw);
-    float* zs = part + size_t(nr) * kWarps * NB;
-    const int8_t** arow = reinterpret_cast<const int8_t**>(zs + size_t(nr) * NB + (nr & 1) * NB);
-    int* srow = reinterpret_cast<int*>(arow + nr);
-    for (int i = threadIdx.x; i < nr; i += kThreads) {
-      arow[i] = P.A + size_t(r0 + i) * P.hidden;
-      srow[i] = r0 + i;
+template <typename WT, typename XT, typename YT, int NB, int LPW, int MODE>
+cudaError_t launch_stream(KParams K, int grid, cudaStream_t s) {
+  // Three stages when that lets two CTAs share an SM (the next kernel's
+  // producer then streams during this kernel's tail); otherwise the most
+  // stages that fit.
+  size_t bytes = layout_for<NB>(3, K.x_elems, int(sizeof(XT)), K.rows_cap).total;
+  K.stages = 3;
+  if (bytes > kCoResidentSmem) {
+    for (K.stages = kMaxStages; K.stages >= 2; --K.stages) {
+      bytes = layout_for<NB>(K.stages, K.x_elems, int(sizeof(XT)), K.rows_cap).total;
+      if (bytes <= kSmemLimit - 2048) break;
     }
-    __syncthreads();
-    if (threadIdx.x < nr && (P.hidden & 15) == 0) prefetch_l2_bulk(arow[threadIdx.x], uint32_t(P.hidden));
-    pdl_wait();
-    phase_dot<int8_t, __nv_bfloat16, NB>(arow, nr, P.hidden, x, P.nb, part);
-    __syncthreads();
-    reduce_parts<NB>(part, nr, zs, P.sA, srow, f16);
-    __syncthreads();
-    phase_rank1<int8_t, NB>(P.B + size_t(r0) * (2 * P.n_lr), 2 * P.n_lr, nr, zs, P.gu_acc, P.nb);
-  } else {
-    // dense branch: row pairs (gate_c, up_c) of D, SwiGLU in the epilogue
-    const int gd = gridDim.x - g_lr, c = blockIdx.x - g_lr;
-    const int p0 = int((long long)P.n_dense * c / gd), p1 = int((long long)P.n_dense * (c + 1) / gd);
-    const int nr = 2 * (p1 - p0);
-    float* part = reinterpret_cast<float*>(smem_raw);
-    float* zs = part + size_t(nr) * kWarps * NB;
-    const int8_t** arow = reinterpret_cast<const int8_t**>(zs + size_t(nr) * NB);
-    int* srow = reinterpret_cast<int*>(arow + nr);
-    for (int i = threadIdx.x; i < nr; i += kThreads) {
-      arow[i] = P.D + size_t(2 * p0 + i) * P.hidden;
-      srow[i] = 2 * p0 + i;
-    }
-    __syncthreads();
-    if (threadIdx.x < nr && (P.hidden & 15) == 0) prefetch_l2_bulk(arow[threadIdx.x], uint32_t(P.hidden));
-    pdl_wait();
-    phase_dot<int8_t, __nv_bfloat16, NB>(arow, nr, P.hidden, x, P.nb, part);
-    __syncthreads();
-    reduce_parts<NB>(part, nr, zs, P.sD, srow, f16);
-    __syncthreads();
-    for (int i = threadIdx.x; i < (p1 - p0) * NB; i += kThreads) {
-      const int pp = i / NB, b = i % NB;
-      if (b < P.nb) {
-        const float g = zs[(2 * pp) * NB + b], u = zs[(2 * pp + 1) * NB + b];
-        P.h_dense[size_t(b) * P.n_dense + p0 + pp] = silu(g) * u;
-      }
-    }
+    if (bytes > kSmemLimit - 2048) return cudaErrorInvalidValue;
   }
-}
-
-template <int NB>
-__global__ void __launch_bounds__(kThreads, 1) ffn_phase2_kernel(const __grid_constant__ FfnParams P) {
-  extern __shared__ __align__(16) unsigned char smem_raw[];
-  const bool f16 = P.scale_f16 != 0;
-  int c0, c1;
-  block_rows(P.inter, &c0, &c1);
-  const int nr = c1 - c0;
-  float* hs = reinterpret_cast<float*>(smem_raw);  // [nr][NB]
-  pdl_launch_dependents();
-  if (threadIdx.x < nr) {
-    const size_t bytes = size_t(P.hidden);
-    const int8_t* row = P.Wd + size_t(c0 + threadIdx.x) * P.hidden;
-    if ((bytes & 15) == 0) prefetch_l2_bulk(row, uint32_t(bytes));
-  }
-  pdl_wait();
-  const int two_n = 2 * P.n_lr;
-  for (int i = threadIdx.x; i < nr * NB; i += kThreads) {
-    const int r = i / NB, b = i % NB, ch = c0 + r;
-    float h = 0.f;
-    if (b < P.nb) {
-      if (ch < P.n_lr) {
-        float* gp = P.gu_acc + size_t(b) * two_n + 2 * ch;
-        float g, u;
-        asm volatile("ld.global.cg.f32 %0, [%1];" : "=f"(g) : "l"(gp) : "memory");
-        asm volatile("ld.global.cg.f32 %0, [%1];" : "=f"(u) : "l"(gp + 1) : "memory");
-        g *= load_scale(P.sB, 2 * ch, f16);
-        u *= load_scale(P.sB, 2 * ch + 1, f16);
-        h = silu(g) * u;
-        asm volatile("st.global.cg.f32 [%0], %1;" :: "l"(gp), "f"(0.f) : "memory");
-        asm volatile("st.global.cg.f32 [%0], %1;" :: "l"(gp + 1), "f"(0.f) : "memory");
-      } else {
-        h = P.h_dense[size_t(b) * P.n_dense + (ch - P.n_lr)];
-      }
-    }
-    hs[r * NB + b] = h;
-  }
-  __syncthreads();
-  phase_rank1<int8_t, NB>(P.Wd + size_t(c0) * P.hidden, P.hidden, nr, hs, P.y_acc, P.nb);
-  if (!last_cta_arrives(P.ticket)) return;
-  finalize<__nv_bfloat16>(P.y_acc, reinterpret_cast<__nv_bfloat16*>(P.y), P.nb, P.hidden, P.sd, f16);
-  if (threadIdx.x == 0) *P.ticket = 0u;
-}
-
-cudaLaunchConfig_t pdl_config(int grid, size_t smem, cudaStream_t s, cudaLaunchAttribute* attr) {
+  auto kern = stream_kernel<WT, XT, YT, NB, LPW, MODE>;
+  cudaError_t e = ensure_smem(kern, bytes);
+  if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = smem;
+  cfg.dynamicSmemBytes = bytes;
   cfg.stream = s;
+  cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cfg;
+  return cudaLaunchKernelEx(&cfg, kern, K);
 }
 
-template <int NB>
-cudaError_t launch_ffn_t(const FfnParams& p, int sm_count, cudaStream_t s) {
+int lpw_for(int d_out) {
+  const int lines = (d_out + kLineElems - 1) / kLineElems;
+  const int need = (lines + kConsumerWarps - 1) / kConsumerWarps;
+  return need <= 1 ? 1 : need <= 2 ? 2 : need <= 4 ? 4 : need <= 8 ? 8 : 0;
+}
+
+// Pick the (NB, LPW) instantiation: NB is the smallest power of two >= nb
+// with NB * LPW <= 8 (accumulator registers).
+template <typename WT, typename XT, typename YT, int MODE>
+cudaError_t dispatch(const KParams& K, int nb, int lpw, int grid, cudaStream_t s) {
+#define LR_CASE(NB_, LPW_) \
+  if (lpw == LPW_ && nb <= NB_) return launch_stream<WT, XT, YT, NB_, LPW_, MODE>(K, grid, s);
+  LR_CASE(1, 1) LR_CASE(2, 1) LR_CASE(4, 1) LR_CASE(8, 1)
+  LR_CASE(1, 2) LR_CASE(2, 2) LR_CASE(4, 2)
+  LR_CASE(1, 4) LR_CASE(2, 4)
+  LR_CASE(1, 8)
+#undef LR_CASE
+  return cudaErrorInvalidValue;
+}
+
+template <typename WT, typename XT, typename YT>
+cudaError_t launch_linear(const Rank1Params& p0, int sm_count, cudaStream_t s) {
+  int max_dout = 0;
+  for (int q = 0; q < p0.n_proj; ++q) max_dout = std::max(max_dout, p0.proj[q].d_out);
+  const int lpw = lpw_for(max_dout);
+  if (lpw == 0) return cudaErrorInvalidValue;
+  if (size_t(p0.d_in) * sizeof(WT) > size_t(kStageBytes) || size_t(max_dout) * sizeof(WT) > size_t(kStageBytes))
+    return cudaErrorInvalidValue;
+  // one CTA per SM at most: the finalize barrier needs every CTA resident
+  const int grid = std::min(sm_count, p0.total_rows);
+  const int nb_max = 8 / lpw;
+  KParams K;
+  std::memset(&K, 0, sizeof(K));
+  K.rows_cap = (p0.total_rows + grid - 1) / grid;
+  K.x_elems = p0.d_in;
+  for (int b0 = 0; b0 < p0.nb; b0 += nb_max) {
+    K.r = p0;
+    K.r.nb = std::min(nb_max, p0.nb - b0);
+    K.r.x = reinterpret_cast<const XT*>(p0.x) + size_t(b0) * p0.d_in;
+    for (int q = 0; q < p0.n_proj; ++q)
+      K.r.proj[q].y = reinterpret_cast<YT*>(p0.proj[q].y) + size_t(b0) * p0.proj[q].d_out;
+    cudaError_t e = dispatch<WT, XT, YT, kLinear>(K, K.r.nb, lpw, grid, s);
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
+cudaError_t launch_ffn_impl(const FfnParams& p0, int sm_count, cudaStream_t s) {
+  const int lpw1 = p0.n_lr > 0 ? lpw_for(2 * p0.n_lr) : 1;
+  const int lpw2 = lpw_for(p0.hidden);
+  if (lpw1 == 0 || lpw2 == 0) return cudaErrorInvalidValue;
+  if (2 * p0.n_lr > kStageBytes || p0.hidden > kStageBytes) return cudaErrorInvalidValue;
   // split phase-1 CTAs between the branches in proportion to their bytes
-  const double lr_bytes = double(p.rank) * (p.hidden + 2.0 * p.n_lr);
-  const double dn_bytes = 2.0 * p.n_dense * p.hidden;
+  const double lr_bytes = double(p0.rank) * (p0.hidden + 2.0 * p0.n_lr);
+  const double dn_bytes = 2.0 * p0.n_dense * p0.hidden;
   int g_lr = 0, g_d = 0;
-  if (p.n_lr > 0 && p.n_dense > 0) {
+  if (p0.n_lr > 0 && p0.n_dense > 0) {
     g_lr = int(sm_count * lr_bytes / (lr_bytes + dn_bytes) + 0.5);
-    if (g_lr < 1) g_lr = 1;
-    if (g_lr > sm_count - 1) g_lr = sm_count - 1;
+    g_lr = std::min(std::max(g_lr, 1), sm_count - 1);
     g_d = sm_count - g_lr;
-  } else if (p.n_lr > 0) {
+  } else if (p0.n_lr > 0) {
     g_lr = sm_count;
   } else {
     g_d = sm_count;
   }
-  if (g_lr > p.rank) g_lr = p.rank;
-  if (g_lr > 0 && (p.rank + g_lr - 1) / g_lr > kMaxRowsCta) g_lr = (p.rank + kMaxRowsCta - 1) / kMaxRowsCta;
-  if (g_d > p.n_dense) g_d = p.n_dense;
-  if (g_d > 0 && 2 * ((p.n_dense + g_d - 1) / g_d) > kMaxRowsCta) g_d = (2 * p.n_dense + kMaxRowsCta - 1) / kMaxRowsCta;
-  const int rows1 = std::max(g_lr ? (p.rank + g_lr - 1) / g_lr : 0, g_d ? 2 * ((p.n_dense + g_d - 1) / g_d) : 0);
-  const size_t smem1 = SmemLayout::bytes(rows1 + 1, NB);
-  cudaLaunchAttribute attr[1];
-  auto k1 = ffn_phase1_kernel<NB>;
-  cudaError_t e = ensure_smem(k1, smem1);
-  if (e != cudaSuccess) return e;
-  cudaLaunchConfig_t c1 = pdl_config(g_lr + g_d, smem1, s, attr);
-  e = cudaLaunchKernelEx(&c1, k1, p, g_lr);
-  if (e != cudaSuccess) return e;
+  if (g_lr > 0) g_lr = std::min(g_lr, p0.rank);
+  if (g_d > 0) g_d = std::min(g_d, p0.n_dense);
+  // one CTA per SM at most: the finalize barrier of phase 2 needs every CTA resident
+  const int g2 = std::min(sm_count, p0.inter);
 
-  int g2 = std::min(sm_count, p.inter);
-  if ((p.inter + g2 - 1) / g2 > kMaxRowsCta) g2 = (p.inter + kMaxRowsCta - 1) / kMaxRowsCta;
-  const size_t smem2 = size_t((p.inter + g2 - 1) / g2) * NB * 4 + 64;
-  auto k2 = ffn_phase2_kernel<NB>;
-  e = ensure_smem(k2, smem2);
-  if (e != cudaSuccess) return e;
-  cudaLaunchConfig_t c2 = pdl_config(g2, smem2, s, attr);
-  return cudaLaunchKernelEx(&c2, k2, p);
+  KParams K1, K2;
+  std::memset(&K1, 0, sizeof(K1));
+  std::memset(&K2, 0, sizeof(K2));
+  K1.g_lr = g_lr;
+  K1.rows_cap = std::max(g_lr ? (p0.rank + g_lr - 1) / g_lr : 0, g_d ? 2 * ((p0.n_dense + g_d - 1) / g_d) : 0);
+  K1.x_elems = p0.hidden;
+  K2.rows_cap = (p0.inter + g2 - 1) / g2;
+  K2.x_elems = 0;
+  const int nb_max = std::min(8 / lpw1, 8 / lpw2);
+  for (int b0 = 0; b0 < p0.nb; b0 += nb_max) {
+    FfnParams f = p0;
+    f.nb = std::min(nb_max, p0.nb - b0);
+    f.x = reinterpret_cast<const __nv_bfloat16*>(p0.x) + size_t(b0) * p0.hidden;
+    f.y = reinterpret_cast<__nv_bfloat16*>(p0.y) + size_t(b0) * p0.hidden;
+    K1.f = f;
+    K2.f = f;
+    cudaError_t e = dispatch<int8_t, __nv_bfloat16, __nv_bfloat16, kFfn1>(K1, f.nb, lpw1, g_lr + g_d, s);
+    if (e != cudaSuccess) return e;
+    e = dispatch<int8_t, __nv_bfloat16, __nv_bfloat16, kFfn2>(K2, f.nb, lpw2, g2, s);
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
 }
 
 }  // namespace
 
 cudaError_t launch_lr_rank1(const Rank1Params& p, lr_dtype_t w_dtype, int sm_count, cudaStream_t s) {
   switch (w_dtype) {
-    case LR_F32: return launch_rank1_nb<float, float, float>(p, sm_count, s);
-    case LR_BF16: return launch_rank1_nb<__nv_bfloat16, __nv_bfloat16, __nv_bfloat16>(p, sm_count, s);
-    case LR_I8: return launch_rank1_nb<int8_t, __nv_bfloat16, __nv_bfloat16>(p, sm_count, s);
+    case LR_F32: return launch_linear<float, float, float>(p, sm_count, s);
+    case LR_BF16: return launch_linear<__nv_bfloat16, __nv_bfloat16, __nv_bfloat16>(p, sm_count, s);
+    case LR_I8: return launch_linear<int8_t, __nv_bfloat16, __nv_bfloat16>(p, sm_count, s);
     default: return cudaErrorInvalidValue;
   }
 }
 
-cudaError_t launch_ffn(const FfnParams& p, int sm_count, cudaStream_t s) {
-  if (p.nb <= 1) return launch_ffn_t<1>(p, sm_count, s);
-  if (p.nb <= 2) return launch_ffn_t<2>(p, sm_count, s);
-  if (p.nb <= 4) return launch_ffn_t<4>(p, sm_count, s);
-  return launch_ffn_t<8>(p, sm_count, s);
+cudaError_t launch_ffn(const FfnParams& p, int sm_count, cudaStream_t s) { return launch_ffn_impl(p, sm_count, s); }
+
+size_t chain_workspace_bytes(const ChainParams& p) { return kTicketBytes + size_t(3) * p.acc_set * 4; }
+
+cudaError_t launch_chain(const ChainParams& p, lr_dtype_t w_dtype, int sm_count, cudaStream_t s) {
+  switch (w_dtype) {
+    case LR_F32: return launch_chain_w<float>(p, sm_count, s);
+    case LR_BF16: return launch_chain_w<__nv_bfloat16>(p, sm_count, s);
+    case LR_I8: return launch_chain_w<int8_t>(p, sm_count, s);
+    default: return cudaErrorInvalidValue;
+  }
 }
 
 }  // namespace lr

@@ -47,6 +47,44 @@ struct Rank1Params {
 // y = (x A) B for up to kMaxGroup projections sharing x; weight-only paths.
 cudaError_t launch_lr_rank1(const Rank1Params& p, lr_dtype_t w_dtype, int sm_count, cudaStream_t s);
 
+// ---- factorised-linear chains (lr_linear, lr_linear_grouped, lr_linear_chain) ----
+constexpr int kMaxChain = LR_MAX_CHAIN;
+
+struct ChainProj {
+  const void* A;      // [rank, d_in]
+  const void* B;      // [rank, d_out]
+  const void* sA;     // int8: [rank]
+  const void* sB;     // int8: [d_out]
+  void* y;            // [batch, d_out], offset to the batch chunk
+  int d_out;
+  int rows;           // active latent rows
+};
+
+struct ChainStep {
+  ChainProj p[kMaxGroup];
+  int n;
+  int d_in;
+  int total_rows;
+  int input_step;     // -1: chain input
+  int input_proj;
+};
+
+struct ChainParams {
+  ChainStep step[kMaxChain];
+  int n_steps;
+  int nb;             // batch rows in this launch (<= kMaxDecodeChunk)
+  const void* x;      // chain input [nb, d_in of step 0], offset to the chunk
+  float* acc;         // 3 accumulator sets of acc_set floats (zero on entry and exit)
+  int acc_set;        // floats per set
+  unsigned int* bar;  // 2 barrier counters (zero on entry and exit)
+  int scale_f16;
+  int* err;
+};
+
+static_assert(sizeof(ChainParams) < 32000, "chain parameters must fit the kernel parameter space");
+size_t chain_workspace_bytes(const ChainParams& p);
+cudaError_t launch_chain(const ChainParams& p, lr_dtype_t w_dtype, int sm_count, cudaStream_t s);
+
 struct FfnParams {
   int hidden, inter, n_lr, n_dense, rank;
   int nb;
@@ -92,11 +130,14 @@ struct W8A8Params {
   float* z;           // [T, rank] fp32 workspace
   int8_t* zq;         // [T, rank_pad] int8 workspace
   float* sz;          // [T]
+  unsigned int* amax; // [T] row max |z| as fp32 bits (zero between calls)
   int rank_pad;
   int* err;           // device error word
 };
 
 size_t w8a8_workspace_bytes(int T, int rank);
+cudaError_t launch_gemm_s8s32(const int8_t* A, const int8_t* B, int b_kn, int M, int N, int K, int32_t* C,
+                              int* err, cudaStream_t s);
 cudaError_t launch_w8a8(const W8A8Params& p, int sm_count, cudaStream_t s);
 
 }  // namespace lr

@@ -1,16 +1,388 @@
-// W8A8 low-rank prefill path (int8 x int8 -> int32 on tcgen05 tensor cores), sm_100a.
+// W8A8 low-rank linear for prefill on tcgen05 tensor cores, sm_100a.
+//
+// LASER results (W8A8 setting) and WSVD QAT section (weights and activations
+// int8): y = (x A) B with int8 activations (one scale per token), int8
+// factors (one scale per output channel), int32 accumulation, and the latent
+// requantised per token between the two products:
+//   acc1 = x_q A_q                   (tcgen05.mma kind::i8, int32 in TMEM)
+//   z    = fp32(fp32(acc1 * s_x[t]) * s_A[j]), per-row max |z|   (epilogue 1)
+//   s_z  = max|z| / 127, z_q = clamp(rint(z / s_z))               (requant)
+//   acc2 = z_q B_q                   (tcgen05.mma kind::i8)
+//   y    = bf16(fp32(fp32(acc2 * s_z[t]) * s_B[k]))                (epilogue 2)
+// Every fp32 step is one IEEE operation (__fmul_rn, __fdiv_rn, rintf), so the
+// codes match an exact emulation bit for bit.
+//
+// GEMM kernel: one CTA per 128 x 256 output tile.  Warp 0 issues TMA loads of
+// 128-byte-swizzled operand tiles into a 4-stage shared-memory ring; warp 1
+// allocates the 256-column TMEM accumulator and one elected thread issues
+// the MMAs (four K=32 steps per 128-byte k-block), releasing each stage with
+// tcgen05.commit; warps 2..5 (one per TMEM lane quarter) wait for the final
+// commit, read the accumulator with tcgen05.ld and run the epilogue.  The
+// first factor A_q [r, d_in] is K-major (the B operand of GEMM 1); the second
+// factor B_q [r, d_out] is N-contiguous, i.e. an MN-major B operand of GEMM 2.
+// Every wait is bounded and records a device error instead of hanging.
+#include <cuda.h>
+
+#include <cstring>
+#include <mutex>
+
 #include "common.cuh"
 #include "internal.h"
 
 namespace lr {
+namespace {
+
+constexpr int kBM = 128;          // tile rows (tokens)
+constexpr int kBN = 256;          // tile columns
+constexpr int kBK = 128;          // k-block: 128 int8 = one 128-byte swizzle atom row
+constexpr int kStages = 4;
+constexpr int kThreads = 192;     // 6 warps
+constexpr int kATileBytes = kBM * kBK;         // 16 KB
+constexpr int kBTileBytes = kBN * kBK;         // 32 KB
+constexpr int kStageBytes = kATileBytes + kBTileBytes;
+constexpr int kTmemCols = 256;
+
+// ---------------------------------------------------------------------------
+// host: tensor maps through the driver entry point (no link against libcuda)
+// ---------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static std::once_flag once;
+  static EncodeTiledFn fn = nullptr;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 2-D int8 tensor [rows, cols] (row stride `ld` bytes), box [box_rows, box_cols],
+// 128-byte swizzle, zero fill outside the tensor.
+bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint64_t ld, uint32_t box_rows,
+              uint32_t box_cols) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {ld};
+  const cuuint32_t box[2] = {box_cols, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// ---------------------------------------------------------------------------
+// device primitives (tcgen05, TMA)
+// ---------------------------------------------------------------------------
+LR_DEV void tma_load_2d(uint32_t smem_dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+      :: "r"(smem_dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar)) : "memory");
+}
+
+// Shared-memory matrix descriptor, 128-byte swizzle, sm_100 version bits.
+LR_DEV uint64_t smem_desc(uint32_t addr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
+  uint64_t d = 0;
+  d |= uint64_t((addr >> 4) & 0x3FFFu);
+  d |= uint64_t((lbo_bytes >> 4) & 0x3FFFu) << 16;
+  d |= uint64_t((sbo_bytes >> 4) & 0x3FFFu) << 32;
+  d |= uint64_t(1) << 46;                // descriptor version for tcgen05
+  d |= uint64_t(2) << 61;                // SWIZZLE_128B
+  return d;
+}
+
+// Instruction descriptor of kind::i8: s8 x s8 -> s32, M = 128, N = 256.
+LR_HD_INLINE uint32_t idesc_i8(bool b_mn_major) {
+  return (2u << 4)                        // D format: S32
+         | (1u << 7) | (1u << 10)         // A, B format: signed 8-bit
+         | (uint32_t(b_mn_major) << 16)   // B major: 0 K, 1 MN
+         | (uint32_t(kBN >> 3) << 17)     // N >> 3
+         | (uint32_t(kBM >> 4) << 24);    // M >> 4
+}
+
+LR_DEV void mma_i8(uint32_t tmem_d, uint64_t a_desc, uint64_t b_desc, uint32_t idesc, bool accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}"
+      :: "r"(tmem_d), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(uint32_t(accumulate)) : "memory");
+}
+
+LR_DEV void mma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
+               :: "r"(smem_u32(bar)) : "memory");
+}
+LR_DEV void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+LR_DEV void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// 32 lanes x 32 columns of 32-bit accumulators: lane i of the warp gets row
+// (lane quarter * 32 + i), columns [col, col + 32).
+LR_DEV void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+        "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15]),
+        "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]),
+        "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+struct GemmParams {
+  int M, N, K;             // tokens, output columns, reduction length
+  int b_mn_major;          // 0: B stored [N, K] (K contiguous); 1: B stored [K, N] (N contiguous)
+  int mode;                // 0: latent epilogue (z, row max); 1: output epilogue (bf16 y); 2: raw int32 C
+  const float* s_row;      // per-token scale (s_x or s_z)
+  const float* s_col;      // per-column scale (s_A or s_B)
+  float* z;                // mode 0: [M, N] fp32
+  unsigned int* amax;      // mode 0: [M] row max |z| (fp32 bits), zero on entry
+  __nv_bfloat16* y;        // mode 1: [M, N]
+  int32_t* c;              // mode 2: [M, N]
+  int* err;
+};
+
+__global__ void __launch_bounds__(kThreads, 1) w8a8_gemm_kernel(const __grid_constant__ CUtensorMap mapA,
+                                                                const __grid_constant__ CUtensorMap mapB,
+                                                                const __grid_constant__ GemmParams P) {
+  extern __shared__ unsigned char smem_raw[];
+  __shared__ __align__(8) uint64_t full[kStages];
+  __shared__ __align__(8) uint64_t empty[kStages];
+  __shared__ __align__(8) uint64_t accum;
+  __shared__ uint32_t tmem_slot;
+  // operand tiles must start on 1024-byte boundaries (128-byte swizzle atoms)
+  const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int m0 = blockIdx.y * kBM, n0 = blockIdx.x * kBN;
+  const int nk = (P.K + kBK - 1) / kBK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(&accum, 1);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                 :: "r"(smem_u32(&tmem_slot)), "r"(kTmemCols) : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_slot;
+  pdl_launch_dependents();
+
+  if (warp == 0) {
+    if (lane == 0) {
+      pdl_wait();  // the A operand (activations) may come from the preceding kernel
+      for (int kb = 0; kb < nk; ++kb) {
+        const int s = kb % kStages, round = kb / kStages;
+        if (round > 0 && !mbar_wait_bounded(&empty[s], uint32_t(round - 1) & 1u, P.err)) break;
+        const uint32_t a_dst = base + uint32_t(s) * kStageBytes, b_dst = a_dst + kATileBytes;
+        mbar_arrive_expect_tx(&full[s], kStageBytes);
+        tma_load_2d(a_dst, &mapA, kb * kBK, m0, &full[s]);
+        if (!P.b_mn_major) {
+          tma_load_2d(b_dst, &mapB, kb * kBK, n0, &full[s]);
+        } else {
+          tma_load_2d(b_dst, &mapB, n0, kb * kBK, &full[s]);
+          tma_load_2d(b_dst + kBK * 128, &mapB, n0 + 128, kb * kBK, &full[s]);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t idesc = idesc_i8(P.b_mn_major != 0);
+      bool ok = true;
+      for (int kb = 0; kb < nk && ok; ++kb) {
+        const int s = kb % kStages, round = kb / kStages;
+        if (!mbar_wait_bounded(&full[s], uint32_t(round) & 1u, P.err)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t a_base = base + uint32_t(s) * kStageBytes, b_base = a_base + kATileBytes;
+#pragma unroll
+        for (int kk = 0; kk < kBK / 32; ++kk) {
+          const uint64_t ad = smem_desc(a_base + kk * 32, 16, 1024);
+          const uint64_t bd = P.b_mn_major ? smem_desc(b_base + kk * 32 * 128, kBK * 128, 1024)
+                                           : smem_desc(b_base + kk * 32, 16, 1024);
+          mma_i8(tmem, ad, bd, idesc, kb > 0 || kk > 0);
+        }
+        mma_commit(&empty[s]);
+      }
+      if (ok) mma_commit(&accum);
+    }
+  } else {
+    // epilogue: warp w reads TMEM lanes 32 * (w % 4) .. + 31 (one accumulator row per thread)
+    const int q = warp & 3;
+    const int row = m0 + q * 32 + lane;
+    const bool have = mbar_wait_bounded(&accum, 0u, P.err);
+    tc_fence_after();
+    if (have) {
+      // the raw int32 mode has no scales (s_row, s_col are null there)
+      const float sr = (P.mode != 2 && row < P.M) ? P.s_row[row] : 0.f;
+      float rmax = 0.f;
+      for (int c = 0; c < kBN / 32; ++c) {
+        uint32_t v[32];
+        tmem_ld32(tmem + (uint32_t(q * 32) << 16) + uint32_t(c * 32), v);
+        const int col0 = n0 + c * 32;
+        if (row >= P.M || col0 >= P.N) continue;
+        if (P.mode == 2) {
+          int32_t* cr = P.c + size_t(row) * P.N + col0;
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            if (col0 + i < P.N) cr[i] = int32_t(v[i]);
+        } else if (P.mode == 0) {
+          float* zr = P.z + size_t(row) * P.N + col0;
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            if (col0 + i < P.N) {
+              const float zv = __fmul_rn(__fmul_rn(__int2float_rn(int(v[i])), sr), P.s_col[col0 + i]);
+              zr[i] = zv;
+              rmax = fmaxf(rmax, fabsf(zv));
+            }
+          }
+        } else {
+          __nv_bfloat16* yr = P.y + size_t(row) * P.N + col0;
+#pragma unroll
+          for (int i = 0; i < 32; i += 2) {
+            if (col0 + i + 1 < P.N) {
+              const float a = __fmul_rn(__fmul_rn(__int2float_rn(int(v[i])), sr), P.s_col[col0 + i]);
+              const float b = __fmul_rn(__fmul_rn(__int2float_rn(int(v[i + 1])), sr), P.s_col[col0 + i + 1]);
+              *reinterpret_cast<__nv_bfloat162*>(yr + i) = __floats2bfloat162_rn(a, b);
+            } else if (col0 + i < P.N) {
+              yr[i] = __float2bfloat16_rn(__fmul_rn(__fmul_rn(__int2float_rn(int(v[i])), sr), P.s_col[col0 + i]));
+            }
+          }
+        }
+      }
+      if (P.mode == 0 && row < P.M) atomicMax(reinterpret_cast<int*>(P.amax) + row, __float_as_int(rmax));
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" :: "r"(tmem), "r"(kTmemCols) : "memory");
+  }
+}
+
+// Per-token requantisation of the latent: s_z = max|z| / 127 (1 for a zero
+// row), z_q = clamp(rint(z / s_z), -127, 127); columns r .. rank_pad-1 of z_q
+// are zero; the row max is reset to zero for the next call.
+__global__ void __launch_bounds__(256) requant_kernel(const float* __restrict__ z, unsigned int* amax, int r,
+                                                      int rank_pad, int8_t* __restrict__ zq, float* __restrict__ sz) {
+  const int t = blockIdx.x;
+  pdl_launch_dependents();
+  pdl_wait();
+  __shared__ float s_sc;
+  __shared__ int s_zero;
+  if (threadIdx.x == 0) {
+    const float a = __int_as_float(int(amax[t]));
+    float sc = __fdiv_rn(a, 127.0f);
+    s_zero = sc == 0.0f;
+    if (sc == 0.0f) sc = 1.0f;
+    s_sc = sc;
+    sz[t] = sc;
+  }
+  __syncthreads();
+  const float sc = s_sc;
+  const bool zero = s_zero != 0;
+  const float* zr = z + size_t(t) * r;
+  int8_t* qr = zq + size_t(t) * rank_pad;
+  for (int j = threadIdx.x * 4; j < rank_pad; j += blockDim.x * 4) {
+    uint32_t w = 0;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      float q = 0.f;
+      if (j + e < r && !zero) q = fminf(fmaxf(rintf(__fdiv_rn(zr[j + e], sc)), -127.f), 127.f);
+      w |= (uint32_t(int(q)) & 0xffu) << (8 * e);
+    }
+    *reinterpret_cast<uint32_t*>(qr + j) = w;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) amax[t] = 0u;
+}
+
+cudaError_t launch_gemm(const CUtensorMap& a, const CUtensorMap& b, const GemmParams& p, cudaStream_t s) {
+  const size_t smem = size_t(kStages) * kStageBytes + 1024;
+  cudaError_t e = ensure_smem(w8a8_gemm_kernel, smem);
+  if (e != cudaSuccess) return e;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t c = {};
+  c.gridDim = dim3((p.N + kBN - 1) / kBN, (p.M + kBM - 1) / kBM);
+  c.blockDim = dim3(kThreads);
+  c.dynamicSmemBytes = smem;
+  c.stream = s;
+  c.attrs = attr;
+  c.numAttrs = 1;
+  return cudaLaunchKernelEx(&c, w8a8_gemm_kernel, a, b, p);
+}
+
+}  // namespace
 
 size_t w8a8_workspace_bytes(int T, int rank) {
   const size_t rp = (size_t(rank) + 127) / 128 * 128;
   const size_t tp = (size_t(T) + 127) / 128 * 128;
   auto ru = [](size_t v) { return (v + 255) / 256 * 256; };
-  return ru(size_t(T) * rank * 4) + ru(tp * rp) + ru(tp * 4);
+  return ru(size_t(T) * rank * 4) + ru(tp * rp) + ru(tp * 4) + ru(tp * 4);
 }
 
-cudaError_t launch_w8a8(const W8A8Params&, int, cudaStream_t) { return cudaErrorNotSupported; }
+cudaError_t launch_gemm_s8s32(const int8_t* A, const int8_t* B, int b_kn, int M, int N, int K, int32_t* C,
+                              int* err, cudaStream_t s) {
+  CUtensorMap ma, mb;
+  if (!make_map(&ma, A, M, K, K, kBM, kBK)) return cudaErrorInvalidValue;
+  if (!b_kn) {
+    if (!make_map(&mb, B, N, K, K, kBN, kBK)) return cudaErrorInvalidValue;
+  } else {
+    if (!make_map(&mb, B, K, N, N, kBK, 128)) return cudaErrorInvalidValue;
+  }
+  GemmParams g;
+  std::memset(&g, 0, sizeof(g));
+  g.M = M; g.N = N; g.K = K; g.b_mn_major = b_kn; g.mode = 2; g.c = C; g.err = err;
+  return launch_gemm(ma, mb, g, s);
+}
+
+cudaError_t launch_w8a8(const W8A8Params& p, int /*sm_count*/, cudaStream_t s) {
+  CUtensorMap mx, ma, mz, mb;
+  if (!make_map(&mx, p.xq, p.T, p.d_in, p.d_in, kBM, kBK)) return cudaErrorInvalidValue;
+  if (!make_map(&ma, p.Aq, p.rank, p.d_in, p.d_in, kBN, kBK)) return cudaErrorInvalidValue;
+  if (!make_map(&mz, p.zq, p.T, p.rank_pad, p.rank_pad, kBM, kBK)) return cudaErrorInvalidValue;
+  if (!make_map(&mb, p.Bq, p.rank, p.d_out, p.d_out, kBK, 128)) return cudaErrorInvalidValue;
+
+  GemmParams g1;
+  std::memset(&g1, 0, sizeof(g1));
+  g1.M = p.T; g1.N = p.rank; g1.K = p.d_in; g1.b_mn_major = 0; g1.mode = 0;
+  g1.s_row = p.sx; g1.s_col = p.sA; g1.z = p.z; g1.amax = p.amax; g1.err = p.err;
+  cudaError_t e = launch_gemm(mx, ma, g1, s);
+  if (e != cudaSuccess) return e;
+
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t c = {};
+  c.gridDim = dim3(p.T);
+  c.blockDim = dim3(256);
+  c.stream = s;
+  c.attrs = attr;
+  c.numAttrs = 1;
+  e = cudaLaunchKernelEx(&c, requant_kernel, static_cast<const float*>(p.z), p.amax, p.rank, p.rank_pad, p.zq, p.sz);
+  if (e != cudaSuccess) return e;
+
+  GemmParams g2;
+  std::memset(&g2, 0, sizeof(g2));
+  g2.M = p.T; g2.N = p.d_out; g2.K = p.rank; g2.b_mn_major = 1; g2.mode = 1;
+  g2.s_row = p.sz; g2.s_col = p.sB; g2.y = reinterpret_cast<__nv_bfloat16*>(p.y); g2.err = p.err;
+  return launch_gemm(mz, mb, g2, s);
+}
 
 }  // namespace lr

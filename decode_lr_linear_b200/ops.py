@@ -162,6 +162,55 @@ def lr_linear_grouped(factors: Sequence[Factor], x: torch.Tensor, ys: Optional[S
     return list(ys)
 
 
+@dataclass
+class ChainStep:
+    """One step of lr_linear_chain: projections sharing one input, which is the
+    chain input (input_step = -1) or output `input_proj` of an earlier step."""
+    factors: Sequence[Factor]
+    input_step: int = -1
+    input_proj: int = 0
+    ys: Optional[Sequence[torch.Tensor]] = None
+
+
+def _chain_array(steps: Sequence[ChainStep]):
+    arr = (L.ChainStep * len(steps))()
+    for i, st in enumerate(steps):
+        arr[i].n = len(st.factors)
+        arr[i].input_step = st.input_step
+        arr[i].input_proj = st.input_proj
+        for p, f in enumerate(st.factors):
+            arr[i].proj[p] = f.desc()
+            arr[i].y[p] = _ptr(st.ys[p]) if st.ys is not None else None
+    return arr
+
+
+def lr_linear_chain_workspace_size(steps: Sequence[ChainStep], batch: int) -> int:
+    n = ctypes.c_size_t(0)
+    arr = _chain_array([ChainStep(s.factors, s.input_step, s.input_proj,
+                                  s.ys if s.ys is not None else [torch.empty(0)] * len(s.factors)) for s in steps])
+    for i in range(len(steps)):  # placeholder outputs: only the shapes matter here
+        for p in range(arr[i].n):
+            arr[i].y[p] = 16
+    L.check("lr_linear_chain_workspace_size", L.load().lr_linear_chain_workspace_size(arr, len(steps), batch,
+                                                                                     ctypes.byref(n)))
+    return n.value
+
+
+def lr_linear_chain(steps: Sequence[ChainStep], x: torch.Tensor, ws: Optional[torch.Tensor] = None,
+                    stream=None) -> list:
+    """Runs the chain in one launch; returns every step's output list."""
+    batch = x.shape[0]
+    for st in steps:
+        if st.ys is None:
+            st.ys = [torch.empty(batch, f.d_out, dtype=f.out_dtype(), device=x.device) for f in st.factors]
+    if ws is None:
+        ws = workspace(lr_linear_chain_workspace_size(steps, batch), x.device)
+    arr = _chain_array(steps)
+    L.check("lr_linear_chain", L.load().lr_linear_chain(arr, len(steps), _ptr(x), batch, _ptr(ws),
+                                                        ws.numel() * ws.element_size(), _stream(stream)))
+    return [list(st.ys) for st in steps]
+
+
 def lr_swiglu_ffn_workspace_size(ffn: FfnWeights, batch: int) -> int:
     n = ctypes.c_size_t(0)
     d = ffn.desc()
@@ -214,6 +263,17 @@ def lr_quantize_per_token(x: torch.Tensor, x_q: Optional[torch.Tensor] = None, s
     L.check("lr_quantize_per_token", L.load().lr_quantize_per_token(_ptr(x), rows, cols, _ptr(x_q), _ptr(s),
                                                                     _stream(stream)))
     return x_q, s
+
+
+def lr_gemm_s8s32(A: torch.Tensor, B: torch.Tensor, b_layout: int, C: Optional[torch.Tensor] = None,
+                  stream=None) -> torch.Tensor:
+    """C = A B (int8 x int8 -> int32).  b_layout 0: B is [N, K]; 1: B is [K, N]."""
+    M, K = A.shape
+    N = B.shape[0] if b_layout == 0 else B.shape[1]
+    if C is None:
+        C = torch.empty(M, N, dtype=torch.int32, device=A.device)
+    L.check("lr_gemm_s8s32", L.load().lr_gemm_s8s32(_ptr(A), _ptr(B), b_layout, M, N, K, _ptr(C), _stream(stream)))
+    return C
 
 
 def lr_workspace_init(ws: torch.Tensor, stream=None) -> None:

@@ -124,6 +124,8 @@ typedef struct lr_factor_desc {
  *     acc2 = z_q B_q (int32);  y = bf16(fp32(fp32(acc2 * s_z[t]) * scale_B[k]))
  *   (LASER results, W8A8 setting; WSVD "Quantization-Aware Training",
  *   weights and activations quantised, e.g. W8A8).
+ * Weight-only limits: d_in and d_out multiples of 8 (of 16 for int8 weights)
+ * and at most 32 KiB per factor row (d <= 16384 for bf16, 8192 for f32).
  * ws: workspace of at least lr_linear_workspace_size(...) bytes.
  * Errors: LR_ERR_INVALID_ARG (null pointers, batch < 1, bad shape or rank),
  * LR_ERR_UNSUPPORTED (dtype combination), LR_ERR_MISALIGNED,
@@ -140,7 +142,7 @@ LR_API lr_status_t lr_linear_workspace_size(const lr_factor_desc_t* desc, int ba
  * launch: y_p = (x A_p) B_p for p < n (1 <= n <= LR_MAX_GROUP).  All
  * descriptors must have the same d_in, w_dtype and scale_dtype; ranks and
  * d_out may differ.  `descs` is a host array of n descriptors and `ys` a host
- * array of n device output pointers.  Weight-only paths only (batch 1..8).
+ * array of n device output pointers.  Weight-only paths only, any batch >= 1.
  * LASER "System Implementation" fuses the input projection with the latent
  * activation; sharing x across Q/K/V reads it once.
  */
@@ -150,6 +152,40 @@ LR_API lr_status_t lr_linear_grouped(const lr_factor_desc_t* descs, int n, const
 
 LR_API lr_status_t lr_linear_grouped_workspace_size(const lr_factor_desc_t* descs, int n, int batch,
                                              size_t* bytes);
+
+/*
+ * A chain of grouped factorised linears in one launch: the projections of a
+ * decode stack (for example Q, K, V of a layer, then O, then the next layer)
+ * where a step's input is the chain input or an output of an earlier step.
+ * Step s computes y[s][p] = (x_s A[s][p]) B[s][p] for p < n, with
+ *   x_s = x                      when input_step < 0,
+ *   x_s = y[input_step][input_proj] otherwise (input_step < s).
+ * An input taken from the step right before is read at fp32 (before the
+ * output rounding to bf16); an older one is read from its stored output.
+ * Every step's outputs are written.  All descriptors of a step share d_in,
+ * which must equal d_out of the projection its input comes from; all steps
+ * share w_dtype (weight-only paths) and scale_dtype; batch 1..8; at most
+ * LR_MAX_CHAIN steps.  One persistent CTA per SM streams the factors of all
+ * steps back to back through shared memory, so the loads of step s+1 proceed
+ * while step s is finishing; the CTAs meet at one (bounded) grid-wide barrier
+ * per step.  LASER "System Implementation" fuses the stages of a layer to cut
+ * memory movement and kernel-launch overhead; this is that fusion across
+ * consecutive factorised projections.
+ */
+#define LR_MAX_CHAIN 64
+typedef struct lr_chain_step {
+  int n;
+  int input_step;
+  int input_proj;
+  lr_factor_desc_t proj[LR_MAX_GROUP];
+  void* y[LR_MAX_GROUP];
+} lr_chain_step_t;
+
+LR_API lr_status_t lr_linear_chain(const lr_chain_step_t* steps, int n_steps, const void* x, int batch, void* ws,
+                                   size_t ws_bytes, lr_stream_t stream);
+
+LR_API lr_status_t lr_linear_chain_workspace_size(const lr_chain_step_t* steps, int n_steps, int batch,
+                                                  size_t* bytes);
 
 /*
  * lr_linear without a caller-provided workspace (the pages have no
@@ -164,9 +200,9 @@ LR_API lr_status_t lr_linear_grouped_workspace_size(const lr_factor_desc_t* desc
  * LR_NOALLOC_SCRATCH_BYTES bytes per device, which every GPU that loads the
  * library keeps until the process exits.  The caller still passes x and y.
  *
- *   - The scratch a call needs is 256 + 256-rounded(min(batch, 8) * d_out * 4)
- *     bytes; a call that needs more returns LR_ERR_WORKSPACE and launches
- *     nothing.
+ *   - The scratch a call needs is what lr_linear_workspace_size reports,
+ *     256 + 3 * 64-rounded(min(batch, 8) * d_out) * 4 bytes; a call that needs
+ *     more returns LR_ERR_WORKSPACE and launches nothing.
  *   - The first call on a device looks the array up and zero-fills it on
  *     `stream`; make that first call before any stream capture.  Every call
  *     leaves the array zeroed again.
@@ -219,8 +255,9 @@ typedef struct lr_ffn_desc {
   const void* s_down;
 } lr_ffn_desc_t;
 
-/* x bf16 [batch, hidden] -> y bf16 [batch, hidden]; batch 1..8.
- * Errors as lr_linear. */
+/* x bf16 [batch, hidden] -> y bf16 [batch, hidden], any batch >= 1.
+ * Limits: hidden a multiple of 16 and <= 32768; n_lr a multiple of 8 and
+ * <= 16384.  Errors as lr_linear. */
 LR_API lr_status_t lr_swiglu_ffn(const lr_ffn_desc_t* desc, const void* x, int batch, void* y, void* ws,
                           size_t ws_bytes, lr_stream_t stream);
 
@@ -287,6 +324,21 @@ LR_API lr_status_t lr_latent_kv_workspace_size(const lr_latent_kv_desc_t* desc, 
  */
 LR_API lr_status_t lr_quantize_per_token(const void* x, int rows, int cols, int8_t* x_q, float* s,
                                   lr_stream_t stream);
+
+/*
+ * The tensor-core product behind the W8A8 path, exposed on its own so that
+ * its integer results can be checked exactly: C = A B with int8 operands and
+ * int32 accumulation (tcgen05 kind::i8), nothing else.
+ *   A      [M, K] int8, row-major
+ *   B      b_layout 0: [N, K] int8 row-major (the layout of the first factor,
+ *          latent-major A_q [r, d_in]); b_layout 1: [K, N] int8 row-major
+ *          (the layout of the second factor B_q [r, d_out])
+ *   C      [M, N] int32, row-major
+ * Limits: K and N multiples of 16; M, N, K >= 1.  No workspace.
+ * |C| must stay below 2^31 (K * 127^2 < 2^31 holds for K < 133144).
+ */
+LR_API lr_status_t lr_gemm_s8s32(const int8_t* A, const int8_t* B, int b_layout, int M, int N, int K, int32_t* C,
+                                 lr_stream_t stream);
 
 /* ------------------------------------------------------------------------ */
 /* Utilities                                                                */

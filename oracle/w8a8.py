@@ -84,6 +84,23 @@ def w8a8_lr_linear(xq, s_x, Aq, s_A, Bq, s_B) -> dict:
     return {"acc1": acc1, "z": z, "zq": zq, "s_z": s_z, "acc2": acc2, "y": bf16_round(y32)}
 
 
+def w8a8_fp64_reference(xq, s_x, Aq, s_A, Bq, s_B) -> np.ndarray:
+    """The same W8A8 method evaluated in float64: z = (X A) in float64, per-token
+    requant of z with the same rule (s_z = max|z| / 127, rint ties to even,
+    clamp to +-127), y = (z_q s_z) B, all in float64 (no fp32 or bf16 rounding).
+    """
+    X = _np(xq).astype(np.float64) * _np(s_x).astype(np.float64)[:, None]
+    A = (_np(Aq).astype(np.float64) * _np(s_A).astype(np.float64)[:, None]).T
+    B = _np(Bq).astype(np.float64) * _np(s_B).astype(np.float64)[None, :]
+    z = X @ A
+    s_z = np.abs(z).max(axis=1) / 127.0
+    zero = s_z == 0.0
+    s_safe = np.where(zero, 1.0, s_z)
+    zq = np.clip(np.rint(z / s_safe[:, None]), -127, 127)
+    zq[zero, :] = 0.0
+    return (zq * s_safe[:, None]) @ B
+
+
 def w8a8_dequant_reference(xq, s_x, Aq, s_A, Bq, s_B) -> np.ndarray:
     """Float64 definition without the latent requant: y = (X A) B with X = xq s_x,
     A = (Aq s_A)^T, B = Bq s_B (column scales)."""

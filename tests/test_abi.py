@@ -42,10 +42,11 @@ def _ws(lib, d, batch, w8a8=0):
 
 
 def test_linear_workspace_sizes(lib):
+    # barrier words + three accumulator sets of min(batch, 8) x d_out floats
     st, n = _ws(lib, _desc(), 1)
-    assert st == L.LR_OK and n == 256 + 4096 * 4
+    assert st == L.LR_OK and n == 256 + 3 * 4096 * 4
     st, n8 = _ws(lib, _desc(), 16)
-    assert st == L.LR_OK and n8 == 256 + 8 * 4096 * 4
+    assert st == L.LR_OK and n8 == 256 + 3 * 8 * 4096 * 4
     st, _ = _ws(lib, _desc(w_dtype=L.LR_I8), 1)
     assert st == L.LR_ERR_INVALID_ARG  # int8 needs scales
     st, n = _ws(lib, _desc(w_dtype=L.LR_I8, scale_A=FAKE, scale_B=FAKE), 2048, 1)
@@ -61,6 +62,9 @@ def test_linear_validation(lib):
     assert call(_desc(active_rank=2000)) == L.LR_ERR_INVALID_ARG
     assert call(_desc(d_in=4100)) == L.LR_ERR_UNSUPPORTED
     assert call(_desc(w_dtype=L.LR_F16)) == L.LR_ERR_UNSUPPORTED
+    i8 = dict(w_dtype=L.LR_I8, scale_A=FAKE, scale_B=FAKE)
+    assert call(_desc(d_in=4104, **i8)) == L.LR_ERR_UNSUPPORTED   # int8 rows must be 16-byte multiples
+    assert call(_desc(d_in=16392)) == L.LR_ERR_UNSUPPORTED        # bf16 row above 32 KiB
     assert call(_desc(A=MIS)) == L.LR_ERR_MISALIGNED
     assert call(_desc(), x=MIS) == L.LR_ERR_MISALIGNED
     assert call(_desc(), b=0) == L.LR_ERR_INVALID_ARG
@@ -80,7 +84,7 @@ def test_grouped_validation(lib):
     arr = (L.FactorDesc * 3)(_desc(), _desc(d_out=1024), _desc(rank=512))
     n = ctypes.c_size_t(0)
     assert lib.lr_linear_grouped_workspace_size(arr, 3, 1, ctypes.byref(n)) == L.LR_OK
-    assert n.value == 256 + 4096 * 4 + 1024 * 4 + 4096 * 4
+    assert n.value == 256 + 3 * (4096 + 1024 + 4096) * 4
 
 
 def _ffn(**kw):
@@ -97,6 +101,8 @@ def test_ffn_validation_and_workspace(lib):
     assert n.value == 256 + 16384 * 4 + 2816 * 4 + 4096 * 4
     bad = _ffn(n_lr=12000)
     assert lib.lr_swiglu_ffn(ctypes.byref(bad), FAKE, 1, FAKE, FAKE, 1 << 20, None) == L.LR_ERR_INVALID_ARG
+    bad = _ffn(n_lr=8196)
+    assert lib.lr_swiglu_ffn(ctypes.byref(bad), FAKE, 1, FAKE, FAKE, 1 << 20, None) == L.LR_ERR_UNSUPPORTED
     bad = _ffn(hidden=4100)
     assert lib.lr_swiglu_ffn(ctypes.byref(bad), FAKE, 1, FAKE, FAKE, 1 << 20, None) == L.LR_ERR_UNSUPPORTED
     bad = _ffn(D=MIS)
@@ -131,3 +137,27 @@ def test_quantize_validation(lib):
     assert lib.lr_quantize_per_token(FAKE, 4, 100, FAKE, FAKE, None) == L.LR_ERR_UNSUPPORTED
     assert lib.lr_quantize_per_token(None, 4, 128, FAKE, FAKE, None) == L.LR_ERR_INVALID_ARG
     assert lib.lr_quantize_per_token(MIS, 4, 128, FAKE, FAKE, None) == L.LR_ERR_MISALIGNED
+
+
+def _step(n=1, input_step=-1, input_proj=0, **kw):
+    st = L.ChainStep()
+    st.n, st.input_step, st.input_proj = n, input_step, input_proj
+    for p in range(n):
+        st.proj[p] = _desc(**kw)
+        st.y[p] = FAKE
+    return st
+
+
+def test_chain_validation_and_workspace(lib):
+    arr = (L.ChainStep * 3)(_step(3), _step(1, 0, 2), _step(3, 1, 0))
+    n = ctypes.c_size_t(0)
+    assert lib.lr_linear_chain_workspace_size(arr, 3, 1, ctypes.byref(n)) == L.LR_OK
+    assert n.value == 256 + 3 * 3 * 4096 * 4
+    bad = (L.ChainStep * 2)(_step(1), _step(1, 1, 0))            # input from itself
+    assert lib.lr_linear_chain(bad, 2, FAKE, 1, FAKE, 1 << 24, None) == L.LR_ERR_INVALID_ARG
+    bad = (L.ChainStep * 2)(_step(1), _step(1, 0, 3))            # no such output
+    assert lib.lr_linear_chain(bad, 2, FAKE, 1, FAKE, 1 << 24, None) == L.LR_ERR_INVALID_ARG
+    bad = (L.ChainStep * 2)(_step(1), _step(1, 0, 0, d_in=2048))  # width mismatch
+    assert lib.lr_linear_chain(bad, 2, FAKE, 1, FAKE, 1 << 24, None) == L.LR_ERR_INVALID_ARG
+    assert lib.lr_linear_chain(arr, 3, FAKE, 1, FAKE, 64, None) == L.LR_ERR_WORKSPACE
+    assert lib.lr_linear_chain(arr, 0, FAKE, 1, FAKE, 1 << 24, None) == L.LR_ERR_INVALID_ARG

@@ -1,0 +1,99 @@
+"""GPU parity: W8A8 prefill path on tcgen05 (int8 x int8 -> int32), against the oracle.
+
+Integer accumulations are compared bit for bit; the full pipeline's bf16
+output too (every fp32 step is specified), plus the 1e-2 normwise bar
+against the same W8A8 method evaluated in float64.
+"""
+import numpy as np
+import pytest
+import torch
+
+import decode_lr_linear_b200 as lr
+from decode_lr_linear_b200 import synth
+from oracle import w8a8 as ow8
+from tests._helpers import NORMWISE_TOL, dev, normwise_rel
+
+pytestmark = pytest.mark.gpu
+
+
+def _rand_i8(rng, shape, lo=-127, hi=127):
+    return torch.from_numpy(rng.integers(lo, hi + 1, size=shape).astype(np.int8))
+
+
+@pytest.mark.parametrize("M,N,K", [(128, 256, 128), (200, 336, 272), (2048, 640, 5120), (7, 16, 16)])
+@pytest.mark.parametrize("b_layout", [0, 1])
+def test_gemm_s8s32_bit_exact(cuda_device, M, N, K, b_layout):
+    rng = np.random.default_rng(M * 7 + N + K + b_layout)
+    A = _rand_i8(rng, (M, K))
+    Bnk = _rand_i8(rng, (N, K))
+    B = Bnk if b_layout == 0 else Bnk.T.contiguous()
+    C = lr.lr_gemm_s8s32(dev(A), dev(B), b_layout)
+    ref = ow8.int_matmul_nt(A, Bnk)
+    assert np.array_equal(C.cpu().numpy().astype(np.int64), ref)
+
+
+@pytest.mark.parametrize("b_layout", [0, 1])
+def test_gemm_s8s32_extreme_values(cuda_device, b_layout):
+    K = 13824
+    A = torch.full((130, K), 127, dtype=torch.int8)
+    A[1::2] = -127
+    Bnk = torch.full((272, K), -127, dtype=torch.int8)
+    Bnk[1:, ::3] = 127          # row 0 keeps one sign: |C| reaches K * 127^2
+    B = Bnk if b_layout == 0 else Bnk.T.contiguous()
+    C = lr.lr_gemm_s8s32(dev(A), dev(B), b_layout).cpu().numpy().astype(np.int64)
+    ref = ow8.int_matmul_nt(A, Bnk)
+    assert np.array_equal(C, ref)
+    assert np.abs(ref).max() > 2 ** 27
+
+
+def _pipeline(d_in, d_out, rank, T, seed):
+    p = synth.make_prefill_projection(d_in, d_out, rank, seed=seed, key=(d_in, d_out, rank))
+    x = synth.make_activations(T, d_in, seed=seed, key=(60, d_in, T), outliers=max(1, d_in // 1000))
+    xq, sx = lr.lr_quantize_per_token(dev(x))
+    f = lr.Factor(dev(p["A_q"]), dev(p["B_q"]), dev(p["s_A"]), dev(p["s_B"]))
+    y = lr.lr_linear(f, xq, x_scale=sx)
+    q_ref, s_ref = ow8.quantize_per_token(x)
+    res = ow8.w8a8_lr_linear(q_ref, s_ref, p["A_q"], p["s_A"], p["B_q"], p["s_B"])
+    # the same W8A8 method in float64 (latent requantised per token in float64)
+    ref64 = ow8.w8a8_fp64_reference(q_ref, s_ref, p["A_q"], p["s_A"], p["B_q"], p["s_B"])
+    return p, xq, sx, q_ref, s_ref, y, res, ref64
+
+
+@pytest.mark.parametrize("d_in,d_out,rank,T", [(512, 768, 320, 256), (256, 512, 96, 130)])
+def test_w8a8_pipeline_small_bit_exact(cuda_device, d_in, d_out, rank, T):
+    p, xq, sx, q_ref, s_ref, y, res, ref64 = _pipeline(d_in, d_out, rank, T, seed=1)
+    assert np.array_equal(xq.cpu().numpy(), q_ref) and np.array_equal(sx.cpu().numpy(), s_ref)
+    assert np.array_equal(y.float().cpu().numpy(), res["y"])
+    assert normwise_rel(y, ref64) < NORMWISE_TOL
+
+
+@pytest.fixture(scope="module")
+def prefill_ranks():
+    return synth.prefill_ranks(0)
+
+
+@pytest.mark.parametrize("proj", ["q", "gate", "down"])
+def test_w8a8_llama13b_shapes(cuda_device, prefill_ranks, proj):
+    j = synth.PREFILL_PROJ.index(proj)
+    d_in, d_out = synth.prefill_shapes()[proj]
+    rank = int(prefill_ranks[0, j])
+    p, xq, sx, q_ref, s_ref, y, res, ref64 = _pipeline(d_in, d_out, rank, 2048, seed=0)
+    # first product bit-exact at full size, and the second on the oracle's requantised latent
+    acc1 = lr.lr_gemm_s8s32(xq, dev(p["A_q"]), 0).cpu().numpy().astype(np.int64)
+    assert np.array_equal(acc1, res["acc1"])
+    acc2 = lr.lr_gemm_s8s32(dev(torch.from_numpy(np.ascontiguousarray(res["zq"]))), dev(p["B_q"]), 1)
+    assert np.array_equal(acc2.cpu().numpy().astype(np.int64), res["acc2"])
+    assert np.array_equal(y.float().cpu().numpy(), res["y"])
+    assert normwise_rel(y, ref64) < NORMWISE_TOL
+
+
+def test_w8a8_repeat_calls_same_workspace(cuda_device):
+    p = synth.make_prefill_projection(512, 512, 160, seed=3, key=(3,))
+    f = lr.Factor(dev(p["A_q"]), dev(p["B_q"]), dev(p["s_A"]), dev(p["s_B"]))
+    x = synth.make_activations(300, 512, seed=3, key=(61,))
+    xq, sx = lr.lr_quantize_per_token(dev(x))
+    ws = lr.workspace(lr.lr_linear_workspace_size(f, 300, w8a8=True), xq.device)
+    y1 = lr.lr_linear(f, xq, x_scale=sx, ws=ws)
+    y2 = lr.lr_linear(f, xq, x_scale=sx, ws=ws)
+    assert torch.equal(y1, y2)
+    assert lr.lr_check_device_error() == 0

@@ -79,3 +79,44 @@ def test_unit_scale_integer_pipeline():
     res = O.w8a8_lr_linear(xq, one(3, np.float32), Aq, one(8, np.float32), Bq, one(6, np.float32))
     acc1 = xq.astype(np.int64) @ Aq.astype(np.int64).T
     assert np.array_equal(res["z"], acc1.astype(np.float32))
+
+
+def _brute_fp64_method(xq, sx, Aq, sA, Bq, sB):
+    T, d_in = xq.shape
+    r, d_out = Aq.shape[0], Bq.shape[1]
+    y = np.zeros((T, d_out))
+    for t in range(T):
+        z = [sum(float(xq[t, i]) * float(sx[t]) * float(Aq[j, i]) * float(sA[j]) for i in range(d_in))
+             for j in range(r)]
+        sz = max(abs(v) for v in z) / 127.0
+        if sz == 0.0:
+            continue
+        zq = [min(127.0, max(-127.0, float(np.rint(v / sz)))) for v in z]
+        for k in range(d_out):
+            y[t, k] = sum(zq[j] * sz * float(Bq[j, k]) * float(sB[k]) for j in range(r))
+    return y
+
+
+def test_fp64_method_brute_force_and_zero_row():
+    rng = np.random.default_rng(8)
+    xq = rng.integers(-127, 128, size=(3, 9)).astype(np.int8)
+    xq[1] = 0
+    sx = rng.uniform(0.01, 0.1, 3)
+    Aq = rng.integers(-127, 128, size=(5, 9)).astype(np.int8)
+    sA = rng.uniform(0.001, 0.01, 5)
+    Bq = rng.integers(-127, 128, size=(5, 4)).astype(np.int8)
+    sB = rng.uniform(0.001, 0.01, 4)
+    y = O.w8a8_fp64_reference(xq, sx, Aq, sA, Bq, sB)
+    assert np.abs(y - _brute_fp64_method(xq, sx, Aq, sA, Bq, sB)).max() < 1e-12
+    assert not y[1].any()
+
+
+def test_fp64_method_agrees_with_fp32_pipeline():
+    """The fp32-exact pipeline and the float64 method differ only by rounding."""
+    p = synth.make_prefill_projection(384, 256, 96, seed=2, key=(2,))
+    x = synth.make_activations(64, 384, seed=2, key=(11,), outliers=1)
+    xq, sx = O.quantize_per_token(x)
+    res = O.w8a8_lr_linear(xq, sx, p["A_q"], p["s_A"], p["B_q"], p["s_B"])
+    y64 = O.w8a8_fp64_reference(xq, sx, p["A_q"], p["s_A"], p["B_q"], p["s_B"])
+    rel = np.linalg.norm(res["y"] - y64, axis=1) / np.linalg.norm(y64, axis=1)
+    assert rel.max() < 5e-3
