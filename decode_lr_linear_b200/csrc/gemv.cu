@@ -609,374 +609,6 @@ __global__ void __launch_bounds__(kThreads, (NB <= 1 && LPW <= 2 ? 2 : 1)) strea
 }
 
 // ---------------------------------------------------------------------------
-// Chains of grouped factorised linears: one persistent CTA per SM.
-//
-// The producer warp streams the factor rows of every step back to back; it
-// never waits for a step boundary, so the loads of step s+1 are in flight
-// while step s finishes.  Consumers, per step: stage the step's input x (fp32)
-// in shared memory, run phase A and phase B on the CTA's latent rows, add the
-// partial outputs into accumulator set s % 3, then meet at a grid barrier
-// (bounded spin; the grid is one CTA per SM, all resident).  After it each
-// CTA writes its slice of the step's outputs and zeroes its slice of set
-// (s-1) % 3, which step s read as its input and nobody reads again.
-// ---------------------------------------------------------------------------
-constexpr int kChainStagesMax = 6;
-int lpw_for(int d_out);
-
-struct ChainLayout {
-  size_t x, part, z, total;
-};
-
-template <int NB>
-LR_HD_INLINE ChainLayout chain_layout(int stages, int x_elems, int rows_cap) {
-  ChainLayout L;
-  L.x = size_t(stages) * kStageBytes;
-  L.part = L.x + round16(size_t(NB) * x_elems * 4);
-  L.z = L.part + round16(size_t(rows_cap) * kConsumerWarps * NB * 4);
-  L.total = L.z + round16(size_t(rows_cap) * NB * 4);
-  return L;
-}
-
-// Segments of step `st` owned by this CTA, in streaming order: all A rows
-// (kind kDot) then all B rows (kind kRank1).
-// f(proj, kind, src, row_bytes, rows, zrow0, j0)
-template <typename WT, class F>
-LR_DEV void for_each_segment(const ChainStep& st, F&& f) {
-  int r0, r1;
-  split_range(st.total_rows, blockIdx.x, gridDim.x, &r0, &r1);
-  for (int kind = kDot; kind <= kRank1; ++kind) {
-    int begin = 0;
-    for (int p = 0; p < st.n; ++p) {
-      const ChainProj& pr = st.p[p];
-      const int a = max(r0, begin), b = min(r1, begin + pr.rows);
-      if (a < b) {
-        const int j0 = a - begin;
-        if (kind == kDot)
-          f(p, kDot, reinterpret_cast<const unsigned char*>(pr.A) + size_t(j0) * st.d_in * sizeof(WT),
-            st.d_in * int(sizeof(WT)), b - a, a - r0, j0);
-        else
-          f(p, kRank1, reinterpret_cast<const unsigned char*>(pr.B) + size_t(j0) * pr.d_out * sizeof(WT),
-            pr.d_out * int(sizeof(WT)), b - a, a - r0, j0);
-      }
-      begin += pr.rows;
-    }
-  }
-}
-
-LR_DEV int step_rows(const ChainStep& st) {
-  int r0, r1;
-  split_range(st.total_rows, blockIdx.x, gridDim.x, &r0, &r1);
-  return r1 - r0;
-}
-
-LR_DEV int acc_offset(const ChainStep& st, int p, int nb) {
-  int o = 0;
-  for (int q = 0; q < p; ++q) o += nb * st.p[q].d_out;
-  return o;
-}
-
-LR_DEV int acc_used(const ChainStep& st, int nb) { return acc_offset(st, st.n, nb); }
-
-template <typename WT>
-LR_DEV void chain_produce(const ChainParams& P, unsigned char* ring, uint64_t* full, uint64_t* empty, int stages) {
-  int st = 0;
-  bool ok = true;
-  for (int s = 0; s < P.n_steps && ok; ++s) {
-    for_each_segment<WT>(P.step[s], [&](int, int, const unsigned char* src, int row_bytes, int rows, int, int) {
-      const int rps = rows_per_stage(row_bytes);
-      for (int r = 0; r < rows && ok; r += rps) {
-        const int k = min(rps, rows - r);
-        const int slot = st % stages, round = st / stages;
-        if (round > 0 && !mbar_wait_bounded(&empty[slot], uint32_t(round - 1) & 1u, P.err)) {
-          ok = false;
-          return;
-        }
-        const uint32_t bytes = uint32_t(k) * uint32_t(row_bytes);
-        mbar_arrive_expect_tx(&full[slot], bytes);
-        bulk_g2s(ring + size_t(slot) * kStageBytes, src + size_t(r) * row_bytes, bytes, &full[slot]);
-        ++st;
-      }
-    });
-  }
-}
-
-// Grid barrier among the consumer threads of every CTA.  words[0] counts
-// arrivals over the whole launch; barrier k is passed once it reaches
-// gridDim.x * (k + 1).  Bounded: gives up after ~2^22 polls, setting the
-// device error word.
-LR_DEV void consumer_grid_barrier(unsigned int* words, unsigned int target, int* err) {
-  __threadfence();
-  consumer_sync();
-  if (threadIdx.x == 0) {
-    atomicAdd(words, 1u);
-    uint32_t i = 0;
-    while (ld_acquire_u32(words) < target) {
-      if (++i > (1u << 22)) {
-        set_device_error(err, kErrGridBarrier);
-        break;
-      }
-      __nanosleep(20);
-    }
-  }
-  consumer_sync();
-  __threadfence();
-}
-
-template <typename WT, int NB, int LPW>
-__global__ void __launch_bounds__(kThreads, 1) chain_kernel(const __grid_constant__ ChainParams P, int stages,
-                                                            int rows_cap, int x_elems_max) {
-  using XT = typename std::conditional<sizeof(WT) == 4, float, __nv_bfloat16>::type;
-  using YT = XT;
-  extern __shared__ __align__(128) unsigned char smem[];
-  __shared__ __align__(8) uint64_t full[kChainStagesMax];
-  __shared__ __align__(8) uint64_t empty[kChainStagesMax];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const ChainLayout L = chain_layout<NB>(stages, x_elems_max, rows_cap);
-  unsigned char* ring = smem;
-  float* xs = reinterpret_cast<float*>(smem + L.x);
-  float* part = reinterpret_cast<float*>(smem + L.part);
-  float* zs = reinterpret_cast<float*>(smem + L.z);
-  const bool f16 = P.scale_f16 != 0;
-  const int nb = P.nb;
-
-  pdl_launch_dependents();
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < stages; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], kConsumerWarps);
-    }
-    fence_mbar_init();
-  }
-  __syncthreads();
-
-  if (warp == kConsumerWarps) {
-    if (lane == 0) chain_produce<WT>(P, ring, full, empty, stages);
-  } else {
-    const int cw = warp;
-    pdl_wait();
-    int st = 0;
-    bool failed = false;
-    for (int s = 0; s < P.n_steps; ++s) {
-      const ChainStep& S = P.step[s];
-      // ---- stage this step's input (fp32) ----
-      {
-        const int n = nb * S.d_in;
-        const int set_prev = (s + 2) % 3;
-        for (int i = threadIdx.x * 4; i < NB * S.d_in; i += kConsumers * 4) {
-          float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-          if (i < n) {
-            if (S.input_step < 0) {
-              const XT* xg = reinterpret_cast<const XT*>(P.x) + i;
-              if constexpr (sizeof(XT) == 4) {
-                v = *reinterpret_cast<const float4*>(xg);
-              } else {
-                const uint2 u = *reinterpret_cast<const uint2*>(xg);
-                v = make_float4(__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xffff0000u),
-                                __uint_as_float(u.y << 16), __uint_as_float(u.y & 0xffff0000u));
-              }
-            } else if (S.input_step == s - 1) {
-              const ChainStep& I = P.step[S.input_step];
-              const float* a = P.acc + size_t(set_prev) * P.acc_set + acc_offset(I, S.input_proj, nb) + i;
-              v = ld_cg_f4(a);
-              const void* sB = I.p[S.input_proj].sB;
-              if (sB) {
-                const int k = i % S.d_in;
-                v.x *= load_scale(sB, k, f16); v.y *= load_scale(sB, k + 1, f16);
-                v.z *= load_scale(sB, k + 2, f16); v.w *= load_scale(sB, k + 3, f16);
-              }
-            } else {
-              const YT* yg = reinterpret_cast<const YT*>(P.step[S.input_step].p[S.input_proj].y) + i;
-              if constexpr (sizeof(YT) == 4) {
-                v = ld_cg_f4(reinterpret_cast<const float*>(yg));
-              } else {
-                uint2 u;
-                asm volatile("ld.global.cg.v2.u32 {%0,%1}, [%2];" : "=r"(u.x), "=r"(u.y) : "l"(yg) : "memory");
-                v = make_float4(__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xffff0000u),
-                                __uint_as_float(u.y << 16), __uint_as_float(u.y & 0xffff0000u));
-              }
-            }
-          }
-          *reinterpret_cast<float4*>(xs + i) = v;
-        }
-      }
-      consumer_sync();
-      float xr[NB][8];
-      const bool x_in_regs = NB <= 2 && (S.d_in + kLineElems - 1) / kLineElems <= kConsumerWarps;
-#pragma unroll
-      for (int b = 0; b < NB; ++b)
-#pragma unroll
-        for (int e = 0; e < 8; ++e) xr[b][e] = 0.f;
-      {
-        const int col = cw * kLineElems + lane * 8;
-        if (x_in_regs && col < S.d_in) {
-#pragma unroll
-          for (int b = 0; b < NB; ++b)
-            SChunk<float>::load(reinterpret_cast<const unsigned char*>(xs + size_t(b) * S.d_in + col), xr[b]);
-        }
-      }
-      // ---- phase A then phase B over this CTA's rows of the step ----
-      float acc[LPW][NB][8];
-#pragma unroll
-      for (int li = 0; li < LPW; ++li)
-#pragma unroll
-        for (int b = 0; b < NB; ++b)
-#pragma unroll
-          for (int e = 0; e < 8; ++e) acc[li][b][e] = 0.f;
-      bool zready = false;
-      const int nrows = step_rows(S);
-      float* acc_set = P.acc + size_t(s % 3) * P.acc_set;
-      for_each_segment<WT>(S, [&](int p, int kind, const unsigned char*, int row_bytes, int rows, int zrow0, int) {
-        if (kind == kRank1 && !zready) {
-          consumer_sync();
-          for (int i = threadIdx.x; i < nrows * NB; i += kConsumers) {
-            const int r = i / NB, b = i % NB;
-            float v = 0.f;
-#pragma unroll 4
-            for (int w = 0; w < kConsumerWarps; ++w) v += part[(r * kConsumerWarps + w) * NB + b];
-            // scale of A for local row r: find its A segment
-            float sc = 1.f;
-            for_each_segment<WT>(S, [&](int q, int kq, const unsigned char*, int, int rq, int z0, int j0) {
-              if (kq == kDot && r >= z0 && r < z0 + rq && S.p[q].sA) sc = load_scale(S.p[q].sA, j0 + (r - z0), f16);
-            });
-            zs[r * NB + b] = v * sc;
-          }
-          consumer_sync();
-          zready = true;
-        }
-        const int elems = row_bytes / int(sizeof(WT));
-        const int rps = rows_per_stage(row_bytes);
-        for (int r = 0; r < rows; r += rps) {
-          const int k = min(rps, rows - r);
-          const int slot = st % stages, round = st / stages;
-          if (!failed && !mbar_wait_bounded(&full[slot], uint32_t(round) & 1u, P.err)) failed = true;
-          if (!failed) {
-            const unsigned char* stage = ring + size_t(slot) * kStageBytes;
-            if (kind == kDot)
-              consume_dot<WT, float, NB>(stage, k, elems, xs, xr, x_in_regs, part, zrow0 + r, cw, lane);
-            else
-              consume_rank1<WT, NB, LPW>(stage, k, elems, zs, zrow0 + r, acc, cw, lane);
-          }
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&empty[slot]);
-          ++st;
-        }
-        if (kind == kRank1 && !failed) flush_rank1<NB, LPW>(acc, acc_set + acc_offset(S, p, nb), elems, nb, cw, lane);
-      });
-      // ---- all partial outputs of step s are in: write them, retire set s-1 ----
-      consumer_grid_barrier(P.bar, gridDim.x * unsigned(s + 1), P.err);
-      {
-        const int total = acc_used(S, nb) / 8;
-        const int c0 = int((long long)total * blockIdx.x / gridDim.x);
-        const int c1 = int((long long)total * (blockIdx.x + 1) / gridDim.x);
-        const bool last = s == P.n_steps - 1;
-        for (int c = c0 + int(threadIdx.x); c < c1; c += kConsumers) {
-          int off = c * 8, p = 0;
-          while (p < S.n - 1 && off >= nb * S.p[p].d_out) { off -= nb * S.p[p].d_out; ++p; }
-          const ChainProj& pr = S.p[p];
-          float* a = acc_set + acc_offset(S, p, nb) + off;
-          const float4 v0 = ld_cg_f4(a), v1 = ld_cg_f4(a + 4);
-          float v[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-          if (pr.sB) {
-            const int k = off % pr.d_out;
-#pragma unroll
-            for (int e = 0; e < 8; ++e) v[e] *= load_scale(pr.sB, k + e, f16);
-          }
-          YT* y = reinterpret_cast<YT*>(pr.y) + off;
-          if constexpr (sizeof(YT) == 2) {
-            uint4 o;
-            uint32_t* ow = reinterpret_cast<uint32_t*>(&o);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * e], v[2 * e + 1]);
-              ow[e] = *reinterpret_cast<uint32_t*>(&h);
-            }
-            *reinterpret_cast<uint4*>(y) = o;
-          } else {
-            *reinterpret_cast<float4*>(y) = make_float4(v[0], v[1], v[2], v[3]);
-            *reinterpret_cast<float4*>(y + 4) = make_float4(v[4], v[5], v[6], v[7]);
-          }
-          if (last) {
-            st_cg_f4(a, make_float4(0.f, 0.f, 0.f, 0.f));
-            st_cg_f4(a + 4, make_float4(0.f, 0.f, 0.f, 0.f));
-          }
-        }
-        if (s >= 1) {
-          const ChainStep& Sp = P.step[s - 1];
-          float* prev = P.acc + size_t((s + 2) % 3) * P.acc_set;
-          const int tp = acc_used(Sp, nb) / 8;
-          const int d0 = int((long long)tp * blockIdx.x / gridDim.x);
-          const int d1 = int((long long)tp * (blockIdx.x + 1) / gridDim.x);
-          for (int c = d0 + int(threadIdx.x); c < d1; c += kConsumers) {
-            st_cg_f4(prev + c * 8, make_float4(0.f, 0.f, 0.f, 0.f));
-            st_cg_f4(prev + c * 8 + 4, make_float4(0.f, 0.f, 0.f, 0.f));
-          }
-        }
-      }
-    }
-  }
-  // ---- leave the barrier counters at zero for the next launch ----
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    __threadfence();
-    const unsigned prev = atomicAdd(P.bar + 1, 1u);
-    if (prev == gridDim.x - 1) {
-      atomicExch(P.bar, 0u);
-      atomicExch(P.bar + 1, 0u);
-    }
-  }
-}
-
-template <typename WT, int NB, int LPW>
-cudaError_t launch_chain_t(const ChainParams& p, int grid, int rows_cap, int x_elems_max, cudaStream_t s) {
-  int stages = kChainStagesMax;
-  size_t bytes = 0;
-  for (; stages >= 2; --stages) {
-    bytes = chain_layout<NB>(stages, x_elems_max, rows_cap).total;
-    if (bytes <= kSmemLimit - 2048) break;
-  }
-  if (bytes > kSmemLimit - 2048) return cudaErrorInvalidValue;
-  auto kern = chain_kernel<WT, NB, LPW>;
-  cudaError_t e = ensure_smem(kern, bytes);
-  if (e != cudaSuccess) return e;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = bytes;
-  cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, p, stages, rows_cap, x_elems_max);
-}
-
-template <typename WT>
-cudaError_t launch_chain_w(const ChainParams& p, int sm_count, cudaStream_t s) {
-  int max_dout = 0, x_max = 0, max_rows = 0;
-  for (int i = 0; i < p.n_steps; ++i) {
-    const ChainStep& st = p.step[i];
-    x_max = std::max(x_max, st.d_in);
-    max_rows = std::max(max_rows, st.total_rows);
-    for (int q = 0; q < st.n; ++q) max_dout = std::max(max_dout, st.p[q].d_out);
-    if (size_t(st.d_in) * sizeof(WT) > size_t(kStageBytes)) return cudaErrorInvalidValue;
-  }
-  if (size_t(max_dout) * sizeof(WT) > size_t(kStageBytes)) return cudaErrorInvalidValue;
-  const int lpw = lpw_for(max_dout);
-  const int grid = std::min(sm_count, std::max(max_rows, 1));
-  const int rows_cap = (max_rows + grid - 1) / grid;
-  const int nb = p.nb;
-#define LR_CCASE(NB_, LPW_) \
-  if (lpw == LPW_ && nb <= NB_) return launch_chain_t<WT, NB_, LPW_>(p, grid, rows_cap, x_max, s);
-  LR_CCASE(1, 1) LR_CCASE(2, 1) LR_CCASE(4, 1) LR_CCASE(8, 1)
-  LR_CCASE(1, 2) LR_CCASE(2, 2) LR_CCASE(4, 2)
-  LR_CCASE(1, 4) LR_CCASE(2, 4)
-  LR_CCASE(1, 8)
-#undef LR_CCASE
-  return cudaErrorInvalidValue;
-}
-
-// ---------------------------------------------------------------------------
 // Launch helpers
 // ---------------------------------------------------------------------------
 template <typename WT, typename XT, typename YT, int NB, int LPW, int MODE>
@@ -1115,16 +747,5 @@ cudaError_t launch_lr_rank1(const Rank1Params& p, lr_dtype_t w_dtype, int sm_cou
 }
 
 cudaError_t launch_ffn(const FfnParams& p, int sm_count, cudaStream_t s) { return launch_ffn_impl(p, sm_count, s); }
-
-size_t chain_workspace_bytes(const ChainParams& p) { return kTicketBytes + size_t(3) * p.acc_set * 4; }
-
-cudaError_t launch_chain(const ChainParams& p, lr_dtype_t w_dtype, int sm_count, cudaStream_t s) {
-  switch (w_dtype) {
-    case LR_F32: return launch_chain_w<float>(p, sm_count, s);
-    case LR_BF16: return launch_chain_w<__nv_bfloat16>(p, sm_count, s);
-    case LR_I8: return launch_chain_w<int8_t>(p, sm_count, s);
-    default: return cudaErrorInvalidValue;
-  }
-}
 
 }  // namespace lr
