@@ -82,6 +82,13 @@ def reduce_max(value: float, device=None) -> float:
     return float(t.item())
 
 
+def whole_job_throughput(world: int, batch: int, ms_step_max: float) -> float:
+    """Tokens/s of the whole job: every rank decodes `batch` tokens per step
+    (independent replicas, no data-path collective), and the step time is the
+    slowest rank's."""
+    return world * batch / (ms_step_max * 1e-3)
+
+
 def barrier(device=None):
     import torch.distributed as dist
     if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
@@ -101,6 +108,15 @@ def host_cores() -> int:
 # ---------------------------------------------------------------------------
 # workload
 # ---------------------------------------------------------------------------
+# DRAM bytes (read + write) per algorithmic byte of chain_kernel<bf16, batch 1>,
+# from one ncu capture of the same kernel on the 2-layer case (163.92 MB of
+# DRAM traffic for 159.48 MB of algorithmic bytes; summary and command in
+# profiles/chain_kernel_bf16_b1_llama7b_2layers.md).  DRAM traffic grows with
+# the factor bytes streamed, so a full launch's traffic is this ratio times its
+# algorithmic bytes.  Valid for that kernel build and batch 1 only.
+CHAIN_TRAFFIC_PER_ALG_BYTE = 163.92e6 / 159481856
+
+
 def algorithmic_bytes_per_step(ranks, batch: int) -> int:
     """Factor bytes (bf16) of all 128 projections plus activation reads/writes."""
     factor = int(sum(int(r) * (HIDDEN + HIDDEN) * 2 for r in ranks[:LAYERS].reshape(-1)))
@@ -294,7 +310,7 @@ def run_ours(args) -> None:
     bytes_step = algorithmic_bytes_per_step(ranks, batch)
     peak, peak_kind = measured_hbm_peak()
     achieved = bytes_step / (ms_step * 1e-3) / 1e9
-    tokens_s = world * batch / (ms_step * 1e-3)
+    tokens_s = whole_job_throughput(world, batch, ms_step)
     out = {
         "metric": METRIC, "value": tokens_s, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
@@ -306,12 +322,15 @@ def run_ours(args) -> None:
         "layer_us": ms_step * 1e3 / LAYERS,
         "hbm_gbs": achieved,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                     "traffic": None, "peak_source": peak_kind,
+                     "traffic": (round(CHAIN_TRAFFIC_PER_ALG_BYTE * bytes_step) if batch == 1 else None),
+                     "traffic_note": "ncu dram__bytes_read.sum + dram__bytes_write.sum of a 2-layer launch, "
+                                     "scaled by factor bytes to the full launch",
+                     "peak_source": peak_kind,
                      "kernel": "chain_kernel<bf16, batch 1> (factorised-linear chain)",
                      "note": "the step is one launch of this kernel only, so its launch duration is the "
                              "event-timed step time"},
         "gpu_launches": launches_per_step * args.steps,
-        "e2e": {"value": world * batch / (ms_e2e * 1e-3), "unit": "tokens/s",
+        "e2e": {"value": whole_job_throughput(world, batch, ms_e2e), "unit": "tokens/s",
                 "h2d_bytes_per_step": int(x_host.numel() * x_host.element_size()),
                 "d2h_bytes_per_step": int(y_host.numel() * y_host.element_size())},
         "clocks": clk,

@@ -77,9 +77,11 @@ struct Cfg {
 
 LR_HD_INLINE int ceil_div(int a, int b) { return (a + b - 1) / b; }
 
-LR_DEV void split_range(long long total, int part, int parts, int* a, int* b) {
-  *a = int(total * part / parts);
-  *b = int(total * (part + 1) / parts);
+// [a, b) of `total` items for part `part` of `parts` (total * parts < 2^31:
+// rows and 8-float chunks of one step over at most one CTA per SM).
+LR_DEV void split_range(int total, int part, int parts, int* a, int* b) {
+  *a = int(unsigned(total) * unsigned(part) / unsigned(parts));
+  *b = int(unsigned(total) * unsigned(part + 1) / unsigned(parts));
 }
 
 // How the warps cover rows of `row_bytes`: wpr warps per row (a power of two,
