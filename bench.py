@@ -48,6 +48,8 @@ def parse(argv=None):
     ap.add_argument("--batch", type=int, default=1)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--secondary", action="store_true",
+                    help="time the FFN, latent-KV and W8A8 rows instead (one JSON line each)")
     ap.add_argument("--layers", type=int, default=LAYERS,
                     help="layers in the stack (default 32; fewer only for profiling small cases)")
     return ap.parse_args(argv)
@@ -379,10 +381,130 @@ def run_reference(args) -> None:
     print(json.dumps(out), flush=True)
 
 
+def _time_rotating(fn, n_copies: int, iters: int, warmup: int = 3) -> float:
+    """Mean ms per call of fn(i), copy i % n_copies: `iters` calls captured in
+    one CUDA graph (no host time between launches), replayed after warm-up,
+    timed with CUDA events on the replay stream."""
+    import torch
+    for i in range(warmup):
+        fn(i % n_copies)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for i in range(iters):
+            fn(i % n_copies)
+    g.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    g.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    del g
+    return e0.elapsed_time(e1) / iters
+
+
+def run_secondary(args) -> None:
+    """One JSON line per further hot-path row, each against its own roofline:
+    the hybrid int8 SwiGLU FFN (7B shapes, batch 1), latent-KV split-K decode
+    (batch 8, 32 heads, rank 32, ctx 16384) and the W8A8 prefill projections
+    of one 13B layer (2048 tokens).  Weight or cache copies rotate so the
+    working set exceeds L2."""
+    import torch
+
+    import decode_lr_linear_b200 as lr
+    from decode_lr_linear_b200 import synth
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    hbm, hbm_kind = measured_hbm_peak()
+    peaks = {}
+    peaks_path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(peaks_path):
+        with open(peaks_path) as f:
+            peaks = json.load(f)
+    lines = []
+
+    # ---- hybrid FFN (int8 weights + fp16 scales), 4 copies of one layer ----
+    d = synth.make_hybrid_ffn(seed=0)
+
+    def ffn_copy():
+        g = lambda t: t.to(dev)
+        return lr.FfnWeights(d["hidden"], d["inter"], d["n_lr"], d["rank"], g(d["A_q"]), g(d["s_A"]), g(d["B_q"]),
+                             g(d["s_B"]), g(d["D_q"]), g(d["s_D"]), g(d["Wd_q"]), g(d["s_d"]))
+    ffns = [ffn_copy() for _ in range(4)]
+    w_bytes = sum(int(d[k].numel() * d[k].element_size()) for k in ("A_q", "s_A", "B_q", "s_B", "D_q", "s_D",
+                                                                  "Wd_q", "s_d"))
+    for batch in (1, 8):
+        x = synth.make_activations(batch, d["hidden"], seed=0, key=(30, batch), outliers=4).to(dev)
+        y = torch.empty_like(x)
+        ws = lr.workspace(lr.lr_swiglu_ffn_workspace_size(ffns[0], batch), dev)
+        ms = _time_rotating(lambda i: lr.lr_swiglu_ffn(ffns[i], x, y, ws), 4, 40)
+        alg = w_bytes + 2 * batch * d["hidden"] * 2
+        gbs = alg / (ms * 1e-3) / 1e9
+        lines.append({"row": "a4-a7 hybrid int8 SwiGLU FFN", "workload": f"7B FFN (hidden 4096, inter 11008, "
+                      f"n_lr 8192, rank 1536), batch {batch}", "us_per_layer": ms * 1e3,
+                      "tokens_s_32_layers": batch / (ms * 1e-3 * 32),
+                      "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
+                                   "peak_source": hbm_kind, "algorithmic_bytes": alg}})
+    del ffns
+
+    # ---- latent-KV split-K decode (absorbed), ctx 16384 ----
+    kvd = synth.make_latent_kv(batch=8, heads=32, ctx=16384, seed=0)
+    kv = lr.LatentKv(kvd["batch"], kvd["heads"], kvd["ctx"], kvd["B_K"].to(dev), kvd["B_V"].to(dev), kvd["scale"],
+                     0, 0)
+    q, CK, CV, sl = (kvd[k].to(dev) for k in ("q", "C_K", "C_V", "seq_lens"))
+    out = torch.empty(kv.batch, kv.heads, kv.head_dim, dtype=torch.bfloat16, device=dev)
+    kws = lr.workspace(lr.lr_latent_kv_workspace_size(kv), dev)
+    ms = _time_rotating(lambda i: lr.lr_latent_kv_decode(kv, q, CK, CV, sl, out, kws), 1, 40)
+    alg = int(CK.numel() * 2 + CV.numel() * 2 + kvd["B_K"].numel() * 2 + kvd["B_V"].numel() * 2)
+    gbs = alg / (ms * 1e-3) / 1e9
+    lines.append({"row": "a8-a10 latent-KV split-K decode", "workload": "batch 8, heads 32, rank 32, head_dim 128, "
+                  "ctx 16384 (1.07 GB of latent cache, larger than L2)", "us": ms * 1e3,
+                  "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
+                               "peak_source": hbm_kind, "algorithmic_bytes": alg}})
+    del q, CK, CV, sl, kv, kvd, out, kws
+
+    # ---- W8A8 prefill: the 7 projections of one 13B layer, 2048 tokens ----
+    T = 2048
+    shapes = synth.prefill_shapes()
+    ranks = synth.prefill_ranks(0)
+    projs, ops = [], 0
+    for j, name in enumerate(synth.PREFILL_PROJ):
+        d_in, d_out = shapes[name]
+        r = int(ranks[0, j])
+        pp = synth.make_prefill_projection(d_in, d_out, r, seed=0, key=(d_in, d_out, r))
+        f = lr.Factor(pp["A_q"].to(dev), pp["B_q"].to(dev), pp["s_A"].to(dev), pp["s_B"].to(dev))
+        xin = synth.make_activations(T, d_in, seed=0, key=(60, d_in, T), outliers=max(1, d_in // 1000)).to(dev)
+        xq, sx = lr.lr_quantize_per_token(xin)
+        ws = lr.workspace(lr.lr_linear_workspace_size(f, T, w8a8=True), dev)
+        y = torch.empty(T, d_out, dtype=torch.bfloat16, device=dev)
+        projs.append((f, xq, sx, y, ws))
+        ops += 2 * T * r * (d_in + d_out)
+
+    def layer(_):
+        for f, xq, sx, y, ws in projs:
+            lr.lr_linear(f, xq, y, ws, x_scale=sx)
+    ms = _time_rotating(layer, 1, 20)
+    tops = ops / (ms * 1e-3) / 1e12
+    bf16 = peaks.get("bf16_tflops")
+    i8_peak = 2.0 * bf16 if bf16 else 2.0 * 1590.0
+    lines.append({"row": "a11-a12 W8A8 prefill (tcgen05 int8)", "workload": "one 13B layer (q,k,v,o,gate,up,down; "
+                  "ranks of layer 0), 2048 tokens, int8 x int8 -> int32", "us_per_layer": ms * 1e3,
+                  "tokens_s_40_layers": T / (ms * 1e-3 * 40),
+                  "roofline": {"bound": "tensor", "achieved": tops, "peak": i8_peak, "unit": "TOPS",
+                               "frac": tops / i8_peak, "peak_source": ("of measured bf16 x 2 (nominal int8/bf16 "
+                                                                       "ratio)" if bf16 else "of fallback x 2"),
+                               "algorithmic_ops": ops}})
+    for ln in lines:
+        print(json.dumps(ln), flush=True)
+
+
 def main(argv=None):
     args = parse(argv)
     if args.impl == "reference":
         run_reference(args)
+    elif args.secondary:
+        run_secondary(args)
     else:
         run_ours(args)
     try:
