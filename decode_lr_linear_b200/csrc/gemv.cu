@@ -269,10 +269,10 @@ LR_DEV void produce(const Plan& pl, unsigned char* ring, uint64_t* full, uint64_
 // the generation changes.  All threads of the CTA call it; on return every
 // CTA's earlier global writes and reductions are visible.
 LR_DEV void grid_barrier(unsigned int* words, int* err) {
-  __threadfence();
   __syncthreads();
   if (threadIdx.x == 0) {
     const unsigned gen = ld_acquire_u32(words + 1);
+    __threadfence();  // after the CTA barrier: covers every thread's earlier writes
     const unsigned prev = atomicAdd(words, 1u);
     if (prev == gridDim.x - 1) {
       atomicExch(words, 0u);
@@ -285,12 +285,10 @@ LR_DEV void grid_barrier(unsigned int* words, int* err) {
           set_device_error(err, kErrGridBarrier);
           break;
         }
-        __nanosleep(32);
       }
     }
   }
   __syncthreads();
-  __threadfence();
 }
 
 // One output of a split reduction: y[b][k] = acc[b][k] * scale[k] (optional).
@@ -719,17 +717,31 @@ cudaError_t launch_ffn_impl(const FfnParams& p0, int sm_count, cudaStream_t s) {
   K1.x_elems = p0.hidden;
   K2.rows_cap = (p0.inter + g2 - 1) / g2;
   K2.x_elems = 0;
-  const int nb_max = std::min(8 / lpw1, 8 / lpw2);
-  for (int b0 = 0; b0 < p0.nb; b0 += nb_max) {
+  // Each phase takes as many batch rows per launch as its accumulator
+  // registers allow (8 / lines per warp; at most 4 in phase 2, whose 8-row
+  // instantiation spills).  Phase 1 writes every row of the intermediate
+  // gate/up accumulator and h_D first, so phase 2 streams W_down once per
+  // group of up to 4 rows even when phase 1 needs more launches.
+  const int nb1 = 8 / lpw1, nb2 = std::min(4, 8 / lpw2);
+  for (int b0 = 0; b0 < p0.nb; b0 += nb1) {
     FfnParams f = p0;
-    f.nb = std::min(nb_max, p0.nb - b0);
+    f.nb = std::min(nb1, p0.nb - b0);
     f.x = reinterpret_cast<const __nv_bfloat16*>(p0.x) + size_t(b0) * p0.hidden;
-    f.y = reinterpret_cast<__nv_bfloat16*>(p0.y) + size_t(b0) * p0.hidden;
+    f.gu_acc = p0.gu_acc + size_t(b0) * 2 * p0.n_lr;
+    f.h_dense = p0.h_dense + size_t(b0) * p0.n_dense;
     K1.f = f;
-    K2.f = f;
     cudaError_t e = dispatch<int8_t, __nv_bfloat16, __nv_bfloat16, kFfn1>(K1, f.nb, lpw1, g_lr + g_d, s);
     if (e != cudaSuccess) return e;
-    e = dispatch<int8_t, __nv_bfloat16, __nv_bfloat16, kFfn2>(K2, f.nb, lpw2, g2, s);
+  }
+  for (int b0 = 0; b0 < p0.nb; b0 += nb2) {
+    FfnParams f = p0;
+    f.nb = std::min(nb2, p0.nb - b0);
+    f.y = reinterpret_cast<__nv_bfloat16*>(p0.y) + size_t(b0) * p0.hidden;
+    f.gu_acc = p0.gu_acc + size_t(b0) * 2 * p0.n_lr;
+    f.h_dense = p0.h_dense + size_t(b0) * p0.n_dense;
+    f.y_acc = p0.y_acc + size_t(b0) * p0.hidden;
+    K2.f = f;
+    cudaError_t e = dispatch<int8_t, __nv_bfloat16, __nv_bfloat16, kFfn2>(K2, f.nb, lpw2, g2, s);
     if (e != cudaSuccess) return e;
   }
   return cudaSuccess;
