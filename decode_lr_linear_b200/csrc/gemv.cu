@@ -1,26 +1,20 @@
-// Decode-time (small batch) kernels for factorised linears and the hybrid
-// SwiGLU FFN on CUDA cores, sm_100a.
+// Decode-time (small batch) hybrid SwiGLU FFN on CUDA cores, sm_100a: LASER
+// ("Hybrid SVD-Quantization for FFNs", "System Implementation").
 //
-// A factorised linear y = (x A) B is evaluated as a sum of rank-1 terms,
-// y = sum_j z_j b_j with z_j = x . a_j, where a_j / b_j are the latent-major
-// rows of the two factors.  Each CTA owns a contiguous block of latent rows.
-// One producer warp streams the CTA's rows of A and then of B through a ring
-// of shared-memory stages with bulk asynchronous copies (cp.async.bulk,
-// completing on mbarriers); sixteen consumer warps compute from shared memory:
-//   phase A: z_j = a_j . x for the CTA's rows (x staged in shared memory),
-//   phase B: partial y += z_j b_j, added into an fp32 accumulator in L2 with
-//            vector reductions (red.global.add.v4.f32).
-// The last CTA to arrive (atomic ticket, no waiting) converts the accumulator
-// to the output type and zeroes it again.  Each factor byte is read once;
-// the weight copies are issued before the programmatic-dependent-launch wait,
-// so they overlap the tail of the preceding kernel.
-//
-// The same engine evaluates the hybrid FFN of LASER ("Hybrid SVD-Quantization
-// for FFNs", "System Implementation") in two launches:
-//   phase 1: low-rank branch  z = x A', [g_S,u_S] += z_j b'_j  (reduction)
+// One streaming engine runs both launches.  Each CTA owns a contiguous block
+// of weight rows; one producer warp streams them through a ring of
+// shared-memory stages with bulk asynchronous copies (cp.async.bulk,
+// completing on mbarriers), and sixteen consumer warps compute from shared
+// memory:
+//   phase 1: low-rank branch  z = x A', [g_S,u_S] += z_j b'_j (fp32 vector
+//            reductions into L2, red.global.add.v4.f32);
 //            dense branch     [g_D,u_D] = x D' row dots, SwiGLU in the epilogue
 //   phase 2: h = [silu(g_S) u_S, h_D]; y += h_c w_c over input channels of
-//            W_down (reduction), last CTA applies the output scales.
+//            W_down (reduction); after a grid barrier each CTA applies the
+//            output scales to its slice of y and zeroes the accumulator.
+// Each weight byte is read once per launch; the weight copies are issued
+// before the programmatic-dependent-launch wait, so they overlap the tail of
+// the preceding kernel.  The factorised linears themselves run in chain.cu.
 #include <algorithm>
 #include <cstring>
 #include <type_traits>
@@ -44,7 +38,7 @@ constexpr int kRowGroup = 4;               // rows reduced together in phase A (
 constexpr int kMaxSegs = 2 * kMaxGroup;
 constexpr size_t kSmemLimit = 227 * 1024;
 
-enum Mode : int { kLinear = 0, kFfn1 = 1, kFfn2 = 2 };
+enum Mode : int { kFfn1 = 1, kFfn2 = 2 };
 enum SegKind : int { kDot = 0, kRank1 = 1 };
 
 struct Seg {
@@ -54,7 +48,6 @@ struct Seg {
   int rps;                   // rows per ring stage
   int kind;                  // kDot: row . x ; kRank1: acc += z_row * row
   int zrow0;                 // CTA-local index of the first row (into part / z)
-  int proj;                  // projection (kLinear)
 };
 
 struct Plan {
@@ -66,7 +59,6 @@ struct Plan {
 };
 
 struct KParams {
-  Rank1Params r;
   FfnParams f;
   int g_lr;                  // kFfn1: CTAs of the low-rank branch
   int stages;                // ring stages in use
@@ -94,12 +86,6 @@ LR_HD_INLINE Layout layout_for(int stages, int x_elems, int x_esize, int rows_ca
 
 // ---- shared-memory chunk loads (8 elements) --------------------------------
 template <typename T> struct SChunk;
-template <> struct SChunk<float> {
-  LR_DEV static void load(const unsigned char* p, float* f) {
-    const float4 a = *reinterpret_cast<const float4*>(p), b = *reinterpret_cast<const float4*>(p + 16);
-    f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w; f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
-  }
-};
 template <> struct SChunk<__nv_bfloat16> {
   LR_DEV static void load(const unsigned char* p, float* f) { bf16x8_to_f32(*reinterpret_cast<const uint4*>(p), f); }
 };
@@ -372,26 +358,8 @@ LR_DEV void build_plan(const KParams& K, Plan& pl) {
     g.rps = rows_per_stage(row_bytes);
     g.kind = kind;
     g.zrow0 = zrow0;
-    g.proj = proj;
   };
-  if constexpr (MODE == kLinear) {
-    const Rank1Params& P = K.r;
-    int r0, r1;
-    split_range(P.total_rows, blockIdx.x, gridDim.x, &r0, &r1);
-    pl.nrows = r1 - r0;
-    pl.row_base = r0;
-    for (int kind = kDot; kind <= kRank1; ++kind) {
-      for (int p = 0; p < P.n_proj; ++p) {
-        const Rank1Proj& pr = P.proj[p];
-        const int a = max(r0, pr.row_begin), b = min(r1, pr.row_begin + pr.rows);
-        if (a >= b) continue;
-        if (kind == kDot)
-          add(pr.A, size_t(a - pr.row_begin), P.d_in * int(sizeof(WT)), b - a, kDot, a - r0, p);
-        else
-          add(pr.B, size_t(a - pr.row_begin), pr.d_out * int(sizeof(WT)), b - a, kRank1, a - r0, p);
-      }
-    }
-  } else if constexpr (MODE == kFfn1) {
+  if constexpr (MODE == kFfn1) {
     const FfnParams& F = K.f;
     if (int(blockIdx.x) < K.g_lr) {
       int r0, r1;
@@ -421,17 +389,8 @@ LR_DEV void build_plan(const KParams& K, Plan& pl) {
 // Scale of CTA-local row r after phase A (per latent / output channel).
 template <int MODE>
 LR_DEV float row_scale(const KParams& K, const Plan& pl, int r) {
-  const bool f16 = (MODE == kLinear ? K.r.scale_f16 : K.f.scale_f16) != 0;
-  if constexpr (MODE == kLinear) {
-    for (int s = 0; s < pl.nseg; ++s) {
-      const Seg& g = pl.seg[s];
-      if (g.kind == kDot && r >= g.zrow0 && r < g.zrow0 + g.rows) {
-        const Rank1Proj& pr = K.r.proj[g.proj];
-        return pr.sA ? load_scale(pr.sA, pl.row_base + r - pr.row_begin, f16) : 1.f;
-      }
-    }
-    return 1.f;
-  } else {
+  const bool f16 = K.f.scale_f16 != 0;
+  {
     if (pl.role == 0) return load_scale(K.f.sA, pl.row_base + r, f16);
     return load_scale(K.f.sD, pl.row_base + r, f16);
   }
@@ -466,10 +425,10 @@ __global__ void __launch_bounds__(kThreads, (NB <= 1 && LPW <= 2 ? 2 : 1)) strea
     if (lane == 0) produce(pl, ring, full, empty, K.stages, K.err);
   } else {
     const int cw = warp;
-    const int nb = (MODE == kLinear) ? K.r.nb : K.f.nb;
+    const int nb = K.f.nb;
     pdl_wait();
     if constexpr (MODE != kFfn2) {
-      const uint4* xg = reinterpret_cast<const uint4*>(MODE == kLinear ? K.r.x : K.f.x);
+      const uint4* xg = reinterpret_cast<const uint4*>(K.f.x);
       const int n16 = int(size_t(NB) * K.x_elems * sizeof(XT) / 16);
       const int valid16 = int(size_t(nb) * K.x_elems * sizeof(XT) / 16);
       for (int i = threadIdx.x; i < n16; i += kConsumers)
@@ -557,8 +516,7 @@ __global__ void __launch_bounds__(kThreads, (NB <= 1 && LPW <= 2 ? 2 : 1)) strea
       }
       if (g.kind == kRank1 && !failed) {
         float* dst;
-        if constexpr (MODE == kLinear) dst = K.r.proj[g.proj].acc;
-        else if constexpr (MODE == kFfn1) dst = K.f.gu_acc;
+        if constexpr (MODE == kFfn1) dst = K.f.gu_acc;
         else dst = K.f.y_acc;
         flush_rank1<NB, LPW>(acc, dst, elems, nb, cw, lane);
       }
@@ -590,16 +548,9 @@ __global__ void __launch_bounds__(kThreads, (NB <= 1 && LPW <= 2 ? 2 : 1)) strea
   if constexpr (MODE == kFfn1) {
     return;
   } else {
-    unsigned int* words = (MODE == kLinear) ? K.r.ticket : K.f.ticket;
+    unsigned int* words = K.f.ticket;
     grid_barrier(words, K.err);
-    if constexpr (MODE == kLinear) {
-      FinalTarget t[kMaxGroup];
-#pragma unroll
-      for (int p = 0; p < kMaxGroup; ++p)
-        t[p] = FinalTarget{K.r.proj[p].acc, K.r.proj[p].y, K.r.proj[p].sB, K.r.nb * K.r.proj[p].d_out,
-                           K.r.proj[p].d_out};
-      finalize_slice<YT, kMaxGroup>(t, K.r.n_proj, K.r.scale_f16 != 0);
-    } else {
+    {
       FinalTarget t[1] = {FinalTarget{K.f.y_acc, K.f.y, K.f.sd, K.f.nb * K.f.hidden, K.f.hidden}};
       finalize_slice<__nv_bfloat16, 1>(t, 1, K.f.scale_f16 != 0);
     }
@@ -657,33 +608,6 @@ cudaError_t dispatch(const KParams& K, int nb, int lpw, int grid, cudaStream_t s
   LR_CASE(1, 8)
 #undef LR_CASE
   return cudaErrorInvalidValue;
-}
-
-template <typename WT, typename XT, typename YT>
-cudaError_t launch_linear(const Rank1Params& p0, int sm_count, cudaStream_t s) {
-  int max_dout = 0;
-  for (int q = 0; q < p0.n_proj; ++q) max_dout = std::max(max_dout, p0.proj[q].d_out);
-  const int lpw = lpw_for(max_dout);
-  if (lpw == 0) return cudaErrorInvalidValue;
-  if (size_t(p0.d_in) * sizeof(WT) > size_t(kStageBytes) || size_t(max_dout) * sizeof(WT) > size_t(kStageBytes))
-    return cudaErrorInvalidValue;
-  // one CTA per SM at most: the finalize barrier needs every CTA resident
-  const int grid = std::min(sm_count, p0.total_rows);
-  const int nb_max = 8 / lpw;
-  KParams K;
-  std::memset(&K, 0, sizeof(K));
-  K.rows_cap = (p0.total_rows + grid - 1) / grid;
-  K.x_elems = p0.d_in;
-  for (int b0 = 0; b0 < p0.nb; b0 += nb_max) {
-    K.r = p0;
-    K.r.nb = std::min(nb_max, p0.nb - b0);
-    K.r.x = reinterpret_cast<const XT*>(p0.x) + size_t(b0) * p0.d_in;
-    for (int q = 0; q < p0.n_proj; ++q)
-      K.r.proj[q].y = reinterpret_cast<YT*>(p0.proj[q].y) + size_t(b0) * p0.proj[q].d_out;
-    cudaError_t e = dispatch<WT, XT, YT, kLinear>(K, K.r.nb, lpw, grid, s);
-    if (e != cudaSuccess) return e;
-  }
-  return cudaSuccess;
 }
 
 cudaError_t launch_ffn_impl(const FfnParams& p0, int sm_count, cudaStream_t s) {
@@ -748,15 +672,6 @@ cudaError_t launch_ffn_impl(const FfnParams& p0, int sm_count, cudaStream_t s) {
 }
 
 }  // namespace
-
-cudaError_t launch_lr_rank1(const Rank1Params& p, lr_dtype_t w_dtype, int sm_count, cudaStream_t s) {
-  switch (w_dtype) {
-    case LR_F32: return launch_linear<float, float, float>(p, sm_count, s);
-    case LR_BF16: return launch_linear<__nv_bfloat16, __nv_bfloat16, __nv_bfloat16>(p, sm_count, s);
-    case LR_I8: return launch_linear<int8_t, __nv_bfloat16, __nv_bfloat16>(p, sm_count, s);
-    default: return cudaErrorInvalidValue;
-  }
-}
 
 cudaError_t launch_ffn(const FfnParams& p, int sm_count, cudaStream_t s) { return launch_ffn_impl(p, sm_count, s); }
 

@@ -21,32 +21,6 @@ constexpr size_t kTicketBytes = 256;
 // Batch rows handled by one launch of the CUDA-core decode kernels.
 constexpr int kMaxDecodeChunk = 8;
 
-struct Rank1Proj {
-  const void* A;      // [rank, d_in]
-  const void* B;      // [rank, d_out]
-  const void* sA;     // int8: [rank]
-  const void* sB;     // int8: [d_out]
-  float* acc;         // [chunk, d_out] fp32 accumulator (zero on entry and exit)
-  void* y;            // [batch, d_out] output (f32 or bf16), already offset to the chunk
-  int d_out;
-  int rows;           // active latent rows
-  int row_begin;      // first global latent index of this projection
-};
-
-struct Rank1Params {
-  Rank1Proj proj[kMaxGroup];
-  int n_proj;
-  int d_in;
-  int nb;             // batch rows in this launch (<= kMaxDecodeChunk)
-  int total_rows;
-  const void* x;      // [nb, d_in], already offset to the chunk
-  unsigned int* ticket;
-  int scale_f16;
-};
-
-// y = (x A) B for up to kMaxGroup projections sharing x; weight-only paths.
-cudaError_t launch_lr_rank1(const Rank1Params& p, lr_dtype_t w_dtype, int sm_count, cudaStream_t s);
-
 // ---- factorised-linear chains (lr_linear, lr_linear_grouped, lr_linear_chain) ----
 constexpr int kMaxChain = LR_MAX_CHAIN;
 
