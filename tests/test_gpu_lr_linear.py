@@ -96,6 +96,23 @@ def test_int8_weight_only(cuda_device, scale_dtype):
     assert normwise_rel(y, lowrank.lr_linear(x.double().numpy(), A, B)) < NORMWISE_TOL
 
 
+@pytest.mark.parametrize("batch", [5, 8, 11])
+def test_batch_pieces_wide_output_and_int8(cuda_device, batch):
+    # a wide bf16 output (11008 columns: 4 lines per warp) takes 2 batch rows per
+    # launch, int8 (16 elements per lane) takes 4: the batch is split into pieces
+    At, B = synth._lr_factors(4096, 11008, 256, 3, (80,))
+    f = {"At": torch.from_numpy(At).to(torch.bfloat16), "B": torch.from_numpy(B).to(torch.bfloat16)}
+    x = synth.make_activations(batch, 4096, seed=3, key=(81, batch))
+    y = lr.lr_linear(_factor_dev(f), dev(x))
+    assert normwise_rel(y, _oracle(f, x.double().numpy())) < NORMWISE_TOL
+    p = synth.make_prefill_projection(4096, 4096, 512, seed=3, key=(82,))
+    xi = synth.make_activations(batch, 4096, seed=3, key=(83, batch))
+    yi = lr.lr_linear(lr.Factor(dev(p["A_q"]), dev(p["B_q"]), dev(p["s_A"]), dev(p["s_B"])), dev(xi))
+    A = (p["A_q"].double() * p["s_A"].double()[:, None]).numpy().T
+    Bq = (p["B_q"].double() * p["s_B"].double()[None, :]).numpy()
+    assert normwise_rel(yi, lowrank.lr_linear(xi.double().numpy(), A, Bq)) < NORMWISE_TOL
+
+
 def test_workspace_left_zeroed_and_reusable(cuda_device, layer0):
     f = _factor_dev(layer0["v"])
     x = dev(synth.make_activations(2, 4096, seed=3, key=(24,)))
