@@ -1,30 +1,42 @@
 #!/usr/bin/env python
 """Benchmark of the low-rank decode path on B200.
 
-Workload (one "step"): one decode token through a LLaMA-7B-shaped stack of
-32 layers whose Q/K/V/O projections are truncated-SVD factorised (bf16,
-hidden 4096, seeded non-uniform ranks in [512, 1536] at 40 % parameter
-reduction, batch 1).  Per layer: one grouped call computes Q, K, V from the
-layer input x; the O projection reads the V output (single-token attention
-returns V exactly) and its output is the next layer's input.  The
-whole stack is one lr_linear_chain call: one launch per step, with one
-grid-wide barrier per dependent projection inside it.
+Headline workload (one "step"): one decode token through a LLaMA-7B-shaped
+stack of 32 layers whose Q/K/V/O projections are truncated-SVD factorised
+(bf16, hidden 4096, seeded non-uniform ranks in [512, 1536] at 40 % parameter
+reduction, batch 1).  Per layer, Q, K and V are computed from the layer input
+x; the O projection reads the V output (single-token attention returns V
+exactly) and its output is the next layer's input.  The whole stack is one
+lr_linear_chain call: one persistent launch per step, in which each
+projection waits only for the projection it reads.
 
-The 32 layers hold 2.58 GB of factors, far above the 126 MB L2, so every
-step streams them from HBM (no L2 flush needed).  Timing: W untimed warm-up
-steps, then exactly K steps of a captured CUDA graph of the step,
-bracketed by a barrier and a device synchronisation, measured with CUDA
-events, max over ranks.  With --gpus N > 1 (torchrun), every rank runs its
-own replica of the workload on its own GPU (independent requests; weak
-scaling, no data-path collective).
+The 32 layers hold 2.58 GB of factors, far above the 126 MB L2, so every step
+streams them from HBM (no L2 flush needed).  Timing: W untimed warm-up steps,
+then exactly K steps of a captured CUDA graph of the step, bracketed by a
+barrier and a device synchronisation, measured with CUDA events, max over
+ranks.  With --gpus N > 1 (torchrun), every rank runs its own replica of the
+workload on its own GPU (independent requests; weak scaling, no data-path
+collective).
+
+At N = 1 the same JSON line carries `rows`: every configuration of the path,
+each with its own CUDA-event time, roofline, CPU-oracle baseline and an
+end-to-end time through the C ABI with host buffers:
+  c1        single fp32 low-rank linear, 256 x 256, rank 32, one token
+  c2b4/b16  the headline stack at batch 4 and 16
+  c3b1/8/32 hybrid int8 SwiGLU FFN (7B shapes), batch 1, 8, 32
+  c4k4/16/32 latent-KV flash decoding, batch 8, 32 heads, rank 32, ctx 4K/16K/32K
+  c5        W8A8 prefill of one 13B layer (7 projections), 2048 tokens
 
 `--impl reference` times the CPU oracle (the float64 reference
-implementation) on the same workload instead, on the host cores.
+implementation) on the headline workload instead, on the host cores.
 """
 from __future__ import annotations
 
 import argparse
+import ctypes
+import hashlib
 import json
+import math
 import os
 import statistics
 import subprocess
@@ -38,6 +50,8 @@ if ROOT not in sys.path:
 METRIC = "decode-layer µs & achieved HBM GB/s (% of B200 roofline) at batch 1; tokens/s"
 LAYERS, HIDDEN = 32, 4096
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+ROW_IDS = ("c1", "c2b4", "c2b16", "c3b1", "c3b8", "c3b32", "c4k4", "c4k16", "c4k32", "c5")
 
 
 def parse(argv=None):
@@ -48,8 +62,8 @@ def parse(argv=None):
     ap.add_argument("--batch", type=int, default=1)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--secondary", action="store_true",
-                    help="time the FFN, latent-KV and W8A8 rows instead (one JSON line each)")
+    ap.add_argument("--no-rows", action="store_true", help="headline only (no per-configuration rows)")
+    ap.add_argument("--only", default="", help="comma list of row ids to run (" + ",".join(ROW_IDS) + ")")
     ap.add_argument("--layers", type=int, default=LAYERS,
                     help="layers in the stack (default 32; fewer only for profiling small cases)")
     return ap.parse_args(argv)
@@ -108,67 +122,58 @@ def host_cores() -> int:
 
 
 # ---------------------------------------------------------------------------
-# workload
+# peaks, DRAM traffic records
 # ---------------------------------------------------------------------------
-# DRAM bytes (read + write) per algorithmic byte of chain_kernel<bf16, batch 1>,
-# from one ncu capture of the same kernel on the 2-layer case (163.92 MB of
-# DRAM traffic for 159.48 MB of algorithmic bytes; summary and command in
-# profiles/chain_kernel_bf16_b1_llama7b_2layers.md).  DRAM traffic grows with
-# the factor bytes streamed, so a full launch's traffic is this ratio times its
-# algorithmic bytes.  Valid for that kernel build and batch 1 only.
-CHAIN_TRAFFIC_PER_ALG_BYTE = 163.92e6 / 159481856
+def measured_peaks() -> dict:
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return json.load(f)
+    except (OSError, ValueError):
+        return {}
 
 
-def algorithmic_bytes_per_step(ranks, batch: int) -> int:
-    """Factor bytes (bf16) of all 128 projections plus activation reads/writes."""
-    factor = int(sum(int(r) * (HIDDEN + HIDDEN) * 2 for r in ranks[:LAYERS].reshape(-1)))
-    act = LAYERS * batch * HIDDEN * 2 * (2 + 4)  # reads: x (shared by Q/K/V), v; writes: q, k, v, o
-    return factor + act
+def hbm_peak():
+    p = measured_peaks()
+    if "hbm_gbs" in p:
+        return float(p["hbm_gbs"]), "of measured"
+    return FALLBACK_HBM_GBS, "of fallback"
 
 
-def build_layers(device, keep_cpu: int = 0):
-    from decode_lr_linear_b200 import synth
-    import decode_lr_linear_b200 as lr
-    ranks = synth.attention_ranks(0)
-    layers, cpu = [], []
-    for l in range(LAYERS):
-        L = synth.make_attention_layer(l, ranks, seed=0)
-        layers.append({n: lr.Factor(L[n]["At"].to(device), L[n]["B"].to(device)) for n in synth.ATTN_PROJ})
-        if l < keep_cpu:
-            cpu.append(L)
-    return ranks, layers, cpu
+def int8_peak_tops():
+    """int8 dense tensor peak: the measured bf16 burst figure times the nominal int8/bf16 ratio (2)."""
+    p = measured_peaks()
+    if "bf16_tflops" in p:
+        return 2.0 * float(p["bf16_tflops"]), "of measured bf16 burst x 2 (nominal int8/bf16 ratio)"
+    return 2.0 * FALLBACK_BF16_TFLOPS, "of fallback bf16 x 2 (nominal int8/bf16 ratio)"
 
 
-def oracle_step(cpu_layers, x):
-    """The CPU oracle on the same chain: Q, K, V from x; O from V; O's output feeds the next layer."""
-    from oracle import lowrank
-    for L in cpu_layers:
-        outs = {}
-        for n in ("q", "k", "v"):
-            outs[n] = lowrank.lr_linear(x, L[n]["At"].double().numpy().T, L[n]["B"].double().numpy())
-        x = lowrank.lr_linear(outs["v"], L["o"]["At"].double().numpy().T, L["o"]["B"].double().numpy())
-    return x
+# DRAM bytes (read + write) per algorithmic byte, from one ncu capture of the
+# kernel named, valid only while its sources hash to the recorded value (the
+# figure is dropped, as null, as soon as the kernel changes).  Filled from
+# the profiles of the current sources.
+TRAFFIC_RECORDS = {
+    # "chain_kernel<bf16,1,1>": {"sources_sha1": "...", "per_alg_byte": 1.0},
+}
+KERNEL_SOURCES = {"chain_kernel<bf16,1,1>": ("chain.cu", "common.cuh", "internal.h")}
 
 
-def cpu_baseline(cpu_layers, batch: int, budget_s: float = 12.0) -> dict:
-    """The oracle as it stands, timed on the host cores over a bounded sample of the workload."""
-    from decode_lr_linear_b200 import synth
-    x = synth.make_activations(batch, HIDDEN, seed=0, key=(90,)).double().numpy()
-    n_done, t_total = 0, 0.0
-    while t_total < budget_s and n_done < 64:
-        t0 = time.perf_counter()
-        oracle_step(cpu_layers, x)
-        t_total += time.perf_counter() - t0
-        n_done += 1
-    per_layer = t_total / (n_done * len(cpu_layers))
-    per_step = per_layer * LAYERS
-    return {"value": batch / per_step, "unit": "tokens/s", "cores": host_cores(), "kind": "oracle",
-            "sample": f"{n_done} pass(es) over layers 0..{len(cpu_layers) - 1} of the 32-layer stack at batch "
-                      f"{batch} (float64 numpy, {t_total:.1f} s), scaled to 32 layers"}
+def sources_sha1(files) -> str:
+    h = hashlib.sha1()
+    for name in files:
+        with open(os.path.join(ROOT, "decode_lr_linear_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def traffic_for(kernel: str, alg_bytes: float):
+    rec = TRAFFIC_RECORDS.get(kernel)
+    if not rec or rec["sources_sha1"] != sources_sha1(KERNEL_SOURCES[kernel]):
+        return None
+    return round(rec["per_alg_byte"] * alg_bytes)
 
 
 class ClockSampler:
-    """nvidia-smi clock/throttle sampling during the timed region."""
+    """nvidia-smi clock/throttle sampling while the GPU runs the timed work."""
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
          "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
          "clocks_event_reasons.sw_power_cap")
@@ -185,6 +190,17 @@ class ClockSampler:
         except (OSError, FileNotFoundError):
             self.proc = None
         return self
+
+    def wait_first_sample(self, limit_s: float = 5.0):
+        """Return once nvidia-smi has written a sample (its start-up takes a while)."""
+        if self.proc is None:
+            return
+        t0 = time.time()
+        while time.time() - t0 < limit_s:
+            self.out.flush()
+            if os.path.getsize(self.out.name) > 0:
+                return
+            time.sleep(0.02)
 
     def stop(self) -> dict:
         if self.proc is None:
@@ -216,183 +232,21 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(rows)}
 
 
-def measured_hbm_peak():
-    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
-    try:
-        with open(path) as f:
-            return float(json.load(f)["hbm_gbs"]), "of measured"
-    except (OSError, KeyError, ValueError):
-        return FALLBACK_HBM_GBS, "of fallback"
-
-
-def run_ours(args) -> None:
-    global LAYERS
-    LAYERS = args.layers
-    import torch
-
-    import decode_lr_linear_b200 as lr
-    from decode_lr_linear_b200 import synth
-
-    rank, local, world = dist_env()
-    device = torch.device("cuda", local)
-    torch.cuda.set_device(device)
-    dist_init("nccl")
-    batch = args.batch
-    want_cpu = rank == 0 and world == 1 and not args.no_cpu_baseline
-    ranks, layers, cpu_layers = build_layers(device, keep_cpu=LAYERS if want_cpu else 0)
-
-    x0 = synth.make_activations(batch, HIDDEN, seed=0, key=(90,)).to(device)
-    qkv = [[torch.empty(batch, HIDDEN, dtype=torch.bfloat16, device=device) for _ in range(3)] for _ in range(LAYERS)]
-    outs = [torch.empty(batch, HIDDEN, dtype=torch.bfloat16, device=device) for _ in range(LAYERS)]
-    # the whole stack as one chain: step 2l = Q/K/V of layer l (input: the previous O), step 2l+1 = O (input: V)
-    steps = []
-    for l in range(LAYERS):
-        L = layers[l]
-        steps.append(lr.ChainStep([L["q"], L["k"], L["v"]], -1 if l == 0 else 2 * l - 1, 0, qkv[l]))
-        steps.append(lr.ChainStep([L["o"]], 2 * l, 2, [outs[l]]))
-    ws = lr.workspace(lr.lr_linear_chain_workspace_size(steps, batch), device)
-
-    def step():
-        lr.lr_linear_chain(steps, x0, ws=ws)
-
-    launches_per_step = (batch + 7) // 8
-    step()
-    torch.cuda.synchronize()
-    g = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g):
-        step()
-    torch.cuda.synchronize()
-
-    clocks = ClockSampler(device.index).start()
-    for _ in range(args.warmup):
-        g.replay()
-    torch.cuda.synchronize()
-    barrier(device)
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(args.steps):
-        g.replay()
-    e1.record()
-    torch.cuda.synchronize()
-    barrier(device)
-    torch.cuda.synchronize()
-    clk = clocks.stop()
-    ms_total = reduce_max(e0.elapsed_time(e1), device)
-    ms_step = ms_total / args.steps
-
-    # end to end through the public API: pinned host input -> device, the step, result -> pinned host
-    x_host = synth.make_activations(batch, HIDDEN, seed=0, key=(90,)).pin_memory()
-    y_host = torch.empty(batch, HIDDEN, dtype=torch.bfloat16).pin_memory()
-    ge = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(ge):
-        step()
-    for _ in range(3):
-        x0.copy_(x_host, non_blocking=True)
-        ge.replay()
-        y_host.copy_(outs[-1], non_blocking=True)
-        torch.cuda.current_stream().synchronize()
-    barrier(device)
-    torch.cuda.synchronize()
-    k_e2e = max(3, min(args.steps, 200))
-    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    f0.record()
-    for _ in range(k_e2e):
-        x0.copy_(x_host, non_blocking=True)
-        ge.replay()
-        y_host.copy_(outs[-1], non_blocking=True)
-        torch.cuda.current_stream().synchronize()
-    f1.record()
-    torch.cuda.synchronize()
-    barrier(device)
-    ms_e2e = reduce_max(f0.elapsed_time(f1), device) / k_e2e
-
-    if rank != 0:
-        return
-    bytes_step = algorithmic_bytes_per_step(ranks, batch)
-    peak, peak_kind = measured_hbm_peak()
-    achieved = bytes_step / (ms_step * 1e-3) / 1e9
-    tokens_s = whole_job_throughput(world, batch, ms_step)
-    out = {
-        "metric": METRIC, "value": tokens_s, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": "llama7b-lowrank-qkvo-decode", "layers": LAYERS, "hidden": HIDDEN, "batch": batch,
-                   "ranks": f"seeded non-uniform in [512,1536], mean {float(ranks.mean()):.2f}, 40% reduction",
-                   "l2": "inputs larger than L2 (2.58 GB of factors streamed per step)",
-                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
-        "layer_us": ms_step * 1e3 / LAYERS,
-        "hbm_gbs": achieved,
-        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                     "traffic": (round(CHAIN_TRAFFIC_PER_ALG_BYTE * bytes_step) if batch == 1 else None),
-                     "traffic_note": "ncu dram__bytes_read.sum + dram__bytes_write.sum of a 2-layer launch, "
-                                     "scaled by factor bytes to the full launch",
-                     "peak_source": peak_kind,
-                     "kernel": "chain_kernel<bf16, batch 1> (factorised-linear chain)",
-                     "note": "the step is one launch of this kernel only, so its launch duration is the "
-                             "event-timed step time"},
-        "gpu_launches": launches_per_step * args.steps,
-        "e2e": {"value": whole_job_throughput(world, batch, ms_e2e), "unit": "tokens/s",
-                "h2d_bytes_per_step": int(x_host.numel() * x_host.element_size()),
-                "d2h_bytes_per_step": int(y_host.numel() * y_host.element_size())},
-        "clocks": clk,
-    }
-    if want_cpu:
-        out["cpu_baseline"] = cpu_baseline(cpu_layers, batch)
-    print(json.dumps(out), flush=True)
-
-
-def run_reference(args) -> None:
-    rank, _, world = dist_env()
-    if rank != 0:
-        return
-    from decode_lr_linear_b200 import synth
-    ranks = synth.attention_ranks(0)
-    # each step: the oracle over a bounded sample of the stack (layers cycled), scaled to 32 layers
-    per_step_layers = 1
-    cache = {}
-
-    def layer(l):
-        if l not in cache:
-            cache.clear()
-            cache[l] = synth.make_attention_layer(l, ranks, seed=0)
-        return cache[l]
-
-    x = synth.make_activations(args.batch, HIDDEN, seed=0, key=(90,)).double().numpy()
-    for i in range(args.warmup):
-        oracle_step([layer(i % LAYERS)], x)
-    t = 0.0
-    for i in range(args.steps):
-        L = layer((args.warmup + i) % LAYERS)
-        t0 = time.perf_counter()
-        oracle_step([L], x)
-        t += time.perf_counter() - t0
-    per_step = t / args.steps * LAYERS / per_step_layers
-    value = args.batch / per_step
-    out = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
-           "steps": args.steps, "warmup": args.warmup, "ms_per_step": per_step * 1e3, "higher_is_better": True,
-           "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-           "config": {"workload": "llama7b-lowrank-qkvo-decode", "layers": LAYERS, "hidden": HIDDEN,
-                      "batch": args.batch},
-           "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": host_cores(), "kind": "oracle",
-                            "sample": f"each step: the float64 oracle over one layer's Q/K/V/O (layers cycled), "
-                                      f"scaled to 32 layers"},
-           "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
-    print(json.dumps(out), flush=True)
-
-
-def _time_rotating(fn, n_copies: int, iters: int, warmup: int = 3) -> float:
-    """Mean ms per call of fn(i), copy i % n_copies: `iters` calls captured in
-    one CUDA graph (no host time between launches), replayed after warm-up,
-    timed with CUDA events on the replay stream."""
+# ---------------------------------------------------------------------------
+# timing helpers
+# ---------------------------------------------------------------------------
+def time_graph(fn, iters: int, warmup: int = 3) -> float:
+    """Mean ms per call of fn(i): `iters` calls captured in one CUDA graph (no
+    host time between launches), replayed once after warm-up, CUDA events on
+    the replay stream."""
     import torch
     for i in range(warmup):
-        fn(i % n_copies)
+        fn(i)
     torch.cuda.synchronize()
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g):
         for i in range(iters):
-            fn(i % n_copies)
+            fn(i)
     g.replay()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -404,107 +258,571 @@ def _time_rotating(fn, n_copies: int, iters: int, warmup: int = 3) -> float:
     return e0.elapsed_time(e1) / iters
 
 
-def run_secondary(args) -> None:
-    """One JSON line per further hot-path row, each against its own roofline:
-    the hybrid int8 SwiGLU FFN (7B shapes, batch 1), latent-KV split-K decode
-    (batch 8, 32 heads, rank 32, ctx 16384) and the W8A8 prefill projections
-    of one 13B layer (2048 tokens).  Weight or cache copies rotate so the
-    working set exceeds L2."""
+def time_e2e(step, iters: int, warmup: int = 3) -> float:
+    """Mean ms per step of step(): each step copies its inputs from pinned host
+    memory, calls the C ABI entry point, copies the result back to pinned host
+    memory and waits for it on the host.  CUDA events around all steps."""
+    import torch
+    s = torch.cuda.current_stream()
+    for _ in range(warmup):
+        step()
+        s.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(iters):
+        step()
+        s.synchronize()
+    e1.record()
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / iters
+
+
+def cpu_timed(fn, budget_s: float, max_calls: int = 1000):
+    """Calls fn() until budget_s of host time is spent (at least once); returns (s per call, calls)."""
+    n, t = 0, 0.0
+    while (t < budget_s or n == 0) and n < max_calls:
+        t0 = time.perf_counter()
+        fn()
+        t += time.perf_counter() - t0
+        n += 1
+    return t / n, n
+
+
+def check_device(lr) -> None:
+    err = lr.lr_check_device_error()
+    if err != 0:
+        raise SystemExit(f"a kernel gave up a bounded wait during the timed work (device error {err}); "
+                         "no number is reported")
+
+
+def stream_ptr() -> int:
+    import torch
+    return torch.cuda.current_stream().cuda_stream
+
+
+# ---------------------------------------------------------------------------
+# headline workload
+# ---------------------------------------------------------------------------
+def algorithmic_bytes_per_step(ranks, batch: int, layers: int) -> int:
+    """Factor bytes (bf16) of all the layers' projections plus activation reads/writes."""
+    factor = int(sum(int(r) * (HIDDEN + HIDDEN) * 2 for r in ranks[:layers].reshape(-1)))
+    act = layers * batch * HIDDEN * 2 * (2 + 4)  # reads: x (shared by Q/K/V), v; writes: q, k, v, o
+    return factor + act
+
+
+def build_layers(device, layers: int):
+    from decode_lr_linear_b200 import synth
+    import decode_lr_linear_b200 as lr
+    ranks = synth.attention_ranks(0)
+    out = []
+    for l in range(layers):
+        L = synth.make_attention_layer(l, ranks, seed=0)
+        out.append({n: lr.Factor(L[n]["At"].to(device), L[n]["B"].to(device)) for n in synth.ATTN_PROJ})
+    return ranks, out
+
+
+def stack_steps(lr, layers, batch, device):
+    """The decode stack as one chain: step 2l = Q/K/V of layer l (input: the previous O), step 2l+1 = O (input: V)."""
+    import torch
+    steps = []
+    for l, L in enumerate(layers):
+        qkv = [torch.empty(batch, HIDDEN, dtype=torch.bfloat16, device=device) for _ in range(3)]
+        steps.append(lr.ChainStep([L["q"], L["k"], L["v"]], -1 if l == 0 else 2 * l - 1, 0, qkv))
+        steps.append(lr.ChainStep([L["o"]], 2 * l, 2,
+                                  [torch.empty(batch, HIDDEN, dtype=torch.bfloat16, device=device)]))
+    return steps
+
+
+def oracle_layer(L, x):
+    """The CPU oracle on one layer of the chain: Q, K, V from x; O from V."""
+    from oracle import lowrank
+    outs = {n: lowrank.lr_linear(x, L[n]["At"].double().numpy().T, L[n]["B"].double().numpy())
+            for n in ("q", "k", "v")}
+    return lowrank.lr_linear(outs["v"], L["o"]["At"].double().numpy().T, L["o"]["B"].double().numpy())
+
+
+def cpu_baseline_stack(batch: int, budget_s: float, layers_in_sample: int = 2) -> dict:
+    """The oracle as it stands, timed on the host cores over a bounded sample
+    of the stack (whole passes over the first layers), scaled to 32 layers."""
+    from decode_lr_linear_b200 import synth
+    ranks = synth.attention_ranks(0)
+    cpu = [synth.make_attention_layer(l, ranks, seed=0) for l in range(layers_in_sample)]
+    x = synth.make_activations(batch, HIDDEN, seed=0, key=(90,)).double().numpy()
+
+    def one_pass():
+        y = x
+        for L in cpu:
+            y = oracle_layer(L, y)
+
+    per_pass, n = cpu_timed(one_pass, budget_s, 64)
+    per_step = per_pass / layers_in_sample * LAYERS
+    return {"value": batch / per_step, "unit": "tokens/s", "cores": host_cores(), "kind": "oracle",
+            "sample": f"{n} pass(es) over layers 0..{layers_in_sample - 1} of the 32-layer stack at batch {batch} "
+                      f"(float64 numpy, {per_pass * n:.1f} s), scaled to 32 layers"}
+
+
+def headline_config(world: int, batch: int, ranks) -> dict:
+    return {"workload": "llama7b-lowrank-qkvo-decode", "layers": LAYERS, "hidden": HIDDEN, "batch": batch,
+            "ranks": f"seeded non-uniform in [512,1536], mean {float(ranks.mean()):.2f}, 40% reduction",
+            "l2": "inputs larger than L2 (2.58 GB of factors streamed per step)",
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU"}
+
+
+def run_ours(args) -> None:
+    global LAYERS
+    LAYERS = args.layers
     import torch
 
     import decode_lr_linear_b200 as lr
+    from decode_lr_linear_b200 import _lib as L
     from decode_lr_linear_b200 import synth
-    dev = torch.device("cuda", 0)
-    torch.cuda.set_device(dev)
-    hbm, hbm_kind = measured_hbm_peak()
-    peaks = {}
-    peaks_path = os.path.join(ROOT, "MEASURED_PEAKS.json")
-    if os.path.exists(peaks_path):
-        with open(peaks_path) as f:
-            peaks = json.load(f)
-    lines = []
 
-    # ---- hybrid FFN (int8 weights + fp16 scales), 4 copies of one layer ----
-    d = synth.make_hybrid_ffn(seed=0)
+    rank, local, world = dist_env()
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    dist_init("nccl")
+    batch = args.batch
+    only = set(filter(None, args.only.split(",")))
+    want_headline = not only or "headline" in only
+    want_cpu = rank == 0 and world == 1 and not args.no_cpu_baseline
 
-    def ffn_copy():
-        g = lambda t: t.to(dev)
-        return lr.FfnWeights(d["hidden"], d["inter"], d["n_lr"], d["rank"], g(d["A_q"]), g(d["s_A"]), g(d["B_q"]),
-                             g(d["s_B"]), g(d["D_q"]), g(d["s_D"]), g(d["Wd_q"]), g(d["s_d"]))
-    ffns = [ffn_copy() for _ in range(4)]
+    ranks, layers = build_layers(device, LAYERS)
+    out = None
+    if want_headline:
+        x0 = synth.make_activations(batch, HIDDEN, seed=0, key=(90,)).to(device)
+        steps = stack_steps(lr, layers, batch, device)
+        ws = lr.workspace(lr.lr_linear_chain_workspace_size(steps, batch), device)
+
+        def step():
+            lr.lr_linear_chain(steps, x0, ws=ws)
+
+        launches_per_step = (batch + 7) // 8
+        step()
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            step()
+        torch.cuda.synchronize()
+
+        clocks = ClockSampler(device.index).start()
+        clocks.wait_first_sample()
+        for _ in range(args.warmup):
+            g.replay()
+        torch.cuda.synchronize()
+        barrier(device)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(args.steps):
+            g.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        barrier(device)
+        torch.cuda.synchronize()
+        ms_total = e0.elapsed_time(e1)
+        # a short timed region gets no clock sample of its own: keep the same
+        # load running (untimed) until the sampler has seen it for 0.3 s
+        t_extra = time.time()
+        while ms_total < 300.0 and time.time() - t_extra < 0.3:
+            for _ in range(50):
+                g.replay()
+            torch.cuda.synchronize()
+        clk = clocks.stop()
+        if ms_total < 300.0:
+            clk["window"] = "timed region plus untimed replays of the same step up to 0.3 s"
+        check_device(lr)
+        ms_step = reduce_max(ms_total, device) / args.steps
+
+        # end to end through the C ABI: each step copies x from pinned host
+        # memory, calls lr_linear_chain (descriptors prepared once, as a caller
+        # keeps them), and copies the last layer's output back to the host
+        x_host = synth.make_activations(batch, HIDDEN, seed=0, key=(90,)).pin_memory()
+        y_host = torch.empty(batch, HIDDEN, dtype=torch.bfloat16).pin_memory()
+        arr = lr.ops._chain_array(steps)
+        lib = L.load()
+        nbytes = ws.numel()
+        y_last = steps[-1].ys[0]
+
+        def e2e_step():
+            x0.copy_(x_host, non_blocking=True)
+            L.check("lr_linear_chain", lib.lr_linear_chain(arr, len(steps), x0.data_ptr(), batch, ws.data_ptr(),
+                                                           nbytes, stream_ptr()))
+            y_host.copy_(y_last, non_blocking=True)
+
+        barrier(device)
+        ms_e2e = reduce_max(time_e2e(e2e_step, max(3, min(args.steps, 200))), device)
+        check_device(lr)
+        del g
+
+        bytes_step = algorithmic_bytes_per_step(ranks, batch, LAYERS)
+        peak, peak_kind = hbm_peak()
+        achieved = bytes_step / (ms_step * 1e-3) / 1e9
+        out = {
+            "metric": METRIC, "value": whole_job_throughput(world, batch, ms_step), "unit": "tokens/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": headline_config(world, batch, ranks),
+            "layer_us": ms_step * 1e3 / LAYERS,
+            "hbm_gbs": achieved,
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                         "traffic": traffic_for("chain_kernel<bf16,1,1>", bytes_step) if batch == 1 else None,
+                         "peak_source": peak_kind,
+                         "kernel": "chain_kernel<bf16, batch 1> (the decode engine)",
+                         "algorithmic_bytes": bytes_step,
+                         "note": "the step is one launch of this kernel per 8 batch rows, so its launch duration "
+                                 "is the event-timed step time"},
+            "gpu_launches": launches_per_step * args.steps,
+            "e2e": {"value": whole_job_throughput(world, batch, ms_e2e), "unit": "tokens/s",
+                    "h2d_bytes_per_step": int(x_host.numel() * x_host.element_size()),
+                    "d2h_bytes_per_step": int(y_host.numel() * y_host.element_size()),
+                    "path": "lr_linear_chain through the C ABI every step, pinned host x in, last output out"},
+            "clocks": clk,
+        }
+        if want_cpu:
+            out["cpu_baseline"] = cpu_baseline_stack(batch, 12.0)
+        del steps, ws
+
+    if rank == 0 and world == 1 and not args.no_rows:
+        rows = run_rows(args, lr, L, synth, device, ranks, layers, only)
+        if out is None:
+            for r in rows:
+                print(json.dumps(r), flush=True)
+            return
+        out["rows"] = rows
+    if rank == 0 and out is not None:
+        print(json.dumps(out), flush=True)
+
+
+# ---------------------------------------------------------------------------
+# rows: every configuration of the path at N = 1
+# ---------------------------------------------------------------------------
+def _roof_hbm(alg_bytes: float, ms: float, note: str = "") -> dict:
+    peak, kind = hbm_peak()
+    gbs = alg_bytes / (ms * 1e-3) / 1e9
+    r = {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s", "frac": gbs / peak, "peak_source": kind,
+         "algorithmic_bytes": int(alg_bytes), "traffic": None}
+    if note:
+        r["note"] = note
+    return r
+
+
+def row_c1(lr, L, synth, device, want_cpu):
+    import torch
+    from oracle import lowrank
+    d = synth.make_single_linear(0)
+    f = lr.Factor(d["At"].to(device), d["B32"].to(device))
+    x = d["x"].to(device)
+    y = torch.empty(1, 256, dtype=torch.float32, device=device)
+    ws = lr.workspace(lr.lr_linear_workspace_size(f, 1), device)
+    ms = time_graph(lambda i: lr.lr_linear(f, x, y, ws), 200)
+    alg = (32 * 256 * 2 + 256 + 256) * 4
+    lib, desc = L.load(), f.desc()
+    xh, yh = d["x"].pin_memory(), torch.empty(1, 256, dtype=torch.float32).pin_memory()
+
+    def e2e():
+        x.copy_(xh, non_blocking=True)
+        L.check("lr_linear", lib.lr_linear(ctypes.byref(desc), x.data_ptr(), None, 1, y.data_ptr(), ws.data_ptr(),
+                                           ws.numel(), stream_ptr()))
+        yh.copy_(y, non_blocking=True)
+    ms_e2e = time_e2e(e2e, 200)
+    row = {"row": "c1", "workload": "single low-rank linear, fp32, d_in = d_out = 256, rank 32, 1 token "
+                                    "(Haar U, V; sigma_i = i^-1/2)",
+           "value": ms * 1e3, "unit": "µs per call", "higher_is_better": False, "launches": 1,
+           "roofline": dict(_roof_hbm(alg, ms, "66 KB that stay in L2: launch-latency bound, no roofline target"),
+                            bound="latency"),
+           "e2e": {"value": ms_e2e * 1e3, "unit": "µs per call", "h2d_bytes_per_step": 1024,
+                   "d2h_bytes_per_step": 1024, "path": "lr_linear through the C ABI"},
+           "l2": "all inputs fit L2 (the configuration is the latency case)"}
+    if want_cpu:
+        xd = d["x"].double().numpy()
+        At, B = d["At"].double().numpy().T, d["B32"].double().numpy()
+        s, n = cpu_timed(lambda: lowrank.lr_linear(xd, At, B), 1.0)
+        row["cpu_baseline"] = {"value": s * 1e6, "unit": "µs per call", "cores": host_cores(), "kind": "oracle",
+                               "sample": f"{n} calls of the float64 oracle on the same inputs"}
+    return row
+
+
+def row_c2(lr, L, synth, device, ranks, layers, batch, want_cpu):
+    import torch
+    steps = stack_steps(lr, layers, batch, device)
+    ws = lr.workspace(lr.lr_linear_chain_workspace_size(steps, batch), device)
+    x0 = synth.make_activations(batch, HIDDEN, seed=0, key=(90, batch)).to(device)
+    ms = time_graph(lambda i: lr.lr_linear_chain(steps, x0, ws=ws), 20)
+    alg = algorithmic_bytes_per_step(ranks, batch, LAYERS)
+    launches = (batch + 7) // 8
+    arr, lib = lr.ops._chain_array(steps), L.load()
+    xh = synth.make_activations(batch, HIDDEN, seed=0, key=(90, batch)).pin_memory()
+    yh = torch.empty(batch, HIDDEN, dtype=torch.bfloat16).pin_memory()
+
+    def e2e():
+        x0.copy_(xh, non_blocking=True)
+        L.check("lr_linear_chain", lib.lr_linear_chain(arr, len(steps), x0.data_ptr(), batch, ws.data_ptr(),
+                                                       ws.numel(), stream_ptr()))
+        yh.copy_(steps[-1].ys[0], non_blocking=True)
+    ms_e2e = time_e2e(e2e, 20)
+    row = {"row": f"c2b{batch}", "workload": f"llama7b-lowrank-qkvo-decode, 32 layers, batch {batch}",
+           "value": batch / (ms * 1e-3), "unit": "tokens/s", "higher_is_better": True,
+           "ms_per_step": ms, "layer_us": ms * 1e3 / LAYERS, "launches": launches,
+           "roofline": _roof_hbm(alg, ms, f"{launches} launch(es) of chain_kernel per step; each streams every "
+                                          f"factor byte once"),
+           "e2e": {"value": batch / (ms_e2e * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": batch * HIDDEN * 2,
+                   "d2h_bytes_per_step": batch * HIDDEN * 2, "path": "lr_linear_chain through the C ABI"},
+           "l2": "2.58 GB of factors streamed per step"}
+    if want_cpu:
+        row["cpu_baseline"] = cpu_baseline_stack(batch, 3.0, 1)
+    return row
+
+
+def row_c3(lr, L, synth, device, d, batch, want_cpu):
+    import torch
+    from oracle import ffn as offn
+    copies = 4
+
+    def g(t):
+        return t.to(device)
+    ffns = [lr.FfnWeights(d["hidden"], d["inter"], d["n_lr"], d["rank"], g(d["A_q"]), g(d["s_A"]), g(d["B_q"]),
+                          g(d["s_B"]), g(d["D_q"]), g(d["s_D"]), g(d["Wd_q"]), g(d["s_d"])) for _ in range(copies)]
     w_bytes = sum(int(d[k].numel() * d[k].element_size()) for k in ("A_q", "s_A", "B_q", "s_B", "D_q", "s_D",
                                                                   "Wd_q", "s_d"))
-    for batch in (1, 8):
-        x = synth.make_activations(batch, d["hidden"], seed=0, key=(30, batch), outliers=4).to(dev)
-        y = torch.empty_like(x)
-        ws = lr.workspace(lr.lr_swiglu_ffn_workspace_size(ffns[0], batch), dev)
-        ms = _time_rotating(lambda i: lr.lr_swiglu_ffn(ffns[i], x, y, ws), 4, 40)
-        alg = w_bytes + 2 * batch * d["hidden"] * 2
-        gbs = alg / (ms * 1e-3) / 1e9
-        lines.append({"row": "a4-a7 hybrid int8 SwiGLU FFN", "workload": f"7B FFN (hidden 4096, inter 11008, "
-                      f"n_lr 8192, rank 1536), batch {batch}", "us_per_layer": ms * 1e3,
-                      "tokens_s_32_layers": batch / (ms * 1e-3 * 32),
-                      "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
-                                   "peak_source": hbm_kind, "algorithmic_bytes": alg}})
-    del ffns
+    xc = synth.make_activations(batch, d["hidden"], seed=0, key=(30, batch), outliers=4)
+    x = xc.to(device)
+    y = torch.empty_like(x)
+    ws = lr.workspace(lr.lr_swiglu_ffn_workspace_size(ffns[0], batch), device)
+    ms = time_graph(lambda i: lr.lr_swiglu_ffn(ffns[i % copies], x, y, ws), 40)
+    alg = w_bytes + 2 * batch * d["hidden"] * 2
+    lib, desc = L.load(), ffns[0].desc()
+    xh, yh = xc.pin_memory(), torch.empty(batch, d["hidden"], dtype=torch.bfloat16).pin_memory()
 
-    # ---- latent-KV split-K decode (absorbed), ctx 16384 ----
-    kvd = synth.make_latent_kv(batch=8, heads=32, ctx=16384, seed=0)
-    kv = lr.LatentKv(kvd["batch"], kvd["heads"], kvd["ctx"], kvd["B_K"].to(dev), kvd["B_V"].to(dev), kvd["scale"],
-                     0, 0)
-    q, CK, CV, sl = (kvd[k].to(dev) for k in ("q", "C_K", "C_V", "seq_lens"))
-    out = torch.empty(kv.batch, kv.heads, kv.head_dim, dtype=torch.bfloat16, device=dev)
-    kws = lr.workspace(lr.lr_latent_kv_workspace_size(kv), dev)
-    ms = _time_rotating(lambda i: lr.lr_latent_kv_decode(kv, q, CK, CV, sl, out, kws), 1, 40)
-    alg = int(CK.numel() * 2 + CV.numel() * 2 + kvd["B_K"].numel() * 2 + kvd["B_V"].numel() * 2)
-    gbs = alg / (ms * 1e-3) / 1e9
-    lines.append({"row": "a8-a10 latent-KV split-K decode", "workload": "batch 8, heads 32, rank 32, head_dim 128, "
-                  "ctx 16384 (1.07 GB of latent cache, larger than L2)", "us": ms * 1e3,
-                  "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
-                               "peak_source": hbm_kind, "algorithmic_bytes": alg}})
-    del q, CK, CV, sl, kv, kvd, out, kws
+    def e2e():
+        x.copy_(xh, non_blocking=True)
+        L.check("lr_swiglu_ffn", lib.lr_swiglu_ffn(ctypes.byref(desc), x.data_ptr(), batch, y.data_ptr(),
+                                                   ws.data_ptr(), ws.numel(), stream_ptr()))
+        yh.copy_(y, non_blocking=True)
+    ms_e2e = time_e2e(e2e, 40)
+    pieces = math.ceil(batch / 2)
+    row = {"row": f"c3b{batch}", "workload": f"hybrid int8 SwiGLU FFN, 7B shapes (hidden 4096, inter 11008, "
+                                             f"n_lr 8192, rank 1536), batch {batch}",
+           "value": ms * 1e3, "unit": "µs per layer", "higher_is_better": False,
+           "tokens_s_32_layers": batch / (ms * 1e-3 * 32), "launches": pieces,
+           "roofline": _roof_hbm(alg, ms, f"{pieces} launch(es) of the decode engine (2 batch rows each), each "
+                                          f"streaming every weight byte"),
+           "e2e": {"value": ms_e2e * 1e3, "unit": "µs per layer", "h2d_bytes_per_step": batch * d["hidden"] * 2,
+                   "d2h_bytes_per_step": batch * d["hidden"] * 2, "path": "lr_swiglu_ffn through the C ABI"},
+           "l2": f"{copies} weight copies rotate ({copies * w_bytes / 1e6:.0f} MB > L2)"}
+    if want_cpu:
+        x64 = xc.double().numpy()
+        s, n = cpu_timed(lambda: offn.hybrid_swiglu_ffn(x64, d["A_q"], d["s_A"], d["B_q"], d["s_B"], d["D_q"],
+                                                        d["s_D"], d["Wd_q"], d["s_d"], d["n_lr"], d["n_dense"]),
+                         3.0, 20)
+        row["cpu_baseline"] = {"value": s * 1e6, "unit": "µs per layer", "cores": host_cores(), "kind": "oracle",
+                               "sample": f"{n} call(s) of the float64 oracle on the same layer and batch"}
+    del ffns, ws
+    return row
 
-    # ---- W8A8 prefill: the 7 projections of one 13B layer, 2048 tokens ----
+
+def row_c4(lr, L, synth, device, ctx, want_cpu):
+    import torch
+    from oracle import latent_kv as okv
+    kvd = synth.make_latent_kv(batch=8, heads=32, ctx=ctx, seed=0)
+    cache_bytes = int(kvd["C_K"].numel() * 2 * 2)
+    copies = max(1, math.ceil(4 * 126e6 / cache_bytes)) if cache_bytes < 4 * 126e6 else 1
+    kv = lr.LatentKv(8, 32, ctx, kvd["B_K"].to(device), kvd["B_V"].to(device), kvd["scale"])
+    caches = [(kvd["C_K"].to(device), kvd["C_V"].to(device)) for _ in range(copies)]
+    q, sl = kvd["q"].to(device), kvd["seq_lens"].to(device)
+    o = torch.empty(8, 32, 128, dtype=torch.bfloat16, device=device)
+    ws = lr.workspace(lr.lr_latent_kv_workspace_size(kv), device)
+    ms = time_graph(lambda i: lr.lr_latent_kv_decode(kv, q, caches[i % copies][0], caches[i % copies][1], sl, o, ws),
+                    40)
+    alg = cache_bytes + int(kvd["B_K"].numel() * 2 * 2) + 2 * q.numel() * 2
+    lib, desc = L.load(), kv.desc()
+    qh, oh = kvd["q"].pin_memory(), torch.empty(8, 32, 128, dtype=torch.bfloat16).pin_memory()
+    CK, CV = caches[0]
+
+    def e2e():
+        q.copy_(qh, non_blocking=True)
+        L.check("lr_latent_kv_decode", lib.lr_latent_kv_decode(ctypes.byref(desc), q.data_ptr(), CK.data_ptr(),
+                                                               CV.data_ptr(), sl.data_ptr(), o.data_ptr(),
+                                                               ws.data_ptr(), ws.numel(), stream_ptr()))
+        oh.copy_(o, non_blocking=True)
+    ms_e2e = time_e2e(e2e, 40)
+    row = {"row": f"c4k{ctx // 1024}", "workload": f"per-head latent-KV flash decoding, batch 8, 32 heads, "
+                                                  f"head_dim 128, rank 32, ctx {ctx} (absorbed form)",
+           "value": ms * 1e3, "unit": "µs per call", "higher_is_better": False,
+           "tokens_s_32_layers": 8 / (ms * 1e-3 * 32), "launches": 2,
+           "roofline": _roof_hbm(alg, ms, "split kernel (dominant) + combine kernel"),
+           "e2e": {"value": ms_e2e * 1e3, "unit": "µs per call", "h2d_bytes_per_step": int(q.numel() * 2),
+                   "d2h_bytes_per_step": int(o.numel() * 2),
+                   "path": "lr_latent_kv_decode through the C ABI (the caches stay resident, as a KV cache does)"},
+           "l2": f"{copies} cache cop{'y' if copies == 1 else 'ies'} ({copies * cache_bytes / 1e6:.0f} MB > L2)"}
+    if want_cpu:
+        pairs = [(b, h) for b in range(0, 8, 2) for h in (0, 17)]
+        s, n = cpu_timed(lambda: okv.latent_kv_decode(kvd["q"], kvd["C_K"], kvd["C_V"], kvd["B_K"], kvd["B_V"],
+                                                      kvd["seq_lens"], kvd["scale"], pairs), 2.0, 10)
+        row["cpu_baseline"] = {"value": s * 1e6 * 256 / len(pairs), "unit": "µs per call", "cores": host_cores(),
+                               "kind": "oracle",
+                               "sample": f"{n} call(s) of the float64 oracle on {len(pairs)} of the 256 (batch, head) "
+                                         f"pairs, scaled to 256"}
+    del caches, ws
+    return row
+
+
+def row_c5(lr, L, synth, device, want_cpu):
+    import torch
+    from oracle import w8a8 as ow8
     T = 2048
     shapes = synth.prefill_shapes()
     ranks = synth.prefill_ranks(0)
-    projs, ops = [], 0
+    projs, ops, xs = {}, 0, {}
+    # distinct inputs of a layer: x (q, k, v), attention output (o), x_ffn (gate, up), h (down)
+    src = {"q": 0, "k": 0, "v": 0, "o": 1, "gate": 2, "up": 2, "down": 3}
     for j, name in enumerate(synth.PREFILL_PROJ):
         d_in, d_out = shapes[name]
         r = int(ranks[0, j])
         pp = synth.make_prefill_projection(d_in, d_out, r, seed=0, key=(d_in, d_out, r))
-        f = lr.Factor(pp["A_q"].to(dev), pp["B_q"].to(dev), pp["s_A"].to(dev), pp["s_B"].to(dev))
-        xin = synth.make_activations(T, d_in, seed=0, key=(60, d_in, T), outliers=max(1, d_in // 1000)).to(dev)
-        xq, sx = lr.lr_quantize_per_token(xin)
-        ws = lr.workspace(lr.lr_linear_workspace_size(f, T, w8a8=True), dev)
-        y = torch.empty(T, d_out, dtype=torch.bfloat16, device=dev)
-        projs.append((f, xq, sx, y, ws))
+        f = lr.Factor(pp["A_q"].to(device), pp["B_q"].to(device), pp["s_A"].to(device), pp["s_B"].to(device))
+        if src[name] not in xs:
+            xc = synth.make_activations(T, d_in, seed=0, key=(60, d_in, T, src[name]), outliers=max(1, d_in // 1000))
+            xd = xc.to(device)
+            xs[src[name]] = [xc, xd, *lr.lr_quantize_per_token(xd)]
+        ws = lr.workspace(lr.lr_linear_workspace_size(f, T, w8a8=True), device)
+        y = torch.empty(T, d_out, dtype=torch.bfloat16, device=device)
+        projs[name] = (f, src[name], y, ws, pp)
         ops += 2 * T * r * (d_in + d_out)
 
+    def gemms(_):
+        for name, (f, s, y, ws, _) in projs.items():
+            lr.lr_linear(f, xs[s][2], y, ws, x_scale=xs[s][3])
+
     def layer(_):
-        for f, xq, sx, y, ws in projs:
-            lr.lr_linear(f, xq, y, ws, x_scale=sx)
-    ms = _time_rotating(layer, 1, 20)
-    tops = ops / (ms * 1e-3) / 1e12
-    bf16 = peaks.get("bf16_tflops")
-    i8_peak = 2.0 * bf16 if bf16 else 2.0 * 1590.0
-    lines.append({"row": "a11-a12 W8A8 prefill (tcgen05 int8)", "workload": "one 13B layer (q,k,v,o,gate,up,down; "
-                  "ranks of layer 0), 2048 tokens, int8 x int8 -> int32", "us_per_layer": ms * 1e3,
-                  "tokens_s_40_layers": T / (ms * 1e-3 * 40),
-                  "roofline": {"bound": "tensor", "achieved": tops, "peak": i8_peak, "unit": "TOPS",
-                               "frac": tops / i8_peak, "peak_source": ("of measured bf16 x 2 (nominal int8/bf16 "
-                                                                       "ratio)" if bf16 else "of fallback x 2"),
-                               "algorithmic_ops": ops}})
-    for ln in lines:
-        print(json.dumps(ln), flush=True)
+        for key, (xc, xd, xq, sx) in xs.items():
+            lr.lr_quantize_per_token(xd, xq, sx)
+        gemms(0)
+    ms_gemm = time_graph(gemms, 10)
+    ms = time_graph(layer, 10)
+    tops = ops / (ms_gemm * 1e-3) / 1e12
+    peak, kind = int8_peak_tops()
+    host_x = {k: v[0].pin_memory() for k, v in xs.items()}
+    host_y = {n: torch.empty_like(p[2], device="cpu").pin_memory() for n, p in projs.items()}
+
+    def e2e():
+        for k, (xc, xd, xq, sx) in xs.items():
+            xd.copy_(host_x[k], non_blocking=True)
+            lr.lr_quantize_per_token(xd, xq, sx)
+        gemms(0)
+        for n, p in projs.items():
+            host_y[n].copy_(p[2], non_blocking=True)
+    ms_e2e = time_e2e(e2e, 5, 1)
+    h2d = sum(int(v.numel() * 2) for v in host_x.values())
+    d2h = sum(int(v.numel() * 2) for v in host_y.values())
+    row = {"row": "c5", "workload": "W8A8 prefill, one 13B layer (q, k, v, o, gate, up, down; ranks of layer 0), "
+                                    "2048 tokens, int8 x int8 -> int32 on tcgen05",
+           "value": ms * 1e3, "unit": "µs per layer", "higher_is_better": False,
+           "tokens_s_40_layers": T / (ms * 1e-3 * 40), "launches": 4 + 7 * 3,
+           "gemm_us_per_layer": ms_gemm * 1e3,
+           "roofline": {"bound": "tensor", "achieved": tops, "peak": peak, "unit": "TOPS", "frac": tops / peak,
+                        "peak_source": kind, "algorithmic_ops": ops, "traffic": None,
+                        "note": "w8a8_gemm_kernel x2 + requant_kernel per projection (the 7 projections' GEMM time); "
+                                "value adds the 4 per-token quantisations of the layer's inputs"},
+           "e2e": {"value": ms_e2e * 1e3, "unit": "µs per layer", "h2d_bytes_per_step": h2d,
+                   "d2h_bytes_per_step": d2h,
+                   "path": "lr_quantize_per_token + lr_linear through the C ABI, bf16 inputs in, 7 outputs out"},
+           "l2": f"{ops / 1e9:.0f} GOP per layer; operands re-read from L2 by the tile loop"}
+    if want_cpu:
+        f, s, y, ws, pp = projs["q"]
+        xc = xs[s][0]
+
+        def one():
+            qx, sx = ow8.quantize_per_token(xc)
+            ow8.w8a8_lr_linear(qx, sx, pp["A_q"], pp["s_A"], pp["B_q"], pp["s_B"])
+        sec, n = cpu_timed(one, 3.0, 5)
+        d_in, d_out = shapes["q"]
+        q_ops = 2 * T * int(ranks[0, 0]) * (d_in + d_out)
+        row["cpu_baseline"] = {"value": sec * 1e6 * ops / q_ops, "unit": "µs per layer", "cores": host_cores(),
+                               "kind": "oracle",
+                               "sample": f"{n} call(s) of the oracle's W8A8 pipeline (quantise + both integer "
+                                         f"products + requant, float64 BLAS) on the q projection, scaled to the "
+                                         f"layer by integer ops"}
+    del projs, xs
+    return row
+
+
+def run_rows(args, lr, L, synth, device, ranks, layers, only) -> list:
+    import torch
+    want_cpu = not args.no_cpu_baseline
+    sel = [r for r in ROW_IDS if not only or r in only]
+    rows = []
+    clocks = ClockSampler(device.index).start()
+    clocks.wait_first_sample()
+    for rid in sel:
+        if rid.startswith("c2"):
+            rows.append(row_c2(lr, L, synth, device, ranks, layers, int(rid[3:]), want_cpu))
+    del layers
+    torch.cuda.empty_cache()
+    if "c1" in sel:
+        rows.insert(0, row_c1(lr, L, synth, device, want_cpu))
+    ffn = None
+    for rid in sel:
+        if rid.startswith("c3"):
+            ffn = ffn or synth.make_hybrid_ffn(seed=0)
+            rows.append(row_c3(lr, L, synth, device, ffn, int(rid[3:]), want_cpu))
+            torch.cuda.empty_cache()
+    for rid in sel:
+        if rid.startswith("c4"):
+            rows.append(row_c4(lr, L, synth, device, int(rid[3:]) * 1024, want_cpu))
+            torch.cuda.empty_cache()
+    if "c5" in sel:
+        rows.append(row_c5(lr, L, synth, device, want_cpu))
+    clk = clocks.stop()
+    check_device(lr)
+    for r in rows:
+        r["clocks"] = clk
+    return rows
+
+
+# ---------------------------------------------------------------------------
+# reference arm: the CPU oracle
+# ---------------------------------------------------------------------------
+def run_reference(args) -> None:
+    rank, _, world = dist_env()
+    if rank != 0:
+        return
+    from decode_lr_linear_b200 import synth
+    ranks = synth.attention_ranks(0)
+    # each step: the oracle over a bounded sample of the stack (one layer, layers cycled), scaled to 32 layers
+    cache = {}
+
+    def layer(l):
+        if l not in cache:
+            cache.clear()
+            cache[l] = synth.make_attention_layer(l, ranks, seed=0)
+        return cache[l]
+
+    x = synth.make_activations(args.batch, HIDDEN, seed=0, key=(90,)).double().numpy()
+    for i in range(args.warmup):
+        oracle_layer(layer(i % LAYERS), x)
+    t = 0.0
+    for i in range(args.steps):
+        L = layer((args.warmup + i) % LAYERS)
+        t0 = time.perf_counter()
+        oracle_layer(L, x)
+        t += time.perf_counter() - t0
+    per_step = t / args.steps * LAYERS
+    value = args.batch / per_step
+    out = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": per_step * 1e3, "higher_is_better": True,
+           "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+           "config": headline_config(world, args.batch, ranks),
+           "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": host_cores(), "kind": "oracle",
+                            "sample": "each step: the float64 oracle over one layer's Q/K/V/O (layers cycled), "
+                                      "scaled to 32 layers, so ms_per_step is 32 times the time each step ran"},
+           "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
 
 
 def main(argv=None):
     args = parse(argv)
     if args.impl == "reference":
         run_reference(args)
-    elif args.secondary:
-        run_secondary(args)
     else:
         run_ours(args)
     try:

@@ -8,7 +8,7 @@ from .ops import (  # noqa: F401
     Factor, FfnWeights, LatentKv, ChainStep, workspace, lr_linear_chain, lr_linear_chain_workspace_size,
     lr_linear, lr_linear_workspace_size, lr_linear_grouped, lr_linear_grouped_workspace_size,
     lr_swiglu_ffn, lr_swiglu_ffn_workspace_size, lr_latent_kv_decode, lr_latent_kv_workspace_size,
-    lr_quantize_per_token, lr_gemm_s8s32, lr_workspace_init, lr_check_device_error,
+    lr_quantize_per_token, lr_gemm_s8s32, lr_workspace_init, lr_check_device_error, lr_set_wait_timeout_us,
 )
 from ._lib import LrError, load  # noqa: F401
 

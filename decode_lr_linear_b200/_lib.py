@@ -22,6 +22,7 @@ LR_MAX_GROUP = 4
 LR_MAX_CHAIN = 64
 LR_KV_ABSORBED, LR_KV_RECONSTRUCT = 0, 1
 LR_NOALLOC_SCRATCH_BYTES = 1 << 20
+DEVICE_ERR_MBAR, DEVICE_ERR_TMEM, DEVICE_ERR_GRID_WAIT = 1, 2, 3
 
 c_int, c_void_p, c_size_t, c_float = ctypes.c_int, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_float
 
@@ -68,6 +69,7 @@ _SIGNATURES = {
     "lr_gemm_s8s32": (c_int, [c_void_p, c_void_p, c_int, c_int, c_int, c_int, c_void_p, c_void_p]),
     "lr_workspace_init": (c_int, [c_void_p, c_size_t, c_void_p]),
     "lr_check_device_error": (c_int, [c_void_p, P(c_int)]),
+    "lr_set_wait_timeout_us": (c_int, [ctypes.c_uint]),
     "lr_status_string": (ctypes.c_char_p, [c_int]),
     "lr_version": (c_int, []),
 }

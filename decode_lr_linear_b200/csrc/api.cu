@@ -1,9 +1,11 @@
 // C ABI of the low-rank decode library: argument validation, workspace sizing
 // and dispatch to the sm_100a kernels.  Nothing here computes on the host.
 #include <algorithm>
+#include <atomic>
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <vector>
 
 #include "common.cuh"
 #include "internal.h"
@@ -13,16 +15,36 @@ namespace lr {
 // The library's device error word: set by kernels whose bounded waits give up.
 __device__ int g_device_error = 0;
 
+// Looked up on every call (cheap): the address belongs to the module loaded in
+// the current context, which a device reset replaces.
 int* device_error_word() {
-  static int* cache[64] = {nullptr};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-  if (!cache[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) return nullptr;
-    cache[dev] = reinterpret_cast<int*>(p);
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) return nullptr;
+  return reinterpret_cast<int*>(p);
+}
+
+namespace {
+std::atomic<unsigned long long> g_grid_wait_ns{kGridWaitDefaultNs};
+}  // namespace
+
+unsigned long long grid_wait_ns() { return g_grid_wait_ns.load(std::memory_order_relaxed); }
+
+cudaError_t check_resident(const void* fn, int threads, size_t smem, int grid, int sm_count) {
+  static std::mutex mu;
+  static std::vector<std::pair<std::pair<const void*, size_t>, int>> cache;
+  int per_sm = -1;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    for (auto& e : cache)
+      if (e.first.first == fn && e.first.second == smem) per_sm = e.second;
   }
-  return cache[dev];
+  if (per_sm < 0) {
+    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, threads, smem);
+    if (e != cudaSuccess) return e;
+    std::lock_guard<std::mutex> lock(mu);
+    cache.push_back({{fn, smem}, per_sm});
+  }
+  return per_sm * sm_count >= grid ? cudaSuccess : cudaErrorCooperativeLaunchTooLarge;
 }
 
 }  // namespace lr
@@ -48,7 +70,12 @@ int sm_count_current() {
 inline bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 inline size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
-inline lr_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? LR_OK : LR_ERR_CUDA; }
+inline lr_status_t from_cuda(cudaError_t e) {
+  if (e == cudaSuccess) return LR_OK;
+  // a persistent grid that cannot be resident at once: a configuration limit
+  if (e == cudaErrorCooperativeLaunchTooLarge) return LR_ERR_UNSUPPORTED;
+  return LR_ERR_CUDA;
+}
 
 
 // Shape/pointer checks common to every factor descriptor.
@@ -158,6 +185,7 @@ lr_status_t run_chain(const HostStep* steps, int n_steps, const void* x, int bat
   P.acc = reinterpret_cast<float*>(reinterpret_cast<char*>(ws) + kTicketBytes);
   P.acc_set = int(chain_acc_set(steps, n_steps, batch));
   P.err = device_error_word();
+  P.wait_ns = grid_wait_ns();
   int x_width = 0;
   for (int s = 0; s < n_steps; ++s) {
     ChainStep& c = P.step[s];
@@ -186,7 +214,8 @@ lr_status_t run_chain(const HostStep* steps, int n_steps, const void* x, int bat
     for (int s = 0; s < n_steps; ++s)
       for (int p = 0; p < P.step[s].n; ++p)
         P.step[s].p[p].y = reinterpret_cast<char*>(steps[s].y[p]) + size_t(b0) * steps[s].d[p].d_out * es;
-    if (launch_chain(P, wt, sms, stream) != cudaSuccess) return LR_ERR_CUDA;
+    st = from_cuda(launch_chain(P, wt, sms, stream));
+    if (st != LR_OK) return st;
   }
   return LR_OK;
 }
@@ -202,33 +231,48 @@ lr_status_t run_rank1(const lr_factor_desc_t* descs, int n, const void* x, int b
 // library, so that callers who cannot allocate device memory still have the
 // split-reduction accumulators and arrival counter that lr_linear needs.  Host
 // code never uses the symbol itself as a pointer: its device address is looked
-// up once per device and cached.
+// up on every call with the device current.  The array is zero-filled on the
+// first call in a CUDA context (the looked-up address is new) and again after
+// lr_check_device_error has reported a kernel that gave up a wait (such a
+// kernel may leave partial sums behind); the kernels leave it zeroed otherwise.
 // ---------------------------------------------------------------------------
 __device__ __align__(256) unsigned char g_noalloc_scratch[LR_NOALLOC_SCRATCH_BYTES];
 
 std::mutex g_noalloc_mu;
-void* g_noalloc_ptr[kMaxDevices] = {nullptr};
+void* g_noalloc_ptr[kMaxDevices] = {nullptr};  // address zero-filled last, per device
 
-// Device address of the scratch on the current device; the first call on a
-// device looks it up and zero-fills it on `s` (the kernels leave it zeroed).
+// Device address of the scratch on the current device, zero-filled on `s`
+// first when it is new or was marked dirty.
 lr_status_t noalloc_scratch(cudaStream_t s, void** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return LR_ERR_CUDA;
   if (dev < 0 || dev >= kMaxDevices) return LR_ERR_UNSUPPORTED;
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return LR_ERR_CUDA;
   std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  if (!g_noalloc_ptr[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return LR_ERR_CUDA;
+  if (g_noalloc_ptr[dev] != p) {
     if (cudaMemsetAsync(p, 0, LR_NOALLOC_SCRATCH_BYTES, s) != cudaSuccess) return LR_ERR_CUDA;
     g_noalloc_ptr[dev] = p;
   }
-  *out = g_noalloc_ptr[dev];
+  *out = p;
   return LR_OK;
+}
+
+void noalloc_mark_dirty() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  g_noalloc_ptr[dev] = nullptr;
 }
 
 }  // namespace
 
 extern "C" {
+
+lr_status_t lr_set_wait_timeout_us(unsigned int us) {
+  g_grid_wait_ns.store(us ? (unsigned long long)us * 1000ull : kGridWaitDefaultNs, std::memory_order_relaxed);
+  return LR_OK;
+}
 
 lr_status_t lr_linear_noalloc(const lr_factor_desc_t* desc, const void* x, int batch, void* y,
                               lr_stream_t stream) {
@@ -236,6 +280,8 @@ lr_status_t lr_linear_noalloc(const lr_factor_desc_t* desc, const void* x, int b
   if (st != LR_OK) return st;
   if (!x || !y || batch < 1) return LR_ERR_INVALID_ARG;
   if (!al16(x) || !al16(y)) return LR_ERR_MISALIGNED;
+  st = check_rank1_limits(desc);
+  if (st != LR_OK) return st;
   if (rank1_ws_bytes(desc, 1, batch) > size_t(LR_NOALLOC_SCRATCH_BYTES)) return LR_ERR_WORKSPACE;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   void* ws = nullptr;
@@ -394,13 +440,16 @@ lr_status_t lr_swiglu_ffn(const lr_ffn_desc_t* d, const void* x, int batch, void
   P.h_dense = reinterpret_cast<float*>(w);
   w += round_up(size_t(chunk) * P.n_dense * 4, 256);
   P.y_acc = reinterpret_cast<float*>(w);
+  P.wait_ns = grid_wait_ns();
+  P.err = device_error_word();
   const int sms = sm_count_current();
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   for (int b0 = 0; b0 < batch; b0 += kMaxDecodeChunk) {
     P.nb = std::min(kMaxDecodeChunk, batch - b0);
     P.x = reinterpret_cast<const char*>(x) + size_t(b0) * d->hidden * 2;
     P.y = reinterpret_cast<char*>(y) + size_t(b0) * d->hidden * 2;
-    if (launch_ffn(P, sms, s) != cudaSuccess) return LR_ERR_CUDA;
+    st = from_cuda(launch_ffn(P, sms, s));
+    if (st != LR_OK) return st;
   }
   return LR_OK;
 }
@@ -486,6 +535,7 @@ lr_status_t lr_check_device_error(lr_stream_t stream, int* err) {
   if (cudaMemcpyFromSymbol(&v, lr::g_device_error, sizeof(int)) != cudaSuccess) return LR_ERR_CUDA;
   *err = v;
   if (v != 0) {
+    noalloc_mark_dirty();
     const int zero = 0;
     if (cudaMemcpyToSymbol(lr::g_device_error, &zero, sizeof(int)) != cudaSuccess) return LR_ERR_CUDA;
     return LR_ERR_DEVICE_TIMEOUT;

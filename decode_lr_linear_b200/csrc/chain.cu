@@ -21,7 +21,8 @@
 //            output line in registers, adding it into the fp32 accumulator
 //            set s % 3 (red.global.add.v4.f32) when a projection's rows end;
 //   barrier  thread 0 arrives with one release reduction and waits on a
-//            monotonic counter (bounded wait).
+//            monotonic counter (bounded in time; every CTA is resident, which
+//            the launch checks).
 // The outputs of step s-1 are written during step s (their accumulator loads
 // share the round trip of the step's input loads), and each CTA then zeroes
 // its slice of set (s-2) % 3, which nothing reads any more; the last step's
@@ -375,9 +376,19 @@ LR_DEV void flush_lines(float (&acc)[L][NB][Lane16<WT>::kElems], float* dst, int
   }
 }
 
+// Wait for a ring stage.  After a first mbarrier timeout the CTA stops
+// computing but keeps to the protocol, with a short bound per stage, so that
+// no copy it issued is left in flight into its shared memory.
 LR_DEV const unsigned char* stage_acquire(unsigned char* ring, uint64_t* full, int st, bool* failed, int* err) {
   const int slot = st % kStages;
-  if (!*failed && !mbar_wait_bounded(&full[slot], uint32_t(st / kStages) & 1u, err)) *failed = true;
+  const uint32_t parity = uint32_t(st / kStages) & 1u;
+  if (!*failed) {
+    if (!mbar_wait_bounded(&full[slot], parity, err)) *failed = true;
+  } else {
+    const uint64_t t0 = global_ns();
+    while (!mbar_try_wait(&full[slot], parity) && global_ns() - t0 < kDegradedMbarNs) {
+    }
+  }
   return ring + size_t(slot) * kStageBytes;
 }
 
@@ -531,14 +542,7 @@ __global__ void __launch_bounds__(kThreads, 1) chain_kernel(const __grid_constan
     for (int i = threadIdx.x; i < rows_cap * NB; i += kConsumers) zs[i] = 0.f;
     if (threadIdx.x == 0) {
       red_release_add(P.bar, 1u);
-      const unsigned target = gridDim.x * unsigned(s + 1);
-      uint32_t i = 0;
-      while (ld_acquire_u32(P.bar) < target) {
-        if (++i > (1u << 22)) {
-          set_device_error(P.err, kErrGridBarrier);
-          break;
-        }
-      }
+      wait_counter_geq(P.bar, gridDim.x * unsigned(s + 1), P.wait_ns, P.err);
     }
     consumer_sync();
   }
@@ -569,11 +573,13 @@ size_t chain_smem(int rows_cap) {
 }
 
 template <typename WT, int NB, int L>
-cudaError_t launch_chain_t(const ChainParams& p, int grid, int rows_cap, cudaStream_t s) {
+cudaError_t launch_chain_t(const ChainParams& p, int grid, int rows_cap, int sm_count, cudaStream_t s) {
   const size_t bytes = chain_smem<NB>(rows_cap);
   if (bytes > kSmemLimit - 1024) return cudaErrorInvalidValue;
   auto kern = chain_kernel<WT, NB, L>;
   cudaError_t e = ensure_smem(kern, bytes);
+  if (e != cudaSuccess) return e;
+  e = check_resident(reinterpret_cast<const void*>(kern), kThreads, bytes, grid, sm_count);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
@@ -598,12 +604,12 @@ constexpr int nb_max_for(int L) {
 }
 
 template <typename WT, int L>
-cudaError_t launch_chain_nb(const ChainParams& p, int grid, int rows_cap, cudaStream_t s) {
+cudaError_t launch_chain_nb(const ChainParams& p, int grid, int rows_cap, int sm_count, cudaStream_t s) {
   constexpr int kMaxNb = nb_max_for<WT>(L);
-  if (p.nb <= 1) return launch_chain_t<WT, 1, L>(p, grid, rows_cap, s);
-  if (p.nb <= 2 && kMaxNb >= 2) return launch_chain_t<WT, (kMaxNb >= 2 ? 2 : 1), L>(p, grid, rows_cap, s);
-  if (p.nb <= 4 && kMaxNb >= 4) return launch_chain_t<WT, (kMaxNb >= 4 ? 4 : 1), L>(p, grid, rows_cap, s);
-  if (p.nb <= 8 && kMaxNb >= 8) return launch_chain_t<WT, (kMaxNb >= 8 ? 8 : 1), L>(p, grid, rows_cap, s);
+  if (p.nb <= 1) return launch_chain_t<WT, 1, L>(p, grid, rows_cap, sm_count, s);
+  if (p.nb <= 2 && kMaxNb >= 2) return launch_chain_t<WT, (kMaxNb >= 2 ? 2 : 1), L>(p, grid, rows_cap, sm_count, s);
+  if (p.nb <= 4 && kMaxNb >= 4) return launch_chain_t<WT, (kMaxNb >= 4 ? 4 : 1), L>(p, grid, rows_cap, sm_count, s);
+  if (p.nb <= 8 && kMaxNb >= 8) return launch_chain_t<WT, (kMaxNb >= 8 ? 8 : 1), L>(p, grid, rows_cap, sm_count, s);
   return cudaErrorInvalidValue;
 }
 
@@ -633,9 +639,9 @@ cudaError_t launch_chain_w(const ChainParams& p0, int sm_count, cudaStream_t s) 
     for (int i = 0; i < P.n_steps; ++i)
       for (int q = 0; q < P.step[i].n; ++q)
         P.step[i].p[q].y = reinterpret_cast<XT*>(p0.step[i].p[q].y) + size_t(b0) * p0.step[i].p[q].d_out;
-    cudaError_t e = L == 1   ? launch_chain_nb<WT, 1>(P, grid, rows_cap, s)
-                    : L == 2 ? launch_chain_nb<WT, 2>(P, grid, rows_cap, s)
-                             : launch_chain_nb<WT, 4>(P, grid, rows_cap, s);
+    cudaError_t e = L == 1   ? launch_chain_nb<WT, 1>(P, grid, rows_cap, sm_count, s)
+                    : L == 2 ? launch_chain_nb<WT, 2>(P, grid, rows_cap, sm_count, s)
+                             : launch_chain_nb<WT, 4>(P, grid, rows_cap, sm_count, s);
     if (e != cudaSuccess) return e;
   }
   return cudaSuccess;

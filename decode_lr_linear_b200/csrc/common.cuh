@@ -28,6 +28,21 @@ LR_DEV void set_device_error(int* err, int code) {
   if (err) atomicCAS(err, 0, code);
 }
 
+// Bounds of the waits, in nanoseconds of the GPU's global timer.  A wait for
+// this CTA's own asynchronous copies (an mbarrier) only ends early if the
+// memory system has failed; a wait for other CTAs (grid barriers, arrival
+// counters) ends early when a CTA of the grid was not resident or a limit
+// shorter than the barrier latency was set on purpose.
+constexpr uint64_t kMbarTimeoutNs = 2000000000ull;      // 2 s
+constexpr uint64_t kGridWaitDefaultNs = 1000000000ull;  // 1 s (lr_set_wait_timeout_us)
+constexpr uint64_t kDegradedMbarNs = 1000000ull;        // per stage, after a first mbarrier timeout (1 ms)
+
+LR_DEV uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
 // ---------------------------------------------------------------------------
 // Programmatic dependent launch (PDL).
 // wait: block until the preceding grid in the stream has completed and its
@@ -200,12 +215,30 @@ LR_DEV bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
       : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity) : "memory");
   return ok != 0;
 }
-// Bounded wait: gives up after ~2^26 polls (each try_wait itself suspends for a
-// while), records the failure in the device error word and returns false.
+// Bounded wait: gives up after kMbarTimeoutNs (checked every 64 polls; each
+// try_wait itself suspends for a while), records the failure in the device
+// error word and returns false.
 LR_DEV bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, int* err) {
-  for (uint32_t i = 0; i < (1u << 26); ++i)
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_ns();
+  for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
+    if ((i & 63u) == 0 && global_ns() - t0 > kMbarTimeoutNs) break;
+  }
   set_device_error(err, kErrMbarTimeout);
+  return false;
+}
+
+// Bounded wait until *word >= target (acquire, gpu scope): gives up after
+// limit_ns, records kErrGridBarrier and returns false.
+LR_DEV bool wait_counter_geq(const unsigned int* word, unsigned int target, uint64_t limit_ns, int* err) {
+  if (ld_acquire_u32(word) >= target) return true;
+  const uint64_t t0 = global_ns();
+  for (;;) {
+    if (ld_acquire_u32(word) >= target) return true;
+    if (global_ns() - t0 > limit_ns) break;  // one timer read per poll: cheap next to the acquire load
+  }
+  set_device_error(err, kErrGridBarrier);
   return false;
 }
 

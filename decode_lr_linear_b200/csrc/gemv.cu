@@ -248,13 +248,14 @@ LR_DEV void produce(const Plan& pl, unsigned char* ring, uint64_t* full, uint64_
 }
 
 // Barrier over the CTAs of one launch.  The grid never exceeds the CTAs that
-// can be resident at once (one per SM at most), so every CTA gets to arrive.
-// words[0] counts arrivals, words[1] is a generation number: the last CTA to
-// arrive resets the count and bumps the generation; the others wait (bounded:
-// after ~2^22 polls the wait gives up and sets the device error word) until
-// the generation changes.  All threads of the CTA call it; on return every
-// CTA's earlier global writes and reductions are visible.
-LR_DEV void grid_barrier(unsigned int* words, int* err) {
+// can be resident at once (one per SM at most, checked before the launch),
+// so every CTA gets to arrive.  words[0] counts arrivals, words[1] is a
+// generation number: the last CTA to arrive resets the count and bumps the
+// generation; the others wait until the generation changes (bounded: after
+// wait_ns the wait gives up and sets the device error word).  All threads of
+// the CTA call it; on return every CTA's earlier global writes and
+// reductions are visible.
+LR_DEV void grid_barrier(unsigned int* words, unsigned long long wait_ns, int* err) {
   __syncthreads();
   if (threadIdx.x == 0) {
     const unsigned gen = ld_acquire_u32(words + 1);
@@ -265,9 +266,9 @@ LR_DEV void grid_barrier(unsigned int* words, int* err) {
       __threadfence();
       atomicAdd(words + 1, 1u);
     } else {
-      uint32_t i = 0;
+      const uint64_t t0 = global_ns();
       while (ld_acquire_u32(words + 1) == gen) {
-        if (++i > (1u << 22)) {
+        if (global_ns() - t0 > wait_ns) {
           set_device_error(err, kErrGridBarrier);
           break;
         }
@@ -503,7 +504,15 @@ __global__ void __launch_bounds__(kThreads, (NB <= 1 && LPW <= 2 ? 2 : 1)) strea
       for (int r = 0; r < g.rows; r += g.rps) {
         const int k = min(g.rps, g.rows - r);
         const int slot = st % K.stages, round = st / K.stages;
-        if (!failed && !mbar_wait_bounded(&full[slot], uint32_t(round) & 1u, K.err)) failed = true;
+        // after a first timeout: stop computing, keep to the protocol with a
+        // short bound so that no issued copy is left in flight
+        if (!failed) {
+          if (!mbar_wait_bounded(&full[slot], uint32_t(round) & 1u, K.err)) failed = true;
+        } else {
+          const uint64_t t0 = global_ns();
+          while (!mbar_try_wait(&full[slot], uint32_t(round) & 1u) && global_ns() - t0 < kDegradedMbarNs) {
+          }
+        }
         if (!failed) {
           const unsigned char* stage = ring + size_t(slot) * kStageBytes;
           if (g.kind == kDot)
@@ -549,7 +558,7 @@ __global__ void __launch_bounds__(kThreads, (NB <= 1 && LPW <= 2 ? 2 : 1)) strea
     return;
   } else {
     unsigned int* words = K.f.ticket;
-    grid_barrier(words, K.err);
+    grid_barrier(words, K.f.wait_ns, K.err);
     {
       FinalTarget t[1] = {FinalTarget{K.f.y_acc, K.f.y, K.f.sd, K.f.nb * K.f.hidden, K.f.hidden}};
       finalize_slice<__nv_bfloat16, 1>(t, 1, K.f.scale_f16 != 0);
@@ -561,7 +570,7 @@ __global__ void __launch_bounds__(kThreads, (NB <= 1 && LPW <= 2 ? 2 : 1)) strea
 // Launch helpers
 // ---------------------------------------------------------------------------
 template <typename WT, typename XT, typename YT, int NB, int LPW, int MODE>
-cudaError_t launch_stream(KParams K, int grid, cudaStream_t s) {
+cudaError_t launch_stream(KParams K, int grid, int sm_count, cudaStream_t s) {
   // Three stages when that lets two CTAs share an SM (the next kernel's
   // producer then streams during this kernel's tail); otherwise the most
   // stages that fit.
@@ -577,6 +586,10 @@ cudaError_t launch_stream(KParams K, int grid, cudaStream_t s) {
   auto kern = stream_kernel<WT, XT, YT, NB, LPW, MODE>;
   cudaError_t e = ensure_smem(kern, bytes);
   if (e != cudaSuccess) return e;
+  if (MODE == kFfn2) {  // the finalize barrier needs every CTA resident
+    e = check_resident(reinterpret_cast<const void*>(kern), kThreads, bytes, grid, sm_count);
+    if (e != cudaSuccess) return e;
+  }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(kThreads);
@@ -599,9 +612,9 @@ int lpw_for(int d_out) {
 // Pick the (NB, LPW) instantiation: NB is the smallest power of two >= nb
 // with NB * LPW <= 8 (accumulator registers).
 template <typename WT, typename XT, typename YT, int MODE>
-cudaError_t dispatch(const KParams& K, int nb, int lpw, int grid, cudaStream_t s) {
+cudaError_t dispatch(const KParams& K, int nb, int lpw, int grid, int sm_count, cudaStream_t s) {
 #define LR_CASE(NB_, LPW_) \
-  if (lpw == LPW_ && nb <= NB_) return launch_stream<WT, XT, YT, NB_, LPW_, MODE>(K, grid, s);
+  if (lpw == LPW_ && nb <= NB_) return launch_stream<WT, XT, YT, NB_, LPW_, MODE>(K, grid, sm_count, s);
   LR_CASE(1, 1) LR_CASE(2, 1) LR_CASE(4, 1) LR_CASE(8, 1)
   LR_CASE(1, 2) LR_CASE(2, 2) LR_CASE(4, 2)
   LR_CASE(1, 4) LR_CASE(2, 4)
@@ -636,6 +649,7 @@ cudaError_t launch_ffn_impl(const FfnParams& p0, int sm_count, cudaStream_t s) {
   KParams K1, K2;
   std::memset(&K1, 0, sizeof(K1));
   std::memset(&K2, 0, sizeof(K2));
+  K1.err = K2.err = p0.err;
   K1.g_lr = g_lr;
   K1.rows_cap = std::max(g_lr ? (p0.rank + g_lr - 1) / g_lr : 0, g_d ? 2 * ((p0.n_dense + g_d - 1) / g_d) : 0);
   K1.x_elems = p0.hidden;
@@ -654,7 +668,7 @@ cudaError_t launch_ffn_impl(const FfnParams& p0, int sm_count, cudaStream_t s) {
     f.gu_acc = p0.gu_acc + size_t(b0) * 2 * p0.n_lr;
     f.h_dense = p0.h_dense + size_t(b0) * p0.n_dense;
     K1.f = f;
-    cudaError_t e = dispatch<int8_t, __nv_bfloat16, __nv_bfloat16, kFfn1>(K1, f.nb, lpw1, g_lr + g_d, s);
+    cudaError_t e = dispatch<int8_t, __nv_bfloat16, __nv_bfloat16, kFfn1>(K1, f.nb, lpw1, g_lr + g_d, sm_count, s);
     if (e != cudaSuccess) return e;
   }
   for (int b0 = 0; b0 < p0.nb; b0 += nb2) {
@@ -665,7 +679,7 @@ cudaError_t launch_ffn_impl(const FfnParams& p0, int sm_count, cudaStream_t s) {
     f.h_dense = p0.h_dense + size_t(b0) * p0.n_dense;
     f.y_acc = p0.y_acc + size_t(b0) * p0.hidden;
     K2.f = f;
-    cudaError_t e = dispatch<int8_t, __nv_bfloat16, __nv_bfloat16, kFfn2>(K2, f.nb, lpw2, g2, s);
+    cudaError_t e = dispatch<int8_t, __nv_bfloat16, __nv_bfloat16, kFfn2>(K2, f.nb, lpw2, g2, sm_count, s);
     if (e != cudaSuccess) return e;
   }
   return cudaSuccess;

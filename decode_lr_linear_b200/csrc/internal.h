@@ -12,6 +12,15 @@ namespace lr {
 // Device address of the library's error word on the current device.
 int* device_error_word();
 
+// Bound of waits on the other CTAs of a persistent grid (lr_set_wait_timeout_us), in nanoseconds.
+unsigned long long grid_wait_ns();
+
+// The CTAs of a persistent grid wait for one another, so all of them must be
+// resident at once: cudaSuccess when `grid` CTAs of `threads` threads and
+// `smem` bytes of dynamic shared memory fit the device together, else
+// cudaErrorCooperativeLaunchTooLarge (cached per kernel and size).
+cudaError_t check_resident(const void* fn, int threads, size_t smem, int grid, int sm_count);
+
 constexpr int kMaxGroup = LR_MAX_GROUP;
 
 // Workspace element shared by the split-reduction kernels: one arrival counter
@@ -53,6 +62,7 @@ struct ChainParams {
   unsigned int* bar;  // 2 barrier counters (zero on entry and exit)
   int scale_f16;
   int* err;
+  unsigned long long wait_ns;  // bound of the grid-barrier waits
 };
 
 static_assert(sizeof(ChainParams) < 32000, "chain parameters must fit the kernel parameter space");
@@ -73,6 +83,8 @@ struct FfnParams {
   float* h_dense;     // [nb, n_dense]
   float* y_acc;       // [nb, hidden]  (zero on entry and exit)
   unsigned int* ticket;
+  unsigned long long wait_ns;  // bound of the grid-barrier wait
+  int* err;                    // device error word
 };
 
 cudaError_t launch_ffn(const FfnParams& p, int sm_count, cudaStream_t s);

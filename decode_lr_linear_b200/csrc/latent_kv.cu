@@ -95,6 +95,9 @@ __global__ void __launch_bounds__(kThreads) latent_kv_split_kernel(const __grid_
   }
   __syncthreads();
   if (!mbar_wait_bounded(&bar, 0, P.err)) {
+    // the copies did not land in time (the error word says so); they must not
+    // land in a later CTA's shared memory, so wait once more before leaving
+    mbar_wait_bounded(&bar, 0, P.err);
     if (threadIdx.x < kPart) outp[threadIdx.x] = threadIdx.x == 0 ? -INFINITY : 0.f;
     return;
   }

@@ -220,7 +220,10 @@ __global__ void __launch_bounds__(kThreads, 1) w8a8_gemm_kernel(const __grid_con
       if (ok) mma_commit(&accum);
     }
   } else {
-    // epilogue: warp w reads TMEM lanes 32 * (w % 4) .. + 31 (one accumulator row per thread)
+    // epilogue: warp w reads TMEM lanes 32 * (w % 4) .. + 31 (one accumulator row per thread).
+    // Its per-token scales, and the row maxima it raises, were written by the
+    // preceding kernels: every thread that touches them waits for those first.
+    pdl_wait();
     const int q = warp & 3;
     const int row = m0 + q * 32 + lane;
     const bool have = mbar_wait_bounded(&accum, 0u, P.err);

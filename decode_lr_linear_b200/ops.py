@@ -287,3 +287,8 @@ def lr_check_device_error(stream=None) -> int:
     if st not in (L.LR_OK, L.LR_ERR_DEVICE_TIMEOUT):
         raise L.LrError("lr_check_device_error", st)
     return err.value
+
+
+def lr_set_wait_timeout_us(us: int) -> None:
+    """Bound of a persistent kernel's waits on its other CTAs, in microseconds (0: default, 1 s)."""
+    L.check("lr_set_wait_timeout_us", L.load().lr_set_wait_timeout_us(int(us)))

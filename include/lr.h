@@ -160,17 +160,20 @@ LR_API lr_status_t lr_linear_grouped_workspace_size(const lr_factor_desc_t* desc
  * Step s computes y[s][p] = (x_s A[s][p]) B[s][p] for p < n, with
  *   x_s = x                      when input_step < 0,
  *   x_s = y[input_step][input_proj] otherwise (input_step < s).
- * An input taken from the step right before is read at fp32 (before the
- * output rounding to bf16); an older one is read from its stored output.
- * Every step's outputs are written.  All descriptors of a step share d_in,
- * which must equal d_out of the projection its input comes from; all steps
- * share w_dtype (weight-only paths) and scale_dtype; batch 1..8; at most
- * LR_MAX_CHAIN steps.  One persistent CTA per SM streams the factors of all
- * steps back to back through shared memory, so the loads of step s+1 proceed
- * while step s is finishing; the CTAs meet at one (bounded) grid-wide barrier
- * per step.  LASER "System Implementation" fuses the stages of a layer to cut
- * memory movement and kernel-launch overhead; this is that fusion across
- * consecutive factorised projections.
+ * An input taken from the step right before is read at fp32 (its accumulator
+ * times the int8 output scale, before the output rounding to bf16); an older
+ * one is read from its stored output.  Every step's outputs are written.  All
+ * descriptors of a step share d_in, which must equal d_out of the projection
+ * its input comes from; all steps share w_dtype (weight-only paths) and
+ * scale_dtype; any batch >= 1 (one launch per 8 rows or fewer, depending on
+ * the widest row); at most LR_MAX_CHAIN steps.
+ * One persistent CTA per SM (all resident: checked before the launch,
+ * LR_ERR_UNSUPPORTED otherwise) streams the factors of all steps back to back
+ * through shared memory, so the loads of step s+1 proceed while step s is
+ * finishing; the CTAs meet at one grid-wide barrier per step, bounded in time
+ * (lr_set_wait_timeout_us).  LASER "System Implementation" fuses the stages
+ * of a layer to cut memory movement and kernel-launch overhead; this is that
+ * fusion across consecutive factorised projections.
  */
 #define LR_MAX_CHAIN 64
 typedef struct lr_chain_step {
@@ -202,10 +205,13 @@ LR_API lr_status_t lr_linear_chain_workspace_size(const lr_chain_step_t* steps, 
  *
  *   - The scratch a call needs is what lr_linear_workspace_size reports,
  *     256 + 3 * 64-rounded(min(batch, 8) * d_out) * 4 bytes; a call that needs
- *     more returns LR_ERR_WORKSPACE and launches nothing.
- *   - The first call on a device looks the array up and zero-fills it on
- *     `stream`; make that first call before any stream capture.  Every call
- *     leaves the array zeroed again.
+ *     more returns LR_ERR_WORKSPACE and launches nothing.  Shapes lr_linear
+ *     refuses are refused the same way (LR_ERR_UNSUPPORTED) before that.
+ *   - The first call on a device (in a CUDA context) looks the array up and
+ *     zero-fills it on `stream`; make that first call before any stream
+ *     capture.  Every call leaves the array zeroed again, except a call whose
+ *     kernel gave up a bounded wait: once lr_check_device_error has reported
+ *     that, the next call zero-fills the array again before it launches.
  *   - All calls on one device share the array: calls that may overlap on the
  *     GPU (different streams without ordering between them) race and give
  *     wrong results.  Serialise them, or use lr_linear with your own workspace.
@@ -278,9 +284,11 @@ LR_API lr_status_t lr_swiglu_ffn_workspace_size(const lr_ffn_desc_t* desc, int b
  *             K_t = C_K[b,h,t,:] B_K[h], value V_t = C_V[b,h,t,:] B_V[h]
  *   scale     softmax scale (1/sqrt(head_dim) for standard attention)
  *   mode      LR_KV_ABSORBED: scores s_t = C_K[t] (B_K q) * scale, latent
- *             values accumulated and reconstructed once per split;
- *             LR_KV_RECONSTRUCT: each tile K_tile = C_K_tile B_K is built on
- *             chip (tensor cores) and scored against q
+ *             values accumulated and reconstructed once per split (the only
+ *             mode implemented);
+ *             LR_KV_RECONSTRUCT: reserved for on-chip reconstruction of the
+ *             key tiles (needed once a position-dependent rotation is applied
+ *             to keys); returns LR_ERR_UNSUPPORTED
  *   split_tokens  tokens per split-K chunk (multiple of 64), 0 = library choice
  * Supported: rank 32, head_dim 128.
  */
@@ -350,10 +358,30 @@ LR_API lr_status_t lr_workspace_init(void* ws, size_t ws_bytes, lr_stream_t stre
 /*
  * Synchronise `stream`, then read and clear the library's device error word on
  * the current device.  *err = 0 when no kernel gave up a bounded wait since the
- * last check; otherwise a nonzero code naming the wait.  Returns
- * LR_ERR_DEVICE_TIMEOUT when *err != 0, LR_ERR_CUDA if synchronisation failed.
+ * last check; otherwise the first code recorded:
+ *   1  a wait for the kernel's own asynchronous copies (an mbarrier) gave up
+ *      after 2 s: the memory system did not deliver; treat the CUDA context as
+ *      unusable;
+ *   2  a tensor-memory allocation could not be obtained;
+ *   3  a wait for the other CTAs of a persistent grid gave up (see
+ *      lr_set_wait_timeout_us): the outputs of that call are wrong and its
+ *      workspace may hold partial sums; zero it with lr_workspace_init before
+ *      reusing it (the lr_linear_noalloc scratch is re-zeroed by the library).
+ * Returns LR_ERR_DEVICE_TIMEOUT when *err != 0, LR_ERR_CUDA if synchronisation
+ * failed.
  */
 LR_API lr_status_t lr_check_device_error(lr_stream_t stream, int* err);
+
+/*
+ * Bound of every wait of a persistent kernel on its other CTAs (the grid-wide
+ * barriers of lr_linear_chain and lr_swiglu_ffn), in microseconds, for
+ * launches issued after this call; 0 restores the default of one second.  The CTAs of one launch
+ * are all resident (checked before every launch), so these waits end within
+ * microseconds unless other work occupies the device; a wait that gives up
+ * records code 3 in the device error word and the kernel carries on without
+ * hanging.  Process-wide.
+ */
+LR_API lr_status_t lr_set_wait_timeout_us(unsigned int us);
 
 /* Static string for a status code. */
 LR_API const char* lr_status_string(lr_status_t status);

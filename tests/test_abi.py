@@ -42,11 +42,13 @@ def _ws(lib, d, batch, w8a8=0):
 
 
 def test_linear_workspace_sizes(lib):
-    # barrier words + three accumulator sets of min(batch, 8) x d_out floats
+    # barrier words + three accumulator sets of min(batch, 8) x d_out floats (64-rounded)
     st, n = _ws(lib, _desc(), 1)
     assert st == L.LR_OK and n == 256 + 3 * 4096 * 4
     st, n8 = _ws(lib, _desc(), 16)
     assert st == L.LR_OK and n8 == 256 + 3 * 8 * 4096 * 4
+    st, n3 = _ws(lib, _desc(d_out=8), 3)
+    assert st == L.LR_OK and n3 == 256 + 3 * 64 * 4
     st, _ = _ws(lib, _desc(w_dtype=L.LR_I8), 1)
     assert st == L.LR_ERR_INVALID_ARG  # int8 needs scales
     st, n = _ws(lib, _desc(w_dtype=L.LR_I8, scale_A=FAKE, scale_B=FAKE), 2048, 1)
@@ -161,3 +163,19 @@ def test_chain_validation_and_workspace(lib):
     assert lib.lr_linear_chain(bad, 2, FAKE, 1, FAKE, 1 << 24, None) == L.LR_ERR_INVALID_ARG
     assert lib.lr_linear_chain(arr, 3, FAKE, 1, FAKE, 64, None) == L.LR_ERR_WORKSPACE
     assert lib.lr_linear_chain(arr, 0, FAKE, 1, FAKE, 1 << 24, None) == L.LR_ERR_INVALID_ARG
+
+
+def test_noalloc_validation_order(lib):
+    # a row wider than 32 KiB is refused as unsupported, as lr_linear refuses it
+    d = _desc(d_out=20000)
+    assert lib.lr_linear_noalloc(ctypes.byref(d), FAKE, 1, FAKE, None) == L.LR_ERR_UNSUPPORTED
+    # a valid shape whose scratch exceeds the fixed array: int8, d_out 32768, batch 8
+    d = _desc(w_dtype=L.LR_I8, scale_A=FAKE, scale_B=FAKE, d_in=64, d_out=32768, rank=32)
+    assert lib.lr_linear_noalloc(ctypes.byref(d), FAKE, 8, FAKE, None) == L.LR_ERR_WORKSPACE
+    st, n = _ws(lib, d, 8)
+    assert st == L.LR_OK and n > L.LR_NOALLOC_SCRATCH_BYTES
+
+
+def test_wait_timeout_setter(lib):
+    assert lib.lr_set_wait_timeout_us(500) == L.LR_OK
+    assert lib.lr_set_wait_timeout_us(0) == L.LR_OK

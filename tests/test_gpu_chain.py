@@ -50,18 +50,34 @@ def test_decode_stack_chain(cuda_device, layers4, batch):
     assert int(ws.count_nonzero()) == 0
 
 
-def test_chain_matches_separate_calls_and_older_inputs(cuda_device, layers4):
+def test_chain_older_inputs_against_oracle(cuda_device, layers4):
     L0, L1 = layers4[0], layers4[1]
-    x = dev(synth.make_activations(2, 4096, seed=6, key=(71,)))
-    # step 2 reads step 0's output (two steps back: the stored bf16 output)
+    x = synth.make_activations(2, 4096, seed=6, key=(71,))
+    # step 1 reads step 0's second output (at fp32, the step right before);
+    # step 2 reads step 0's first output two steps back (its stored bf16 output)
     steps = [lr.ChainStep([_fac(L0["q"]), _fac(L0["v"])]), lr.ChainStep([_fac(L0["o"])], 0, 1),
              lr.ChainStep([_fac(L1["k"])], 0, 0)]
-    outs = lr.lr_linear_chain(steps, x)
-    q, v = lr.lr_linear_grouped([_fac(L0["q"]), _fac(L0["v"])], x)
-    o = lr.lr_linear(_fac(L0["o"]), v)
-    k = lr.lr_linear(_fac(L1["k"]), q)
+    outs = lr.lr_linear_chain(steps, dev(x))
+    x64 = x.double().numpy()
+    q, v = _oracle(L0["q"], x64), _oracle(L0["v"], x64)
+    o, k = _oracle(L0["o"], v), _oracle(L1["k"], q)
     for got, ref in ((outs[0][0], q), (outs[0][1], v), (outs[1][0], o), (outs[2][0], k)):
-        assert normwise_rel(got, ref.double().cpu().numpy()) < NORMWISE_TOL
+        assert normwise_rel(got, ref) < NORMWISE_TOL
+
+
+def test_chain_four_projections_one_consumed(cuda_device, layers4):
+    # three steps of four projections each; only the last projection of a step
+    # feeds the next, so the other three are scheduled as fillers
+    x = synth.make_activations(1, 4096, seed=8, key=(73,))
+    names = ("q", "k", "v", "o")
+    steps = [lr.ChainStep([_fac(layers4[l][n]) for n in names], -1 if l == 0 else l - 1, 3) for l in range(3)]
+    outs = lr.lr_linear_chain(steps, dev(x))
+    x64 = x.double().numpy()
+    for l in range(3):
+        refs = [_oracle(layers4[l][n], x64) for n in names]
+        for got, ref in zip(outs[l], refs):
+            assert normwise_rel(got, ref) < NORMWISE_TOL, l
+        x64 = refs[3]
 
 
 def test_chain_int8_and_fp32(cuda_device):
