@@ -26,6 +26,11 @@ end-to-end time through the C ABI with host buffers:
   c3b1/8/32 hybrid int8 SwiGLU FFN (7B shapes), batch 1, 8, 32
   c4k4/16/32 latent-KV flash decoding, batch 8, 32 heads, rank 32, ctx 4K/16K/32K
   c5        W8A8 prefill of one 13B layer (7 projections), 2048 tokens
+and the uncompressed baselines the pages compare against, with the speed-up
+of the low-rank path over each:
+  c2dense   dense bf16 Q/K/V/O stack, 32 layers, batch 1
+  c3dense   dense int8 SwiGLU FFN (all 11008 channels dense), batch 1
+  c4full*   flash decoding over full K/V reconstructed from the same latents
 
 `--impl reference` times the CPU oracle (the float64 reference
 implementation) on the headline workload instead, on the host cores.
@@ -51,7 +56,8 @@ METRIC = "decode-layer µs & achieved HBM GB/s (% of B200 roofline) at batch 1; 
 LAYERS, HIDDEN = 32, 4096
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
-ROW_IDS = ("c1", "c2b4", "c2b16", "c3b1", "c3b8", "c3b32", "c4k4", "c4k16", "c4k32", "c5")
+ROW_IDS = ("c1", "c2b4", "c2b16", "c2dense", "c3b1", "c3b8", "c3b32", "c3dense", "c4k4", "c4k16", "c4k32",
+           "c4full4", "c4full16", "c4full32", "c5")
 
 
 def parse(argv=None):
@@ -484,6 +490,9 @@ def run_ours(args) -> None:
 
     if rank == 0 and world == 1 and not args.no_rows:
         rows = run_rows(args, lr, L, synth, device, ranks, layers, only)
+        dense = [r for r in rows if r["row"] == "c2dense"]
+        if out is not None and dense:
+            out["speedup_vs_uncompressed"] = out["value"] / dense[0]["value"]
         if out is None:
             for r in rows:
                 print(json.dumps(r), flush=True)
@@ -746,6 +755,108 @@ def row_c5(lr, L, synth, device, want_cpu):
     return row
 
 
+def row_c2dense(lr, L, synth, device, want_cpu):
+    """Dense bf16 Q/K/V/O stack (the uncompressed model's projections), 32 layers, batch 1."""
+    import torch
+    from oracle import lowrank
+    gen = torch.Generator(device=device).manual_seed(0)
+    Wqkv = [(torch.randn(3 * HIDDEN, HIDDEN, device=device, generator=gen) / 64).to(torch.bfloat16) for _ in range(LAYERS)]
+    Wo = [(torch.randn(HIDDEN, HIDDEN, device=device, generator=gen) / 64).to(torch.bfloat16) for _ in range(LAYERS)]
+    x0 = synth.make_activations(1, HIDDEN, seed=0, key=(90,)).to(device)
+    qkv = [torch.empty(1, 3 * HIDDEN, dtype=torch.bfloat16, device=device) for _ in range(LAYERS)]
+    outs = [torch.empty(1, HIDDEN, dtype=torch.bfloat16, device=device) for _ in range(LAYERS)]
+
+    def step(_):
+        x = x0
+        for l in range(LAYERS):
+            lr.lr_dense_linear(Wqkv[l], x, y=qkv[l])
+            lr.lr_dense_linear(Wo[l], qkv[l][:, 2 * HIDDEN:], y=outs[l])
+            x = outs[l]
+    ms = time_graph(step, 5)
+    alg = LAYERS * 4 * HIDDEN * HIDDEN * 2 + LAYERS * HIDDEN * 2 * 6
+    lib = L.load()
+    xh = synth.make_activations(1, HIDDEN, seed=0, key=(90,)).pin_memory()
+    yh = torch.empty(1, HIDDEN, dtype=torch.bfloat16).pin_memory()
+
+    def e2e():
+        x0.copy_(xh, non_blocking=True)
+        x = x0
+        for l in range(LAYERS):
+            L.check("lr_dense_linear", lib.lr_dense_linear(Wqkv[l].data_ptr(), L.LR_BF16, None, L.LR_F32, HIDDEN,
+                                                           3 * HIDDEN, x.data_ptr(), 1, qkv[l].data_ptr(), stream_ptr()))
+            v = qkv[l][:, 2 * HIDDEN:]
+            L.check("lr_dense_linear", lib.lr_dense_linear(Wo[l].data_ptr(), L.LR_BF16, None, L.LR_F32, HIDDEN, HIDDEN,
+                                                           v.data_ptr(), 1, outs[l].data_ptr(), stream_ptr()))
+            x = outs[l]
+        yh.copy_(outs[-1], non_blocking=True)
+    ms_e2e = time_e2e(e2e, 10)
+    row = {"row": "c2dense", "workload": "dense bf16 Q/K/V/O (4096 x 4096 each), 32 layers, batch 1 (the "
+                                         "uncompressed baseline of the headline stack)",
+           "value": 1 / (ms * 1e-3), "unit": "tokens/s", "higher_is_better": True, "ms_per_step": ms,
+           "layer_us": ms * 1e3 / LAYERS, "launches": 2 * LAYERS,
+           "roofline": _roof_hbm(alg, ms, "lr_dense_linear (dense dot rows), one launch for Q/K/V and one for O per "
+                                          "layer"),
+           "e2e": {"value": 1 / (ms_e2e * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": HIDDEN * 2,
+                   "d2h_bytes_per_step": HIDDEN * 2, "path": "lr_dense_linear through the C ABI"},
+           "l2": "4.3 GB of weights streamed per step"}
+    if want_cpu:
+        W1 = Wqkv[0].double().cpu().numpy()
+        W2 = Wo[0].double().cpu().numpy()
+        x64 = x0.double().cpu().numpy()
+        sec, n = cpu_timed(lambda: lowrank.dense_linear(lowrank.dense_linear(x64, W1.T)[:, 2 * HIDDEN:], W2.T), 2.0)
+        row["cpu_baseline"] = {"value": 1 / (sec * LAYERS), "unit": "tokens/s", "cores": host_cores(),
+                               "kind": "oracle", "sample": f"{n} call(s) of the float64 oracle on one layer, scaled "
+                                                          f"to 32 layers"}
+    del Wqkv, Wo
+    return row
+
+
+def row_c4full(lr, L, synth, device, ctx, want_cpu):
+    """Flash decoding over full K/V reconstructed (bf16) from the latent caches of c4."""
+    import torch
+    from oracle import attention
+    kvd = synth.make_latent_kv(batch=8, heads=32, ctx=ctx, seed=0)
+    CK, CV = kvd["C_K"].to(device), kvd["C_V"].to(device)
+    K = torch.einsum("bhtr,hrd->bhtd", CK.float(), kvd["B_K"].to(device).float()).to(torch.bfloat16).contiguous()
+    V = torch.einsum("bhtr,hrd->bhtd", CV.float(), kvd["B_V"].to(device).float()).to(torch.bfloat16).contiguous()
+    del CK, CV
+    q, sl = kvd["q"].to(device), kvd["seq_lens"].to(device)
+    o = torch.empty(8, 32, 128, dtype=torch.bfloat16, device=device)
+    d = L.FlashDesc(8, 32, 128, ctx, float(kvd["scale"]), 0)
+    n = ctypes.c_size_t(0)
+    lib = L.load()
+    L.check("ws", lib.lr_flash_decode_workspace_size(ctypes.byref(d), ctypes.byref(n)))
+    ws = lr.workspace(n.value, device)
+    ms = time_graph(lambda i: lr.lr_flash_decode(q, K, V, sl, kvd["scale"], o, ws), 20)
+    alg = int(K.numel() * 2 * 2 + 2 * q.numel() * 2)
+    qh, oh = kvd["q"].pin_memory(), torch.empty(8, 32, 128, dtype=torch.bfloat16).pin_memory()
+
+    def e2e():
+        q.copy_(qh, non_blocking=True)
+        L.check("lr_flash_decode", lib.lr_flash_decode(ctypes.byref(d), q.data_ptr(), K.data_ptr(), V.data_ptr(),
+                                                       sl.data_ptr(), o.data_ptr(), ws.data_ptr(), ws.numel(),
+                                                       stream_ptr()))
+        oh.copy_(o, non_blocking=True)
+    ms_e2e = time_e2e(e2e, 20)
+    row = {"row": f"c4full{ctx // 1024}", "workload": f"flash decoding over full K/V (bf16, head_dim 128, "
+                                                     f"reconstructed from the c4 latents), batch 8, 32 heads, ctx {ctx}",
+           "value": ms * 1e3, "unit": "µs per call", "higher_is_better": False, "launches": 2,
+           "roofline": _roof_hbm(alg, ms, "split kernel (dominant) + combine kernel"),
+           "e2e": {"value": ms_e2e * 1e3, "unit": "µs per call", "h2d_bytes_per_step": int(q.numel() * 2),
+                   "d2h_bytes_per_step": int(o.numel() * 2), "path": "lr_flash_decode through the C ABI"},
+           "l2": f"{alg / 1e9:.2f} GB of K/V per call"}
+    if want_cpu:
+        pairs = [(b, h) for b in range(0, 8, 2) for h in (0, 17)]
+        Kc, Vc = K.cpu(), V.cpu()
+        sec, cnt = cpu_timed(lambda: attention.decode_attention(kvd["q"], Kc, Vc, kvd["seq_lens"], kvd["scale"], pairs),
+                             2.0, 10)
+        row["cpu_baseline"] = {"value": sec * 1e6 * 256 / len(pairs), "unit": "µs per call", "cores": host_cores(),
+                               "kind": "oracle", "sample": f"{cnt} call(s) of the float64 oracle on {len(pairs)} of "
+                                                          f"the 256 (batch, head) pairs, scaled to 256"}
+    del K, V, ws
+    return row
+
+
 def run_rows(args, lr, L, synth, device, ranks, layers, only) -> list:
     import torch
     want_cpu = not args.no_cpu_baseline
@@ -754,26 +865,45 @@ def run_rows(args, lr, L, synth, device, ranks, layers, only) -> list:
     clocks = ClockSampler(device.index).start()
     clocks.wait_first_sample()
     for rid in sel:
-        if rid.startswith("c2"):
+        if rid.startswith("c2b"):
             rows.append(row_c2(lr, L, synth, device, ranks, layers, int(rid[3:]), want_cpu))
     del layers
     torch.cuda.empty_cache()
     if "c1" in sel:
         rows.insert(0, row_c1(lr, L, synth, device, want_cpu))
+    if "c2dense" in sel:
+        rows.append(row_c2dense(lr, L, synth, device, want_cpu))
+        torch.cuda.empty_cache()
     ffn = None
     for rid in sel:
-        if rid.startswith("c3"):
+        if rid.startswith("c3b"):
             ffn = ffn or synth.make_hybrid_ffn(seed=0)
             rows.append(row_c3(lr, L, synth, device, ffn, int(rid[3:]), want_cpu))
             torch.cuda.empty_cache()
+    if "c3dense" in sel:
+        dense = synth.make_hybrid_ffn(seed=0, n_lr=0, rotate=False)
+        r = row_c3(lr, L, synth, device, dense, 1, want_cpu)
+        r["row"], r["workload"] = "c3dense", ("dense int8 SwiGLU FFN (all 11008 channels dense), 7B shapes, batch 1 "
+                                              "(the uncompressed baseline of c3)")
+        rows.append(r)
+        del dense
+        torch.cuda.empty_cache()
     for rid in sel:
-        if rid.startswith("c4"):
+        if rid.startswith("c4k"):
             rows.append(row_c4(lr, L, synth, device, int(rid[3:]) * 1024, want_cpu))
+            torch.cuda.empty_cache()
+        elif rid.startswith("c4full"):
+            rows.append(row_c4full(lr, L, synth, device, int(rid[6:]) * 1024, want_cpu))
             torch.cuda.empty_cache()
     if "c5" in sel:
         rows.append(row_c5(lr, L, synth, device, want_cpu))
     clk = clocks.stop()
     check_device(lr)
+    by = {r["row"]: r for r in rows}
+    # speed-up of each low-rank row over its uncompressed baseline (same work, same units)
+    for low, base in (("c3b1", "c3dense"), ("c4k4", "c4full4"), ("c4k16", "c4full16"), ("c4k32", "c4full32")):
+        if low in by and base in by:
+            by[low]["speedup_vs_uncompressed"] = by[base]["value"] / by[low]["value"]
     for r in rows:
         r["clocks"] = clk
     return rows

@@ -38,6 +38,10 @@ class ChainStep(ctypes.Structure):
                 ("proj", FactorDesc * 4), ("y", c_void_p * 4)]
 
 
+class RankVec(ctypes.Structure):
+    _fields_ = [("n", c_int), ("ranks", ctypes.POINTER(c_int))]
+
+
 class FfnDesc(ctypes.Structure):
     _fields_ = [("hidden", c_int), ("inter", c_int), ("n_lr", c_int), ("rank", c_int), ("scale_dtype", c_int),
                 ("A", c_void_p), ("s_A", c_void_p), ("B", c_void_p), ("s_B", c_void_p),
@@ -50,6 +54,11 @@ class LatentKvDesc(ctypes.Structure):
                 ("split_tokens", c_int)]
 
 
+class FlashDesc(ctypes.Structure):
+    _fields_ = [("batch", c_int), ("heads", c_int), ("head_dim", c_int), ("max_ctx", c_int), ("scale", c_float),
+                ("split_tokens", c_int)]
+
+
 P = ctypes.POINTER
 _SIGNATURES = {
     "lr_linear": (c_int, [P(FactorDesc), c_void_p, c_void_p, c_int, c_void_p, c_void_p, c_size_t, c_void_p]),
@@ -57,14 +66,21 @@ _SIGNATURES = {
     "lr_linear_noalloc": (c_int, [P(FactorDesc), c_void_p, c_int, c_void_p, c_void_p]),
     "lr_linear_chain": (c_int, [P(ChainStep), c_int, c_void_p, c_int, c_void_p, c_size_t, c_void_p]),
     "lr_linear_chain_workspace_size": (c_int, [P(ChainStep), c_int, c_int, P(c_size_t)]),
+    "lr_rank_allocate": (c_int, [P(ctypes.c_double), c_int, ctypes.c_double, P(RankVec), P(c_int)]),
+    "lr_linear_chain_ranked": (c_int, [P(ChainStep), c_int, P(RankVec), c_void_p, c_int, c_void_p, c_size_t,
+                                       c_void_p]),
     "lr_linear_grouped": (c_int, [P(FactorDesc), c_int, c_void_p, c_int, P(c_void_p), c_void_p, c_size_t,
                                   c_void_p]),
     "lr_linear_grouped_workspace_size": (c_int, [P(FactorDesc), c_int, c_int, P(c_size_t)]),
+    "lr_dense_linear": (c_int, [c_void_p, c_int, c_void_p, c_int, c_int, c_int, c_void_p, c_int, c_void_p, c_void_p]),
     "lr_swiglu_ffn": (c_int, [P(FfnDesc), c_void_p, c_int, c_void_p, c_void_p, c_size_t, c_void_p]),
     "lr_swiglu_ffn_workspace_size": (c_int, [P(FfnDesc), c_int, P(c_size_t)]),
     "lr_latent_kv_decode": (c_int, [P(LatentKvDesc), c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                                     c_size_t, c_void_p]),
     "lr_latent_kv_workspace_size": (c_int, [P(LatentKvDesc), P(c_size_t)]),
+    "lr_flash_decode": (c_int, [P(FlashDesc), c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_size_t,
+                                c_void_p]),
+    "lr_flash_decode_workspace_size": (c_int, [P(FlashDesc), P(c_size_t)]),
     "lr_quantize_per_token": (c_int, [c_void_p, c_int, c_int, c_void_p, c_void_p, c_void_p]),
     "lr_gemm_s8s32": (c_int, [c_void_p, c_void_p, c_int, c_int, c_int, c_int, c_void_p, c_void_p]),
     "lr_workspace_init": (c_int, [c_void_p, c_size_t, c_void_p]),

@@ -2,6 +2,7 @@
 // and dispatch to the sm_100a kernels.  Nothing here computes on the host.
 #include <algorithm>
 #include <atomic>
+#include <cmath>
 #include <cstdint>
 #include <cstring>
 #include <mutex>
@@ -378,6 +379,48 @@ lr_status_t lr_linear_chain_workspace_size(const lr_chain_step_t* steps, int n_s
   return LR_OK;
 }
 
+lr_status_t lr_rank_allocate(const double* alpha, int n, double r_budget, const lr_rank_vec_t* cap,
+                             int* ranks_out) {
+  if (!alpha || n < 1 || !cap || !cap->ranks || cap->n != n || !ranks_out) return LR_ERR_INVALID_ARG;
+  if (!(r_budget >= 0.0) || !std::isfinite(r_budget)) return LR_ERR_INVALID_ARG;
+  double S = 0.0;
+  for (int p = 0; p < n; ++p) {
+    if (!(alpha[p] > 0.0) || !std::isfinite(alpha[p]) || cap->ranks[p] < 1) return LR_ERR_INVALID_ARG;
+    S += alpha[p];
+  }
+  for (int p = 0; p < n; ++p) {
+    const double r = std::nearbyint((alpha[p] / S) * r_budget);  // default rounding: to nearest, ties to even
+    ranks_out[p] = int(std::min(std::max(r, 1.0), double(cap->ranks[p])));
+  }
+  return LR_OK;
+}
+
+lr_status_t lr_linear_chain_ranked(const lr_chain_step_t* steps, int n_steps, const lr_rank_vec_t* active,
+                                   const void* x, int batch, void* ws, size_t ws_bytes, lr_stream_t stream) {
+  if (!steps || n_steps < 1 || n_steps > LR_MAX_CHAIN || !active || !active->ranks) return LR_ERR_INVALID_ARG;
+  int total = 0;
+  for (int s = 0; s < n_steps; ++s) {
+    if (steps[s].n < 1 || steps[s].n > LR_MAX_GROUP) return LR_ERR_INVALID_ARG;
+    total += steps[s].n;
+  }
+  if (active->n != total) return LR_ERR_INVALID_ARG;
+  static lr_factor_desc_t descs[LR_MAX_CHAIN][LR_MAX_GROUP];  // the steps' descriptors with the vector's ranks
+  static std::mutex mu;
+  std::lock_guard<std::mutex> lock(mu);
+  HostStep h[LR_MAX_CHAIN];
+  int k = 0;
+  for (int s = 0; s < n_steps; ++s) {
+    for (int p = 0; p < steps[s].n; ++p, ++k) {
+      descs[s][p] = steps[s].proj[p];
+      const int r = active->ranks[k];
+      if (r < 0 || r > descs[s][p].rank) return LR_ERR_INVALID_ARG;
+      descs[s][p].active_rank = r == descs[s][p].rank ? 0 : r;
+    }
+    h[s] = HostStep{descs[s], steps[s].n, steps[s].input_step, steps[s].input_proj, steps[s].y};
+  }
+  return run_chain(h, n_steps, x, batch, ws, ws_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
 lr_status_t lr_linear_chain(const lr_chain_step_t* steps, int n_steps, const void* x, int batch, void* ws,
                             size_t ws_bytes, lr_stream_t stream) {
   if (!steps || n_steps < 1 || n_steps > LR_MAX_CHAIN) return LR_ERR_INVALID_ARG;
@@ -408,6 +451,29 @@ static size_t ffn_ws_bytes(const lr_ffn_desc_t* d, int batch) {
   const int n_dense = d->inter - d->n_lr;
   return kTicketBytes + round_up(size_t(chunk) * 2 * d->n_lr * 4, 256) + round_up(size_t(chunk) * n_dense * 4, 256) +
          round_up(size_t(chunk) * d->hidden * 4, 256);
+}
+
+lr_status_t lr_dense_linear(const void* W, lr_dtype_t w_dtype, const void* scale, lr_dtype_t scale_dtype, int d_in,
+                            int d_out, const void* x, int batch, void* y, lr_stream_t stream) {
+  if (!W || !x || !y || d_in <= 0 || d_out <= 0 || batch < 1) return LR_ERR_INVALID_ARG;
+  if (w_dtype != LR_BF16 && w_dtype != LR_I8) return LR_ERR_UNSUPPORTED;
+  if (w_dtype == LR_I8 && !scale) return LR_ERR_INVALID_ARG;
+  if (scale && scale_dtype != LR_F16 && scale_dtype != LR_F32) return LR_ERR_UNSUPPORTED;
+  const size_t es = w_dtype == LR_BF16 ? 2 : 1;
+  if ((d_in % 16) != 0 || size_t(d_in) * es > 32768) return LR_ERR_UNSUPPORTED;
+  if (!al16(W) || !al16(x) || !al16(y) || (scale && !al16(scale))) return LR_ERR_MISALIGNED;
+  FfnParams P;
+  std::memset(&P, 0, sizeof(P));
+  P.hidden = d_in;
+  P.n_dense = d_out;
+  P.nb = batch;
+  P.D = reinterpret_cast<const int8_t*>(W);
+  P.sD = scale;
+  P.scale_f16 = scale_dtype == LR_F16 ? 1 : 0;
+  P.x = x;
+  P.y = y;
+  P.err = device_error_word();
+  return from_cuda(launch_dense(P, w_dtype, sm_count_current(), reinterpret_cast<cudaStream_t>(stream)));
 }
 
 lr_status_t lr_swiglu_ffn_workspace_size(const lr_ffn_desc_t* desc, int batch, size_t* bytes) {
@@ -503,6 +569,47 @@ lr_status_t lr_latent_kv_decode(const lr_latent_kv_desc_t* d, const void* q, con
 }
 
 // --------------------------------------------------------------------------
+
+static lr_status_t check_flash(const lr_flash_desc_t* d, int* split) {
+  if (!d) return LR_ERR_INVALID_ARG;
+  if (d->batch <= 0 || d->heads <= 0 || d->max_ctx <= 0 || d->head_dim <= 0) return LR_ERR_INVALID_ARG;
+  if (d->head_dim != 128) return LR_ERR_UNSUPPORTED;
+  if (d->split_tokens < 0 || (d->split_tokens % 64) != 0 || d->split_tokens > 256) return LR_ERR_INVALID_ARG;
+  if (d->heads > 65535 || d->batch > 65535) return LR_ERR_UNSUPPORTED;
+  *split = d->split_tokens ? d->split_tokens : 128;
+  return LR_OK;
+}
+
+lr_status_t lr_flash_decode_workspace_size(const lr_flash_desc_t* d, size_t* bytes) {
+  int t = 0;
+  if (!bytes) return LR_ERR_INVALID_ARG;
+  lr_status_t st = check_flash(d, &t);
+  if (st != LR_OK) return st;
+  const size_t ns = (size_t(d->max_ctx) + t - 1) / t;
+  *bytes = size_t(d->batch) * d->heads * ns * flash_partial_floats() * 4;
+  return LR_OK;
+}
+
+lr_status_t lr_flash_decode(const lr_flash_desc_t* d, const void* q, const void* K, const void* V,
+                            const int* seq_lens, void* out, void* ws, size_t ws_bytes, lr_stream_t stream) {
+  int t = 0;
+  lr_status_t st = check_flash(d, &t);
+  if (st != LR_OK) return st;
+  if (!q || !K || !V || !seq_lens || !out) return LR_ERR_INVALID_ARG;
+  if (!al16(q) || !al16(K) || !al16(V) || !al16(seq_lens) || !al16(out)) return LR_ERR_MISALIGNED;
+  size_t need = 0;
+  lr_flash_decode_workspace_size(d, &need);
+  if (!ws || ws_bytes < need) return LR_ERR_WORKSPACE;
+  if (!al16(ws)) return LR_ERR_MISALIGNED;
+  FlashParams P;
+  std::memset(&P, 0, sizeof(P));
+  P.batch = d->batch; P.heads = d->heads; P.max_ctx = d->max_ctx;
+  P.split_tokens = t; P.n_splits = (d->max_ctx + t - 1) / t; P.scale = d->scale;
+  P.q = q; P.K = K; P.V = V; P.seq_lens = seq_lens; P.out = out;
+  P.partial = reinterpret_cast<float*>(ws);
+  P.err = device_error_word();
+  return from_cuda(launch_flash(P, reinterpret_cast<cudaStream_t>(stream)));
+}
 
 lr_status_t lr_quantize_per_token(const void* x, int rows, int cols, int8_t* x_q, float* s, lr_stream_t stream) {
   if (!x || !x_q || !s || rows < 1 || cols < 1) return LR_ERR_INVALID_ARG;

@@ -38,7 +38,7 @@ constexpr int kRowGroup = 4;               // rows reduced together in phase A (
 constexpr int kMaxSegs = 2 * kMaxGroup;
 constexpr size_t kSmemLimit = 227 * 1024;
 
-enum Mode : int { kFfn1 = 1, kFfn2 = 2 };
+enum Mode : int { kFfn1 = 1, kFfn2 = 2, kDense = 3 };
 enum SegKind : int { kDot = 0, kRank1 = 1 };
 
 struct Seg {
@@ -377,6 +377,15 @@ LR_DEV void build_plan(const KParams& K, Plan& pl) {
       pl.row_base = 2 * p0;
       add(F.D, size_t(2 * p0), F.hidden, 2 * (p1 - p0), kDot, 0, 0);
     }
+  } else if constexpr (MODE == kDense) {
+    // dense output-major rows W [d_out, d_in]: f.D = W, f.n_dense = d_out, f.hidden = d_in
+    const FfnParams& F = K.f;
+    int c0, c1;
+    split_range(F.n_dense, blockIdx.x, gridDim.x, &c0, &c1);
+    pl.role = 2;
+    pl.nrows = c1 - c0;
+    pl.row_base = c0;
+    add(F.D, size_t(c0), F.hidden * int(sizeof(WT)), c1 - c0, kDot, 0, 0);
   } else {
     const FfnParams& F = K.f;
     int c0, c1;
@@ -393,6 +402,7 @@ LR_DEV float row_scale(const KParams& K, const Plan& pl, int r) {
   const bool f16 = K.f.scale_f16 != 0;
   {
     if (pl.role == 0) return load_scale(K.f.sA, pl.row_base + r, f16);
+    if (pl.role == 2 && !K.f.sD) return 1.f;
     return load_scale(K.f.sD, pl.row_base + r, f16);
   }
 }
@@ -530,6 +540,20 @@ __global__ void __launch_bounds__(kThreads, (NB <= 1 && LPW <= 2 ? 2 : 1)) strea
         flush_rank1<NB, LPW>(acc, dst, elems, nb, cw, lane);
       }
     }
+    if constexpr (MODE == kDense) {
+      // y[b][row] = row . x_b * scale[row]
+      consumer_sync();
+      for (int i = threadIdx.x; i < pl.nrows * NB; i += kConsumers) {
+        const int r = i / NB, b = i % NB;
+        if (b < nb) {
+          float v = 0.f;
+#pragma unroll 4
+          for (int w = 0; w < kConsumerWarps; ++w) v += part[(r * kConsumerWarps + w) * NB + b];
+          reinterpret_cast<__nv_bfloat16*>(K.f.y)[size_t(b) * K.f.n_dense + pl.row_base + r] =
+              __float2bfloat16_rn(v * row_scale<MODE>(K, pl, r));
+        }
+      }
+    }
     if constexpr (MODE == kFfn1) {
       if (pl.role == 1) {
         // dense branch: g, u of each channel pair, SwiGLU, h_D
@@ -554,7 +578,7 @@ __global__ void __launch_bounds__(kThreads, (NB <= 1 && LPW <= 2 ? 2 : 1)) strea
     }
   }
 
-  if constexpr (MODE == kFfn1) {
+  if constexpr (MODE == kFfn1 || MODE == kDense) {
     return;
   } else {
     unsigned int* words = K.f.ticket;
@@ -685,8 +709,35 @@ cudaError_t launch_ffn_impl(const FfnParams& p0, int sm_count, cudaStream_t s) {
   return cudaSuccess;
 }
 
+// Dense GEMV: every CTA owns a block of output rows; no reduction, no barrier.
+template <typename WT>
+cudaError_t launch_dense_impl(const FfnParams& p0, int sm_count, cudaStream_t s) {
+  if (p0.hidden * int(sizeof(WT)) > kStageBytes) return cudaErrorInvalidValue;
+  const int grid = std::min(sm_count, p0.n_dense);
+  KParams K;
+  std::memset(&K, 0, sizeof(K));
+  K.err = p0.err;
+  K.rows_cap = (p0.n_dense + grid - 1) / grid;
+  K.x_elems = p0.hidden;
+  for (int b0 = 0; b0 < p0.nb; b0 += kMaxDecodeChunk) {
+    FfnParams f = p0;
+    f.nb = std::min(kMaxDecodeChunk, p0.nb - b0);
+    f.x = reinterpret_cast<const __nv_bfloat16*>(p0.x) + size_t(b0) * p0.hidden;
+    f.y = reinterpret_cast<__nv_bfloat16*>(p0.y) + size_t(b0) * p0.n_dense;
+    K.f = f;
+    cudaError_t e = dispatch<WT, __nv_bfloat16, __nv_bfloat16, kDense>(K, f.nb, 1, grid, sm_count, s);
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
 }  // namespace
 
 cudaError_t launch_ffn(const FfnParams& p, int sm_count, cudaStream_t s) { return launch_ffn_impl(p, sm_count, s); }
+
+cudaError_t launch_dense(const FfnParams& p, lr_dtype_t w_dtype, int sm_count, cudaStream_t s) {
+  return w_dtype == LR_BF16 ? launch_dense_impl<__nv_bfloat16>(p, sm_count, s)
+                            : launch_dense_impl<int8_t>(p, sm_count, s);
+}
 
 }  // namespace lr

@@ -88,6 +88,9 @@ struct FfnParams {
 };
 
 cudaError_t launch_ffn(const FfnParams& p, int sm_count, cudaStream_t s);
+// Dense GEMV y = x W^T for output-major W [n_dense rows, hidden] in p.D (bf16 or
+// int8 with per-row scales p.sD, or none); p.x, p.y, p.nb as for the FFN.
+cudaError_t launch_dense(const FfnParams& p, lr_dtype_t w_dtype, int sm_count, cudaStream_t s);
 
 struct LatentKvParams {
   int batch, heads, head_dim, rank, max_ctx;
@@ -103,6 +106,21 @@ struct LatentKvParams {
 };
 
 cudaError_t launch_latent_kv(const LatentKvParams& p, cudaStream_t s);
+
+// Full-K/V flash decoding (the uncompressed baseline).
+struct FlashParams {
+  int batch, heads, max_ctx;
+  int split_tokens, n_splits;
+  float scale;
+  const void* q; const void* K; const void* V;   // bf16 [batch, heads, (max_ctx,) 128]
+  const int* seq_lens;
+  void* out;          // bf16 [batch, heads, 128]
+  float* partial;     // [batch, heads, n_splits, 130]
+  int* err;
+};
+
+size_t flash_partial_floats();
+cudaError_t launch_flash(const FlashParams& p, cudaStream_t s);
 
 cudaError_t launch_quantize_per_token(const void* x, int rows, int cols, int8_t* xq, float* s,
                                       cudaStream_t st);

@@ -292,3 +292,67 @@ def lr_check_device_error(stream=None) -> int:
 def lr_set_wait_timeout_us(us: int) -> None:
     """Bound of a persistent kernel's waits on its other CTAs, in microseconds (0: default, 1 s)."""
     L.check("lr_set_wait_timeout_us", L.load().lr_set_wait_timeout_us(int(us)))
+
+
+def _rank_vec(values):
+    arr = (ctypes.c_int * len(values))(*[int(v) for v in values])
+    return L.RankVec(len(values), arr), arr
+
+
+def lr_rank_allocate(alpha: Sequence[float], r_budget: float, caps: Sequence[int]) -> list:
+    """FLRC ranks r_p = clamp(round(alpha_p / S * r_budget), 1, caps_p), computed by the library (host)."""
+    n = len(alpha)
+    a = (ctypes.c_double * n)(*[float(v) for v in alpha])
+    cap, _keep = _rank_vec(caps)
+    out = (ctypes.c_int * n)()
+    L.check("lr_rank_allocate", L.load().lr_rank_allocate(a, n, float(r_budget), ctypes.byref(cap), out))
+    return list(out)
+
+
+def lr_linear_chain_ranked(steps: Sequence[ChainStep], x: torch.Tensor, active: Sequence[int],
+                           ws: Optional[torch.Tensor] = None, stream=None) -> list:
+    """lr_linear_chain with per-projection active ranks (chain order, 0 = every component)."""
+    batch = x.shape[0]
+    for st in steps:
+        if st.ys is None:
+            st.ys = [torch.empty(batch, f.d_out, dtype=f.out_dtype(), device=x.device) for f in st.factors]
+    if ws is None:
+        ws = workspace(lr_linear_chain_workspace_size(steps, batch), x.device)
+    arr = _chain_array(steps)
+    rv, _keep = _rank_vec(active)
+    L.check("lr_linear_chain_ranked", L.load().lr_linear_chain_ranked(arr, len(steps), ctypes.byref(rv), _ptr(x), batch,
+                                                                      _ptr(ws), ws.numel() * ws.element_size(),
+                                                                      _stream(stream)))
+    return [list(st.ys) for st in steps]
+
+
+def lr_dense_linear(W: torch.Tensor, x: torch.Tensor, scale: Optional[torch.Tensor] = None,
+                    y: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Dense baseline y = x W_store^T for an output-major weight W_store [d_out, d_in] (bf16, or int8 + scale)."""
+    d_out, d_in = W.shape
+    batch = x.shape[0]
+    if y is None:
+        y = torch.empty(batch, d_out, dtype=torch.bfloat16, device=x.device)
+    sd = _DT[scale.dtype] if scale is not None else L.LR_F32
+    L.check("lr_dense_linear", L.load().lr_dense_linear(_ptr(W), _DT[W.dtype], _ptr(scale), sd, d_in, d_out, _ptr(x),
+                                                        batch, _ptr(y), _stream(stream)))
+    return y
+
+
+def lr_flash_decode(q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, seq_lens: torch.Tensor, scale: float,
+                    out: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None, split_tokens: int = 0,
+                    stream=None) -> torch.Tensor:
+    """Flash decoding over full K/V [batch, heads, max_ctx, 128] (the uncompressed baseline)."""
+    batch, heads, max_ctx, hd = K.shape
+    d = L.FlashDesc(batch, heads, hd, max_ctx, float(scale), split_tokens)
+    if out is None:
+        out = torch.empty(batch, heads, hd, dtype=torch.bfloat16, device=q.device)
+    if ws is None:
+        n = ctypes.c_size_t(0)
+        L.check("lr_flash_decode_workspace_size", L.load().lr_flash_decode_workspace_size(ctypes.byref(d),
+                                                                                          ctypes.byref(n)))
+        ws = workspace(n.value, q.device)
+    L.check("lr_flash_decode", L.load().lr_flash_decode(ctypes.byref(d), _ptr(q), _ptr(K), _ptr(V), _ptr(seq_lens),
+                                                        _ptr(out), _ptr(ws), ws.numel() * ws.element_size(),
+                                                        _stream(stream)))
+    return out

@@ -191,6 +191,44 @@ LR_API lr_status_t lr_linear_chain_workspace_size(const lr_chain_step_t* steps, 
                                                   size_t* bytes);
 
 /*
+ * Rank vectors: one rank per projection, in chain order (step 0's projections,
+ * then step 1's, ...).  `ranks` is a host array of n entries, read during the
+ * call and not kept.
+ */
+typedef struct lr_rank_vec {
+  int n;
+  const int* ranks;
+} lr_rank_vec_t;
+
+/*
+ * FLRC rank allocation (FLRC "Fisher-based layer-wise rank allocation":
+ * r_{l,p} = round(alpha_{l,p} / S * R_budget), S the total importance; FLRC
+ * "progressive low-rank decoding": the same rule per token t with a
+ * non-increasing budget R_budget(t)).  Host-only, no device work:
+ *   alpha      host array of n importances (> 0, finite)
+ *   r_budget   total rank budget (>= 0)
+ *   cap        the stored ranks (cap->n == n); each result is clamped to
+ *              [1, cap->ranks[p]] (a rank of 0 would drop the projection)
+ *   ranks_out  host array of n results
+ * S is summed in index order, alpha_p / S * r_budget is evaluated in double
+ * and rounded to nearest, ties to even.  Errors: LR_ERR_INVALID_ARG.
+ */
+LR_API lr_status_t lr_rank_allocate(const double* alpha, int n, double r_budget, const lr_rank_vec_t* cap,
+                                    int* ranks_out);
+
+/*
+ * lr_linear_chain with the active rank of every projection taken from a rank
+ * vector (active->n = total projections of the chain, entry p in [0, rank];
+ * 0 = every stored component), e.g. the per-token ranks of FLRC progressive
+ * decoding from lr_rank_allocate.  The factors are SVD-ordered, so a lower
+ * active rank streams a prefix of each factor and the bytes read fall with it.
+ * Everything else as lr_linear_chain (the descriptors' own active_rank fields
+ * are ignored); the workspace of lr_linear_chain_workspace_size suffices.
+ */
+LR_API lr_status_t lr_linear_chain_ranked(const lr_chain_step_t* steps, int n_steps, const lr_rank_vec_t* active,
+                                          const void* x, int batch, void* ws, size_t ws_bytes, lr_stream_t stream);
+
+/*
  * lr_linear without a caller-provided workspace (the pages have no
  * counterpart to this call; it exists for integration).
  *
@@ -220,6 +258,23 @@ LR_API lr_status_t lr_linear_chain_workspace_size(const lr_chain_step_t* steps, 
 #define LR_NOALLOC_SCRATCH_BYTES (1u << 20)
 LR_API lr_status_t lr_linear_noalloc(const lr_factor_desc_t* desc, const void* x, int batch, void* y,
                                      lr_stream_t stream);
+
+/*
+ * Dense linear, the uncompressed baseline of a factorised projection:
+ * y = x W for a weight stored output-major as W_store [d_out, d_in] (row k =
+ * output channel k, the layout of a framework's linear weight), bf16 or int8
+ * with one scale per output channel (y_k = (x . W_store[k]) * scale[k]).  The
+ * pages compare their factorised kernels against uncompressed execution
+ * (LASER results: decode speed-up over the uncompressed model; SAES-SVD:
+ * inference speed-up of the compressed model); this call is that reference
+ * on the same hardware.  Streams every weight byte once per 8 batch rows;
+ * no workspace.
+ *   W      [d_out, d_in] bf16 (scale NULL) or int8 (scale [d_out], LR_F16/LR_F32)
+ *   x      bf16 [batch, d_in] -> y bf16 [batch, d_out]
+ * Limits: d_in a multiple of 16 with d_in * element size <= 32 KiB.
+ */
+LR_API lr_status_t lr_dense_linear(const void* W, lr_dtype_t w_dtype, const void* scale, lr_dtype_t scale_dtype,
+                                   int d_in, int d_out, const void* x, int batch, void* y, lr_stream_t stream);
 
 /* ------------------------------------------------------------------------ */
 /* Hybrid SwiGLU FFN                                                        */
@@ -319,6 +374,33 @@ LR_API lr_status_t lr_latent_kv_decode(const lr_latent_kv_desc_t* desc, const vo
                                 size_t ws_bytes, lr_stream_t stream);
 
 LR_API lr_status_t lr_latent_kv_workspace_size(const lr_latent_kv_desc_t* desc, size_t* bytes);
+
+/*
+ * Standard single-query flash decoding over full K/V caches: the uncompressed
+ * baseline of the latent-KV path (WSVD "Resultaten" and LASER results report
+ * speed-ups over FlashDecoding).  out[b,h] = softmax((K q) * scale) V over the
+ * first seq_lens[b] positions, split over the context and merged with
+ * log-sum-exp rescaling.
+ *   q    bf16 [batch, heads, head_dim];  K, V bf16 [batch, heads, max_ctx, head_dim]
+ *   seq_lens int32 [batch] (device), clamped to [0, max_ctx]; 0 gives a zero row
+ *   out  bf16 [batch, heads, head_dim]
+ *   split_tokens  positions per split (multiple of 64, at most 256), 0 = library choice
+ * Supported: head_dim 128.  ws: lr_flash_decode_workspace_size bytes (fp32
+ * partials; no zero-fill needed).
+ */
+typedef struct lr_flash_desc {
+  int batch;
+  int heads;
+  int head_dim;
+  int max_ctx;
+  float scale;
+  int split_tokens;
+} lr_flash_desc_t;
+
+LR_API lr_status_t lr_flash_decode(const lr_flash_desc_t* desc, const void* q, const void* K, const void* V,
+                                   const int* seq_lens, void* out, void* ws, size_t ws_bytes, lr_stream_t stream);
+
+LR_API lr_status_t lr_flash_decode_workspace_size(const lr_flash_desc_t* desc, size_t* bytes);
 
 /* ------------------------------------------------------------------------ */
 /* W8A8 helpers                                                             */

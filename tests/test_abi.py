@@ -179,3 +179,57 @@ def test_noalloc_validation_order(lib):
 def test_wait_timeout_setter(lib):
     assert lib.lr_set_wait_timeout_us(500) == L.LR_OK
     assert lib.lr_set_wait_timeout_us(0) == L.LR_OK
+
+
+def test_rank_allocate_matches_oracle_exactly(lib):
+    # the library's FLRC rule on the host against the oracle, on random importances,
+    # budgets and caps (integer results: bit-exact)
+    import numpy as np
+
+    import decode_lr_linear_b200 as lr
+    from oracle import ranks
+    rng = np.random.default_rng(5)
+    for trial in range(200):
+        n = int(rng.integers(1, 130))
+        alpha = rng.lognormal(0.0, 0.6, n)
+        caps = rng.integers(1, 2000, n)
+        budget = float(rng.uniform(0, 3000 * n)) if trial % 7 else float(n) * 0.5
+        assert lr.lr_rank_allocate(alpha, budget, caps) == ranks.flrc_ranks(alpha, budget, caps).tolist()
+
+
+def test_rank_allocate_and_ranked_chain_validation(lib):
+    a = (ctypes.c_double * 2)(1.0, -1.0)
+    caps = (ctypes.c_int * 2)(10, 10)
+    cap = L.RankVec(2, caps)
+    out = (ctypes.c_int * 2)()
+    assert lib.lr_rank_allocate(a, 2, 10.0, ctypes.byref(cap), out) == L.LR_ERR_INVALID_ARG   # alpha <= 0
+    a = (ctypes.c_double * 2)(1.0, 1.0)
+    assert lib.lr_rank_allocate(a, 2, -1.0, ctypes.byref(cap), out) == L.LR_ERR_INVALID_ARG   # negative budget
+    bad_cap = L.RankVec(3, caps)
+    assert lib.lr_rank_allocate(a, 2, 10.0, ctypes.byref(bad_cap), out) == L.LR_ERR_INVALID_ARG
+    arr = (L.ChainStep * 2)(_step(3), _step(1, 0, 2))
+    r = (ctypes.c_int * 3)(100, 200, 300)
+    short = L.RankVec(3, r)                       # the chain has 4 projections
+    assert lib.lr_linear_chain_ranked(arr, 2, ctypes.byref(short), FAKE, 1, FAKE, 1 << 24, None) == \
+        L.LR_ERR_INVALID_ARG
+    r4 = (ctypes.c_int * 4)(100, 200, 2000, 5)    # 2000 > stored rank 1024
+    over = L.RankVec(4, r4)
+    assert lib.lr_linear_chain_ranked(arr, 2, ctypes.byref(over), FAKE, 1, FAKE, 1 << 24, None) == \
+        L.LR_ERR_INVALID_ARG
+
+
+def test_dense_and_flash_validation(lib):
+    assert lib.lr_dense_linear(FAKE, L.LR_F32, None, L.LR_F32, 4096, 4096, FAKE, 1, FAKE, None) == L.LR_ERR_UNSUPPORTED
+    assert lib.lr_dense_linear(FAKE, L.LR_I8, None, L.LR_F32, 4096, 4096, FAKE, 1, FAKE, None) == L.LR_ERR_INVALID_ARG
+    assert lib.lr_dense_linear(FAKE, L.LR_BF16, None, L.LR_F32, 4100, 4096, FAKE, 1, FAKE, None) == L.LR_ERR_UNSUPPORTED
+    assert lib.lr_dense_linear(FAKE, L.LR_BF16, None, L.LR_F32, 32768, 8, FAKE, 1, FAKE, None) == L.LR_ERR_UNSUPPORTED
+    assert lib.lr_dense_linear(MIS, L.LR_BF16, None, L.LR_F32, 4096, 8, FAKE, 1, FAKE, None) == L.LR_ERR_MISALIGNED
+    d = L.FlashDesc(8, 32, 128, 4096, 0.088, 0)
+    n = ctypes.c_size_t(0)
+    assert lib.lr_flash_decode_workspace_size(ctypes.byref(d), ctypes.byref(n)) == L.LR_OK
+    assert n.value == 8 * 32 * (4096 // 128) * 130 * 4
+    for bad, code in ((L.FlashDesc(8, 32, 64, 4096, 0.1, 0), L.LR_ERR_UNSUPPORTED),
+                      (L.FlashDesc(8, 32, 128, 4096, 0.1, 100), L.LR_ERR_INVALID_ARG),
+                      (L.FlashDesc(8, 32, 128, 4096, 0.1, 512), L.LR_ERR_INVALID_ARG)):
+        assert lib.lr_flash_decode(ctypes.byref(bad), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1 << 30, None) == code
+    assert lib.lr_flash_decode(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 16, None) == L.LR_ERR_WORKSPACE

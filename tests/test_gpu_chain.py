@@ -103,3 +103,33 @@ def test_chain_int8_and_fp32(cuda_device):
     r2 = lowrank.lr_linear(r1, d["At"].double().numpy().T, d["B32"].double().numpy())
     assert normwise_rel(outs[1][0], r2) < 1e-5
     assert lr.lr_check_device_error() == 0
+
+
+def test_ranked_chain_progressive_schedule(cuda_device, layers4):
+    # FLRC progressive decoding: per-token budgets, ranks from the library's
+    # allocation rule, applied to a 2-layer chain; every output against the
+    # oracle on factors truncated to the same ranks
+    from oracle import ranks as oranks
+    steps = _decode_stack_steps(layers4[:2])
+    caps = [layers4[l][n]["rank"] for l in range(2) for n in ("q", "k", "v", "o")]
+    alpha = np.random.default_rng(3).lognormal(0.0, 0.35, len(caps))
+    ws = lr.workspace(lr.lr_linear_chain_workspace_size(steps, 1), torch.device("cuda"))
+    for t, budget in enumerate((9000.0, 6000.0, 2500.0)):
+        active = lr.lr_rank_allocate(alpha, budget, caps)
+        assert active == oranks.flrc_ranks(alpha, budget, caps).tolist()
+        x = synth.make_activations(1, 4096, seed=10, key=(75, t))
+        outs = lr.lr_linear_chain_ranked(steps, dev(x), active, ws=ws)
+        x64, k = x.double().numpy(), 0
+        for l in range(2):
+            L_ = layers4[l]
+            ref = {}
+            for n in ("q", "k", "v"):
+                ref[n] = lowrank.lr_linear(x64, L_[n]["At"].double().numpy().T, L_[n]["B"].double().numpy(), active[k])
+                k += 1
+            ref["o"] = lowrank.lr_linear(ref["v"], L_["o"]["At"].double().numpy().T, L_["o"]["B"].double().numpy(),
+                                         active[k])
+            k += 1
+            for got, n in zip(outs[2 * l] + outs[2 * l + 1], ("q", "k", "v", "o")):
+                assert normwise_rel(got, ref[n]) < NORMWISE_TOL, (t, l, n)
+            x64 = ref["o"]
+    assert int(ws.count_nonzero()) == 0
