@@ -358,6 +358,30 @@ def make_latent_kv(batch: int = 8, heads: int = 32, ctx: int = 4096, rank: int =
             "scale": 1.0 / math.sqrt(head_dim)}
 
 
+def make_latent_kv_int8(batch: int = 8, heads: int = 32, ctx: int = 4096, rank: int = 32, head_dim: int = 128,
+                        seed: int = 0, seq_lens=None, scale_dtype=np.float16) -> dict:
+    """int8 latent caches with one positive scale per (batch, head, position): codes C_Kq, C_Vq
+    [batch, heads, ctx, rank] drawn as rint(N(0,1) * 127 / 4) clipped to +-127, scales s_K, s_V
+    [batch, heads, ctx] ~ 4/127 * U(0.5, 1.5) in ``scale_dtype``; B_K, B_V, q and seq_lens as
+    make_latent_kv (the decode's inputs, as a cache writer would have left them)."""
+    key = (6, ctx, batch, heads)
+    out = make_latent_kv(batch=batch, heads=heads, ctx=1, rank=rank, head_dim=head_dim, seed=seed)
+    for name, k in (("C_Kq", 0), ("C_Vq", 1)):
+        g = normals((batch, heads, ctx, rank), seed, key + (k,))
+        out[name] = torch.from_numpy(np.clip(np.rint(g * (127.0 / 4.0)), -127, 127).astype(np.int8))
+    for name, k in (("s_K", 2), ("s_V", 3)):
+        u = rng_for(seed, key + (k,)).uniform(0.5, 1.5, size=(batch, heads, ctx))
+        out[name] = torch.from_numpy((u * 4.0 / 127.0).astype(scale_dtype))
+    q = normals((batch, heads, head_dim), seed, key + (4,))
+    out["q"] = to_bf16(q)
+    if seq_lens is None:
+        seq_lens = np.full(batch, ctx, np.int32)
+    out["seq_lens"] = torch.as_tensor(np.asarray(seq_lens, np.int32))
+    out["ctx"] = ctx
+    del out["C_K"], out["C_V"]
+    return out
+
+
 # --------------------------------------------------------------------------
 # W8A8 prefill (LLaMA-13B shapes).
 # --------------------------------------------------------------------------

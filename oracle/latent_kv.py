@@ -76,3 +76,15 @@ def latent_kv_decode_absorbed(q, C_K, C_V, B_K, B_V, seq_lens, scale: float, pai
         out[b, h] = decode_head_absorbed(q[b, h], C_K[b, h], C_V[b, h], B_K[h], B_V[h],
                                          int(seq_lens[b]), scale)
     return out
+
+
+def dequantize_cache(Cq, s) -> np.ndarray:
+    """int8 latent cache with one scale per (batch, head, position): C[..., t, j] = Cq[..., t, j] * s[..., t]."""
+    return _f64(Cq) * _f64(s)[..., None]
+
+
+def latent_kv_decode_q8(q, CKq, sK, CVq, sV, B_K, B_V, seq_lens, scale: float, pairs=None) -> np.ndarray:
+    """Decode attention over int8 latent caches with per-token scales (LASER results:
+    the KV cache kept in 8 bits under W8A8): dequantize, then the reconstructed form."""
+    return latent_kv_decode(q, dequantize_cache(CKq, sK), dequantize_cache(CVq, sV), B_K, B_V, seq_lens, scale,
+                            pairs)

@@ -98,3 +98,30 @@ def test_identity_factors_reduce_to_sdpa():
                                          torch.from_numpy(CV), scale=scale)[:, :, 0]
     assert np.abs(o[..., :r] - ref.numpy()).max() < 1e-12
     assert np.abs(o[..., r:]).max() == 0.0
+
+
+def test_int8_cache_dequantization_and_invariants():
+    from decode_lr_linear_b200 import synth
+    d = synth.make_latent_kv_int8(batch=2, heads=2, ctx=40, seed=3, seq_lens=[40, 13])
+    # dequantization is the elementwise product with the per-position scale
+    from oracle import latent_kv
+    C = latent_kv.dequantize_cache(d["C_Kq"], d["s_K"])
+    t = 7
+    assert np.array_equal(C[1, 0, t], d["C_Kq"][1, 0, t].double().numpy() * float(d["s_K"][1, 0, t]))
+    o = latent_kv.latent_kv_decode_q8(d["q"], d["C_Kq"], d["s_K"], d["C_Vq"], d["s_V"], d["B_K"], d["B_V"],
+                                      d["seq_lens"], d["scale"])
+    # scaling every key scale by c and the query by 1/c leaves the scores unchanged
+    o2 = latent_kv.latent_kv_decode_q8(d["q"].double() / 8.0, d["C_Kq"], d["s_K"].double() * 8.0, d["C_Vq"],
+                                       d["s_V"], d["B_K"], d["B_V"], d["seq_lens"], d["scale"])
+    assert np.abs(o - o2).max() < 1e-12
+    # scaling every value scale by c scales the output by c
+    o3 = latent_kv.latent_kv_decode_q8(d["q"], d["C_Kq"], d["s_K"], d["C_Vq"], d["s_V"].double() * 3.0, d["B_K"],
+                                       d["B_V"], d["seq_lens"], d["scale"])
+    assert np.abs(o3 - 3.0 * o).max() < 1e-12
+    # brute force on one head, written out
+    b, h, n = 1, 1, 13
+    K = (d["C_Kq"][b, h, :n].double().numpy() * d["s_K"][b, h, :n].double().numpy()[:, None]) @ d["B_K"][h].double().numpy()
+    V = (d["C_Vq"][b, h, :n].double().numpy() * d["s_V"][b, h, :n].double().numpy()[:, None]) @ d["B_V"][h].double().numpy()
+    s = np.array([K[i] @ d["q"][b, h].double().numpy() for i in range(n)]) * d["scale"]
+    p = np.exp(s - s.max()) / np.exp(s - s.max()).sum()
+    assert np.abs(o[b, h] - sum(p[i] * V[i] for i in range(n))).max() < 1e-12
