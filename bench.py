@@ -31,6 +31,7 @@ of the low-rank path over each:
   c2dense   dense bf16 Q/K/V/O stack, 32 layers, batch 1
   c3dense   dense int8 SwiGLU FFN (all 11008 channels dense), batch 1
   c4full*   flash decoding over full K/V reconstructed from the same latents
+and  c4q8k*   the latent decode over int8 caches with per-position scales.
 
 `--impl reference` times the CPU oracle (the float64 reference
 implementation) on the headline workload instead, on the host cores.
@@ -57,7 +58,7 @@ LAYERS, HIDDEN = 32, 4096
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 ROW_IDS = ("c1", "c2b4", "c2b16", "c2dense", "c3b1", "c3b8", "c3b32", "c3dense", "c4k4", "c4k16", "c4k32",
-           "c4full4", "c4full16", "c4full32", "c5")
+           "c4full4", "c4full16", "c4full32", "c4q8k4", "c4q8k16", "c4q8k32", "c5")
 
 
 def parse(argv=None):
@@ -811,6 +812,50 @@ def row_c2dense(lr, L, synth, device, want_cpu):
     return row
 
 
+def row_c4q8(lr, L, synth, device, ctx, want_cpu):
+    """Latent-KV decode over int8 caches (one fp16 scale per position), batch 8, 32 heads, rank 32."""
+    import torch
+    from oracle import latent_kv as okv
+    d = synth.make_latent_kv_int8(batch=8, heads=32, ctx=ctx, seed=0)
+    cache_bytes = int(d["C_Kq"].numel() * 2 + d["s_K"].numel() * 2 * 2)
+    copies = max(1, math.ceil(4 * 126e6 / cache_bytes)) if cache_bytes < 4 * 126e6 else 1
+    kv = lr.LatentKv(8, 32, ctx, d["B_K"].to(device), d["B_V"].to(device), d["scale"])
+    caches = [tuple(d[k].to(device) for k in ("C_Kq", "s_K", "C_Vq", "s_V")) for _ in range(copies)]
+    q, sl = d["q"].to(device), d["seq_lens"].to(device)
+    o = torch.empty(8, 32, 128, dtype=torch.bfloat16, device=device)
+    ws = lr.workspace(lr.lr_latent_kv_workspace_size(kv), device)
+    ms = time_graph(lambda i: lr.lr_latent_kv_decode_q8(kv, q, *caches[i % copies][:2], *caches[i % copies][2:], sl,
+                                                        o, ws), 40)
+    alg = cache_bytes + int(d["B_K"].numel() * 2 * 2) + 2 * q.numel() * 2
+    lib, desc = L.load(), kv.desc(L.LR_F16)
+    qh, oh = d["q"].pin_memory(), torch.empty(8, 32, 128, dtype=torch.bfloat16).pin_memory()
+    CK, sK, CV, sV = caches[0]
+
+    def e2e():
+        q.copy_(qh, non_blocking=True)
+        L.check("lr_latent_kv_decode_q8", lib.lr_latent_kv_decode_q8(
+            ctypes.byref(desc), q.data_ptr(), CK.data_ptr(), sK.data_ptr(), CV.data_ptr(), sV.data_ptr(),
+            sl.data_ptr(), o.data_ptr(), ws.data_ptr(), ws.numel(), stream_ptr()))
+        oh.copy_(o, non_blocking=True)
+    ms_e2e = time_e2e(e2e, 40)
+    row = {"row": f"c4q8k{ctx // 1024}", "workload": f"latent-KV decode over int8 caches (fp16 scale per position), "
+                                                    f"batch 8, 32 heads, head_dim 128, rank 32, ctx {ctx}",
+           "value": ms * 1e3, "unit": "µs per call", "higher_is_better": False, "launches": 3,
+           "roofline": _roof_hbm(alg, ms, "q projection + split kernel (dominant) + combine kernel"),
+           "e2e": {"value": ms_e2e * 1e3, "unit": "µs per call", "h2d_bytes_per_step": int(q.numel() * 2),
+                   "d2h_bytes_per_step": int(o.numel() * 2), "path": "lr_latent_kv_decode_q8 through the C ABI"},
+           "l2": f"{copies} cache cop{'y' if copies == 1 else 'ies'} ({copies * cache_bytes / 1e6:.0f} MB > L2)"}
+    if want_cpu:
+        pairs = [(b, h) for b in range(0, 8, 2) for h in (0, 17)]
+        sec, n = cpu_timed(lambda: okv.latent_kv_decode_q8(d["q"], d["C_Kq"], d["s_K"], d["C_Vq"], d["s_V"], d["B_K"],
+                                                           d["B_V"], d["seq_lens"], d["scale"], pairs), 2.0, 10)
+        row["cpu_baseline"] = {"value": sec * 1e6 * 256 / len(pairs), "unit": "µs per call", "cores": host_cores(),
+                               "kind": "oracle", "sample": f"{n} call(s) of the float64 oracle on {len(pairs)} of "
+                                                          f"the 256 (batch, head) pairs, scaled to 256"}
+    del caches, ws
+    return row
+
+
 def row_c4full(lr, L, synth, device, ctx, want_cpu):
     """Flash decoding over full K/V reconstructed (bf16) from the latent caches of c4."""
     import torch
@@ -895,13 +940,17 @@ def run_rows(args, lr, L, synth, device, ranks, layers, only) -> list:
         elif rid.startswith("c4full"):
             rows.append(row_c4full(lr, L, synth, device, int(rid[6:]) * 1024, want_cpu))
             torch.cuda.empty_cache()
+        elif rid.startswith("c4q8k"):
+            rows.append(row_c4q8(lr, L, synth, device, int(rid[5:]) * 1024, want_cpu))
+            torch.cuda.empty_cache()
     if "c5" in sel:
         rows.append(row_c5(lr, L, synth, device, want_cpu))
     clk = clocks.stop()
     check_device(lr)
     by = {r["row"]: r for r in rows}
     # speed-up of each low-rank row over its uncompressed baseline (same work, same units)
-    for low, base in (("c3b1", "c3dense"), ("c4k4", "c4full4"), ("c4k16", "c4full16"), ("c4k32", "c4full32")):
+    for low, base in (("c3b1", "c3dense"), ("c4k4", "c4full4"), ("c4k16", "c4full16"), ("c4k32", "c4full32"),
+                      ("c4q8k4", "c4full4"), ("c4q8k16", "c4full16"), ("c4q8k32", "c4full32")):
         if low in by and base in by:
             by[low]["speedup_vs_uncompressed"] = by[base]["value"] / by[low]["value"]
     for r in rows:

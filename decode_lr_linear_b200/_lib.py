@@ -51,7 +51,7 @@ class FfnDesc(ctypes.Structure):
 class LatentKvDesc(ctypes.Structure):
     _fields_ = [("batch", c_int), ("heads", c_int), ("head_dim", c_int), ("rank", c_int), ("max_ctx", c_int),
                 ("scale", c_float), ("B_K", c_void_p), ("B_V", c_void_p), ("mode", c_int),
-                ("split_tokens", c_int)]
+                ("split_tokens", c_int), ("cache_scale_dtype", c_int)]
 
 
 class FlashDesc(ctypes.Structure):
@@ -78,6 +78,8 @@ _SIGNATURES = {
     "lr_latent_kv_decode": (c_int, [P(LatentKvDesc), c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                                     c_size_t, c_void_p]),
     "lr_latent_kv_workspace_size": (c_int, [P(LatentKvDesc), P(c_size_t)]),
+    "lr_latent_kv_decode_q8": (c_int, [P(LatentKvDesc), c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                                       c_void_p, c_void_p, c_size_t, c_void_p]),
     "lr_flash_decode": (c_int, [P(FlashDesc), c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_size_t,
                                 c_void_p]),
     "lr_flash_decode_workspace_size": (c_int, [P(FlashDesc), P(c_size_t)]),

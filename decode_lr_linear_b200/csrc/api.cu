@@ -536,23 +536,36 @@ static lr_status_t check_kv(const lr_latent_kv_desc_t* d, int* split) {
   return LR_OK;
 }
 
+// int8 caches: twice the positions per split keep 32 KiB of cache per CTA.
+static int kv_split_q8(const lr_latent_kv_desc_t* d, int t) { return d->split_tokens ? t : 2 * t; }
+
+static size_t kv_partial_bytes(const lr_latent_kv_desc_t* d, int t) {
+  const size_t ns = (size_t(d->max_ctx) + t - 1) / t;
+  return round_up(size_t(d->batch) * d->heads * ns * (d->rank + 2) * 4, 256);
+}
+
 lr_status_t lr_latent_kv_workspace_size(const lr_latent_kv_desc_t* d, size_t* bytes) {
   int t = 0;
   if (!bytes) return LR_ERR_INVALID_ARG;
   lr_status_t st = check_kv(d, &t);
   if (st != LR_OK) return st;
-  const size_t ns = (size_t(d->max_ctx) + t - 1) / t;
-  *bytes = size_t(d->batch) * d->heads * ns * (d->rank + 2) * 4;
+  *bytes = kv_partial_bytes(d, t) + size_t(d->batch) * d->heads * d->rank * 4;
   return LR_OK;
 }
 
-lr_status_t lr_latent_kv_decode(const lr_latent_kv_desc_t* d, const void* q, const void* C_K, const void* C_V,
-                                const int* seq_lens, void* out, void* ws, size_t ws_bytes, lr_stream_t stream) {
+static lr_status_t run_latent_kv(const lr_latent_kv_desc_t* d, const void* q, const void* C_K, const void* s_K,
+                                 const void* C_V, const void* s_V, bool q8, const int* seq_lens, void* out, void* ws,
+                                 size_t ws_bytes, lr_stream_t stream) {
   int t = 0;
   lr_status_t st = check_kv(d, &t);
   if (st != LR_OK) return st;
+  if (q8) t = kv_split_q8(d, t);  // fewer splits: the workspace sized for t suffices
   if (!q || !C_K || !C_V || !seq_lens || !out) return LR_ERR_INVALID_ARG;
   if (!al16(q) || !al16(C_K) || !al16(C_V) || !al16(seq_lens) || !al16(out)) return LR_ERR_MISALIGNED;
+  if (q8) {
+    if (!s_K || !s_V) return LR_ERR_INVALID_ARG;
+    if (d->cache_scale_dtype != LR_F16 && d->cache_scale_dtype != LR_F32) return LR_ERR_UNSUPPORTED;
+  }
   size_t need = 0;
   lr_latent_kv_workspace_size(d, &need);
   if (!ws || ws_bytes < need) return LR_ERR_WORKSPACE;
@@ -563,9 +576,24 @@ lr_status_t lr_latent_kv_decode(const lr_latent_kv_desc_t* d, const void* q, con
   P.split_tokens = t; P.n_splits = (d->max_ctx + t - 1) / t; P.scale = d->scale;
   P.q = q; P.CK = C_K; P.CV = C_V; P.BK = d->B_K; P.BV = d->B_V; P.seq_lens = seq_lens; P.out = out;
   P.partial = reinterpret_cast<float*>(ws);
+  P.qt = reinterpret_cast<float*>(reinterpret_cast<char*>(ws) + kv_partial_bytes(d, t));
   P.mode = d->mode;
+  P.cache_q8 = q8 ? 1 : 0;
+  P.cache_scale_f16 = d->cache_scale_dtype == LR_F16 ? 1 : 0;
+  P.sK = s_K; P.sV = s_V;
   P.err = device_error_word();
   return from_cuda(launch_latent_kv(P, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+lr_status_t lr_latent_kv_decode(const lr_latent_kv_desc_t* d, const void* q, const void* C_K, const void* C_V,
+                                const int* seq_lens, void* out, void* ws, size_t ws_bytes, lr_stream_t stream) {
+  return run_latent_kv(d, q, C_K, nullptr, C_V, nullptr, false, seq_lens, out, ws, ws_bytes, stream);
+}
+
+lr_status_t lr_latent_kv_decode_q8(const lr_latent_kv_desc_t* d, const void* q, const int8_t* C_K, const void* s_K,
+                                   const int8_t* C_V, const void* s_V, const int* seq_lens, void* out, void* ws,
+                                   size_t ws_bytes, lr_stream_t stream) {
+  return run_latent_kv(d, q, C_K, s_K, C_V, s_V, true, seq_lens, out, ws, ws_bytes, stream);
 }
 
 // --------------------------------------------------------------------------

@@ -101,7 +101,11 @@ struct LatentKvParams {
   const int* seq_lens;
   void* out;
   float* partial;     // [batch, heads, n_splits, rank + 2]
+  float* qt;          // [batch, heads, rank]: B_K q * scale * log2(e)
   int mode;
+  int cache_q8;       // 1: int8 caches with per-position scales sK, sV
+  int cache_scale_f16;
+  const void* sK; const void* sV;   // [batch, heads, max_ctx]
   int* err;           // device error word
 };
 

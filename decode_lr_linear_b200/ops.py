@@ -101,9 +101,9 @@ class LatentKv:
     def __post_init__(self):
         self.rank, self.head_dim = self.B_K.shape[1], self.B_K.shape[2]
 
-    def desc(self) -> L.LatentKvDesc:
+    def desc(self, cache_scale_dtype: int = L.LR_F16) -> L.LatentKvDesc:
         return L.LatentKvDesc(self.batch, self.heads, self.head_dim, self.rank, self.max_ctx, self.scale,
-                              _ptr(self.B_K), _ptr(self.B_V), self.mode, self.split_tokens)
+                              _ptr(self.B_K), _ptr(self.B_V), self.mode, self.split_tokens, cache_scale_dtype)
 
 
 def workspace(nbytes: int, device) -> torch.Tensor:
@@ -355,4 +355,20 @@ def lr_flash_decode(q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, seq_lens:
     L.check("lr_flash_decode", L.load().lr_flash_decode(ctypes.byref(d), _ptr(q), _ptr(K), _ptr(V), _ptr(seq_lens),
                                                         _ptr(out), _ptr(ws), ws.numel() * ws.element_size(),
                                                         _stream(stream)))
+    return out
+
+
+def lr_latent_kv_decode_q8(kv: LatentKv, q: torch.Tensor, C_K: torch.Tensor, s_K: torch.Tensor, C_V: torch.Tensor,
+                           s_V: torch.Tensor, seq_lens: torch.Tensor, out: Optional[torch.Tensor] = None,
+                           ws: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Latent-KV decode over int8 caches with one scale per (batch, head, position)."""
+    if out is None:
+        out = torch.empty(kv.batch, kv.heads, kv.head_dim, dtype=torch.bfloat16, device=q.device)
+    if ws is None:
+        ws = workspace(lr_latent_kv_workspace_size(kv), q.device)
+    d = kv.desc(_DT[s_K.dtype])
+    L.check("lr_latent_kv_decode_q8",
+            L.load().lr_latent_kv_decode_q8(ctypes.byref(d), _ptr(q), _ptr(C_K), _ptr(s_K), _ptr(C_V), _ptr(s_V),
+                                            _ptr(seq_lens), _ptr(out), _ptr(ws), ws.numel() * ws.element_size(),
+                                            _stream(stream)))
     return out

@@ -360,6 +360,7 @@ typedef struct lr_latent_kv_desc {
   const void* B_V;
   int mode;
   int split_tokens;
+  lr_dtype_t cache_scale_dtype;  /* lr_latent_kv_decode_q8 only: LR_F16 or LR_F32 */
 } lr_latent_kv_desc_t;
 
 /*
@@ -374,6 +375,20 @@ LR_API lr_status_t lr_latent_kv_decode(const lr_latent_kv_desc_t* desc, const vo
                                 size_t ws_bytes, lr_stream_t stream);
 
 LR_API lr_status_t lr_latent_kv_workspace_size(const lr_latent_kv_desc_t* desc, size_t* bytes);
+
+/*
+ * The same decode over int8 latent caches (LASER results: under W8A8 the KV
+ * cache is kept in 8 bits), half the cache bytes of bf16:
+ *   C_K, C_V  int8 [batch, heads, max_ctx, rank] codes
+ *   s_K, s_V  [batch, heads, max_ctx] one scale per cached position
+ *             (desc->cache_scale_dtype: LR_F16 or LR_F32)
+ * C[t, j] = code[t, j] * s[t]; the key scale multiplies the token's score,
+ * the value scale its softmax weight.  Everything else as lr_latent_kv_decode
+ * (same workspace size).
+ */
+LR_API lr_status_t lr_latent_kv_decode_q8(const lr_latent_kv_desc_t* desc, const void* q, const int8_t* C_K,
+                                          const void* s_K, const int8_t* C_V, const void* s_V, const int* seq_lens,
+                                          void* out, void* ws, size_t ws_bytes, lr_stream_t stream);
 
 /*
  * Standard single-query flash decoding over full K/V caches: the uncompressed

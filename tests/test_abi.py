@@ -116,7 +116,7 @@ def test_ffn_validation_and_workspace(lib):
 
 def _kv(**kw):
     d = dict(batch=8, heads=32, head_dim=128, rank=32, max_ctx=4096, scale=128 ** -0.5, B_K=FAKE, B_V=FAKE,
-             mode=L.LR_KV_ABSORBED, split_tokens=0)
+             mode=L.LR_KV_ABSORBED, split_tokens=0, cache_scale_dtype=L.LR_F16)
     d.update(kw)
     return L.LatentKvDesc(**d)
 
@@ -125,7 +125,7 @@ def test_latent_kv_validation_and_workspace(lib):
     n = ctypes.c_size_t(0)
     d = _kv()
     assert lib.lr_latent_kv_workspace_size(ctypes.byref(d), ctypes.byref(n)) == L.LR_OK
-    assert n.value == 8 * 32 * (4096 // 256) * 34 * 4
+    assert n.value == 8 * 32 * (4096 // 256) * 34 * 4 + 8 * 32 * 32 * 4   # partials + the projected queries
     for bad, code in ((_kv(rank=16), L.LR_ERR_UNSUPPORTED), (_kv(head_dim=64), L.LR_ERR_UNSUPPORTED),
                       (_kv(split_tokens=100), L.LR_ERR_INVALID_ARG), (_kv(batch=0), L.LR_ERR_INVALID_ARG),
                       (_kv(B_K=MIS), L.LR_ERR_MISALIGNED)):
@@ -233,3 +233,14 @@ def test_dense_and_flash_validation(lib):
                       (L.FlashDesc(8, 32, 128, 4096, 0.1, 512), L.LR_ERR_INVALID_ARG)):
         assert lib.lr_flash_decode(ctypes.byref(bad), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1 << 30, None) == code
     assert lib.lr_flash_decode(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 16, None) == L.LR_ERR_WORKSPACE
+
+
+def test_latent_kv_q8_validation(lib):
+    d = _kv()
+    assert lib.lr_latent_kv_decode_q8(ctypes.byref(d), FAKE, FAKE, None, FAKE, FAKE, FAKE, FAKE, FAKE, 1 << 30,
+                                      None) == L.LR_ERR_INVALID_ARG
+    bad = _kv(cache_scale_dtype=L.LR_BF16)
+    assert lib.lr_latent_kv_decode_q8(ctypes.byref(bad), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1 << 30,
+                                      None) == L.LR_ERR_UNSUPPORTED
+    assert lib.lr_latent_kv_decode_q8(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 16,
+                                      None) == L.LR_ERR_WORKSPACE

@@ -113,3 +113,39 @@ def test_quantize_zero_row_and_ties(cuda_device):
     assert np.array_equal(xq.cpu().numpy(), q_ref) and np.array_equal(s.cpu().numpy(), s_ref)
     assert s[0].item() == 1.0 and int(xq[0].abs().max()) == 0
 
+
+
+def _kv8_run(d, split=0):
+    kv = lr.LatentKv(d["q"].shape[0], d["q"].shape[1], d["ctx"], dev(d["B_K"]), dev(d["B_V"]), d["scale"], 0, split)
+    return lr.lr_latent_kv_decode_q8(kv, dev(d["q"]), dev(d["C_Kq"]), dev(d["s_K"]), dev(d["C_Vq"]), dev(d["s_V"]),
+                                     dev(d["seq_lens"]))
+
+
+def _kv8_oracle(d, pairs=None):
+    return okv.latent_kv_decode_q8(d["q"], d["C_Kq"], d["s_K"], d["C_Vq"], d["s_V"], d["B_K"], d["B_V"],
+                                   d["seq_lens"], d["scale"], pairs)
+
+
+@pytest.mark.parametrize("split,scale_dtype", [(0, np.float16), (64, np.float32), (512, np.float16)])
+def test_latent_kv_int8_ragged_all_pairs(cuda_device, split, scale_dtype):
+    seq = [1, 63, 64, 65, 300, 1000, 0, 777]
+    d = synth.make_latent_kv_int8(batch=8, heads=4, ctx=1000, seed=13, seq_lens=seq, scale_dtype=scale_dtype)
+    o = _kv8_run(d, split).float().cpu().numpy()
+    ref = _kv8_oracle(d)
+    for b in range(8):
+        if seq[b] == 0:
+            assert np.abs(o[b]).max() == 0.0
+            continue
+        assert normwise_rel(o[b], ref[b]) < NORMWISE_TOL, (b, seq[b])
+
+
+def test_latent_kv_int8_full_size_sampled(cuda_device):
+    d = synth.make_latent_kv_int8(batch=8, heads=32, ctx=16384, seed=0)
+    o = _kv8_run(d).float().cpu().numpy()
+    rng = np.random.default_rng(16384)
+    pairs = [(int(b), int(h)) for b, h in zip(rng.integers(0, 8, 12), rng.integers(0, 32, 12))]
+    ref = _kv8_oracle(d, pairs)
+    for b, h in pairs:
+        assert normwise_rel(o[b, h][None], ref[b, h][None]) < NORMWISE_TOL, (b, h)
+    assert np.isfinite(o).all()
+    assert lr.lr_check_device_error() == 0
