@@ -159,9 +159,11 @@ def int8_peak_tops():
 # figure is dropped, as null, as soon as the kernel changes).  Filled from
 # the profiles of the current sources.
 TRAFFIC_RECORDS = {
-    # "chain_kernel<bf16,1,1>": {"sources_sha1": "...", "per_alg_byte": 1.0},
+    # ncu dram__bytes_read.sum + dram__bytes_write.sum of one launch of the first 2 layers of the
+    # stack (bench.py --layers 2): 159,678,976 bytes for 159,481,856 algorithmic bytes
+    "chain_kernel<bf16,1,1>": {"sources_sha1": "3e0d40c7a871cf50ce720457e1441a2f329a0831", "per_alg_byte": 159678976 / 159481856},
 }
-KERNEL_SOURCES = {"chain_kernel<bf16,1,1>": ("chain.cu", "common.cuh", "internal.h")}
+KERNEL_SOURCES = {"chain_kernel<bf16,1,1>": ("chain.cu", "common.cuh")}
 
 
 def sources_sha1(files) -> str:
