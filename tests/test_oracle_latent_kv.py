@@ -125,3 +125,129 @@ def test_int8_cache_dequantization_and_invariants():
     s = np.array([K[i] @ d["q"][b, h].double().numpy() for i in range(n)]) * d["scale"]
     p = np.exp(s - s.max()) / np.exp(s - s.max()).sum()
     assert np.abs(o[b, h] - sum(p[i] * V[i] for i in range(n))).max() < 1e-12
+
+
+# ---- rotary positions, the reconstruct-on-chip form and the producer -------
+def test_rope_matches_complex_rotation():
+    # RoFormer's complex form: pair (x_i, x_{i+h}) as x_i + i x_{i+h}, multiplied by e^{i pos theta_i}
+    rng = np.random.default_rng(10)
+    x = rng.standard_normal((5, 16))
+    pos = np.array([0, 1, 7, 1000, 32767])
+    base = 10000.0
+    theta = base ** (-np.arange(8) * 2.0 / 16.0)
+    z = (x[:, :8] + 1j * x[:, 8:]) * np.exp(1j * pos[:, None] * theta[None, :])
+    want = np.concatenate([z.real, z.imag], axis=1)
+    assert np.abs(O.rope(x, pos, base) - want).max() < 1e-12
+    assert np.abs(O.rope(x[:1], 0, base) - x[:1]).max() == 0.0          # position 0: identity
+    assert np.allclose(np.linalg.norm(O.rope(x, pos, base), axis=1), np.linalg.norm(x, axis=1))
+
+
+def test_rope_matches_llama_library_routine():
+    from transformers.models.llama.modeling_llama import apply_rotary_pos_emb
+    rng = np.random.default_rng(11)
+    hd, L, base = 128, 40, 10000.0
+    q = torch.from_numpy(rng.standard_normal((1, 1, L, hd)))
+    k = torch.from_numpy(rng.standard_normal((1, 1, L, hd)))
+    inv = 1.0 / (base ** (torch.arange(0, hd, 2, dtype=torch.float64) / hd))
+    ang = torch.arange(L, dtype=torch.float64)[:, None] * inv[None, :]
+    emb = torch.cat([ang, ang], dim=-1)
+    qr, kr = apply_rotary_pos_emb(q, k, emb.cos()[None], emb.sin()[None])
+    pos = np.arange(L)
+    assert np.abs(O.rope(q[0, 0].numpy(), pos, base) - qr[0, 0].numpy()).max() < 1e-12
+    assert np.abs(O.rope(k[0, 0].numpy(), pos, base) - kr[0, 0].numpy()).max() < 1e-12
+
+
+def test_rope_scores_depend_on_relative_position_only():
+    rng = np.random.default_rng(12)
+    q, k = rng.standard_normal(64), rng.standard_normal(64)
+    for a, b, c in ((3, 10, 5), (100, 7, 4000), (0, 0, 31)):
+        s1 = O.rope(q, a, 500.0) @ O.rope(k, b, 500.0)
+        s2 = O.rope(q, a + c, 500.0) @ O.rope(k, b + c, 500.0)
+        assert abs(s1 - s2) < 1e-9
+
+
+def _brute_rope(q, CK, CV, BK, BV, seq_lens, scale, base):
+    nb, nh, hd = q.shape
+    r, half = CK.shape[-1], hd // 2
+    out = np.zeros((nb, nh, hd))
+
+    def rot(v, pos):
+        w = [0.0] * hd
+        for i in range(half):
+            a = pos * base ** (-2.0 * i / hd)
+            w[i] = v[i] * math.cos(a) - v[i + half] * math.sin(a)
+            w[i + half] = v[i + half] * math.cos(a) + v[i] * math.sin(a)
+        return w
+
+    for b in range(nb):
+        for h in range(nh):
+            n = int(seq_lens[b])
+            if n == 0:
+                continue
+            qr = rot(list(q[b, h]), n - 1)
+            s = []
+            for t in range(n):
+                kt = rot([sum(CK[b, h, t, j] * BK[h, j, d] for j in range(r)) for d in range(hd)], t)
+                s.append(scale * sum(qr[d] * kt[d] for d in range(hd)))
+            m = max(s)
+            w = [math.exp(v - m) for v in s]
+            tot = sum(w)
+            for d in range(hd):
+                out[b, h, d] = sum(w[t] / tot * sum(CV[b, h, t, j] * BV[h, j, d] for j in range(r))
+                                   for t in range(n))
+    return out
+
+
+def test_rope_decode_brute_force_ragged():
+    rng = np.random.default_rng(13)
+    q, CK, CV, BK, BV = _case(rng, nb=3, nh=2, L=11, r=3, hd=6)
+    seq = np.array([11, 4, 0])
+    ref = _brute_rope(q, CK, CV, BK, BV, seq, 0.41, 50.0)
+    got = O.latent_kv_decode_rope(q, CK, CV, BK, BV, seq, 0.41, 50.0)
+    assert np.abs(got - ref).max() < 1e-12
+    assert np.all(got[2] == 0.0)
+
+
+def test_rope_decode_special_cases():
+    rng = np.random.default_rng(14)
+    q, CK, CV, BK, BV = _case(rng, nb=2, nh=2, L=6, r=4, hd=8)
+    # one cached token: query and key both at position 0, no rotation; output V_0
+    one = np.array([1, 1])
+    assert np.abs(O.latent_kv_decode_rope(q, CK, CV, BK, BV, one, 0.3, 10000.0)
+                  - O.latent_kv_decode(q, CK, CV, BK, BV, one, 0.3)).max() < 1e-12
+    # rotation changes the scores of a longer context (the absorbed form is not exact any more)
+    full = np.array([6, 6])
+    d = np.abs(O.latent_kv_decode_rope(q, CK, CV, BK, BV, full, 0.3, 10.0)
+               - O.latent_kv_decode(q, CK, CV, BK, BV, full, 0.3)).max()
+    assert d > 1e-3
+    # keys rotated explicitly, then the unrotated oracle on a cache whose factor is the identity
+    b, h, n, base = 0, 1, 6, 10.0
+    K = O.rope(CK[b, h, :n] @ BK[h], np.arange(n), base)
+    qr = O.rope(q[b, h], n - 1, base)
+    ref = O.decode_head(qr, K, CV[b, h, :n], np.eye(8), BV[h], n, 0.3)
+    assert np.abs(O.decode_head_rope(q[b, h], CK[b, h], CV[b, h], BK[h], BV[h], n, 0.3, base) - ref).max() < 1e-12
+
+
+def test_append_latents_brute_force_and_exact_rank_key():
+    rng = np.random.default_rng(15)
+    nb, nh, r, hidden, ctx, hd = 3, 2, 3, 10, 5, 4
+    x = rng.standard_normal((nb, hidden))
+    A = rng.standard_normal((2 * nh * r, hidden))
+    CK, CV = rng.standard_normal((nb, nh, ctx, r)), rng.standard_normal((nb, nh, ctx, r))
+    pos = np.array([2, 4, 5])                     # the last one is outside the cache: unchanged
+    ck, cv = O.append_latents(x, A, nh, r, CK, CV, pos)
+    for b in range(nb):
+        for h in range(nh):
+            for t in range(ctx):
+                for j in range(r):
+                    if t == pos[b]:
+                        wk = sum(x[b, i] * A[h * r + j, i] for i in range(hidden))
+                        wv = sum(x[b, i] * A[(nh + h) * r + j, i] for i in range(hidden))
+                    else:
+                        wk, wv = CK[b, h, t, j], CV[b, h, t, j]
+                    assert abs(ck[b, h, t, j] - wk) < 1e-12 and abs(cv[b, h, t, j] - wv) < 1e-12
+    # the appended latent reconstructs the key of the exactly-rank-r per-head projection W_Kh = A_Kh B_Kh
+    BK = rng.standard_normal((nh, r, hd))
+    for h in range(nh):
+        W = A[h * r:(h + 1) * r].T @ BK[h]         # hidden x head_dim
+        assert np.abs(ck[0, h, pos[0]] @ BK[h] - x[0] @ W).max() < 1e-12
