@@ -7,8 +7,8 @@ stack of 32 layers whose Q/K/V/O projections are truncated-SVD factorised
 reduction, batch 1).  Per layer, Q, K and V are computed from the layer input
 x; the O projection reads the V output (single-token attention returns V
 exactly) and its output is the next layer's input.  The whole stack is one
-lr_linear_chain call: one persistent launch per step, in which each
-projection waits only for the projection it reads.
+lr_linear_chain call, one persistent launch per step, of three chain steps per
+layer (V; Q and K; O), each waiting only for the step it reads.
 
 The 32 layers hold 2.58 GB of factors, far above the 126 MB L2, so every step
 streams them from HBM (no L2 flush needed).  Timing: W untimed warm-up steps,
@@ -31,7 +31,10 @@ of the low-rank path over each:
   c2dense   dense bf16 Q/K/V/O stack, 32 layers, batch 1
   c3dense   dense int8 SwiGLU FFN (all 11008 channels dense), batch 1
   c4full*   flash decoding over full K/V reconstructed from the same latents
-and  c4q8k*   the latent decode over int8 caches with per-position scales.
+and  c4q8k*   the latent decode over int8 caches with per-position scales,
+     c4rk*    the latent decode with keys reconstructed on the tensor cores and
+              rotated (rotary base 10000), ctx 4K/16K/32K,
+     c4app    the latent producer writing one token's per-head latents.
 
 `--impl reference` times the CPU oracle (the float64 reference
 implementation) on the headline workload instead, on the host cores.
@@ -57,8 +60,10 @@ METRIC = "decode-layer µs & achieved HBM GB/s (% of B200 roofline) at batch 1; 
 LAYERS, HIDDEN = 32, 4096
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
+TC_MIN = [9, 9]   # smallest batch on the tensor-core path (linears, FFN): the library's default
 ROW_IDS = ("c1", "c2b4", "c2b16", "c2dense", "c3b1", "c3b8", "c3b32", "c3dense", "c4k4", "c4k16", "c4k32",
-           "c4full4", "c4full16", "c4full32", "c4q8k4", "c4q8k16", "c4q8k32", "c5")
+           "c4rk4", "c4rk16", "c4rk32", "c4app", "c4full4", "c4full16", "c4full32", "c4q8k4", "c4q8k16", "c4q8k32",
+           "c5")
 
 
 def parse(argv=None):
@@ -73,6 +78,8 @@ def parse(argv=None):
     ap.add_argument("--only", default="", help="comma list of row ids to run (" + ",".join(ROW_IDS) + ")")
     ap.add_argument("--layers", type=int, default=LAYERS,
                     help="layers in the stack (default 32; fewer only for profiling small cases)")
+    ap.add_argument("--tc-min-batch", default="",
+                    help="LINEAR,FFN: smallest batch on the tensor-core path (lr_set_tensor_core_min_batch)")
     return ap.parse_args(argv)
 
 
@@ -330,15 +337,26 @@ def build_layers(device, layers: int):
     return ranks, out
 
 
-def stack_steps(lr, layers, batch, device):
-    """The decode stack as one chain: step 2l = Q/K/V of layer l (input: the previous O), step 2l+1 = O (input: V)."""
+def stack_steps(lr, layers, batch, device, split_v: bool = True):
+    """The decode stack as one chain.  split_v (the CUDA-core path, one persistent launch): three
+    steps per layer, V (input: the previous O), then Q and K (same input), then O (input: V); O waits
+    only for V, so Q and K stream while V's result is handed over, and the next layer's V waits for
+    O.  Otherwise (the tensor-core path, a sequence of launches): Q/K/V in one step, then O."""
     import torch
+
+    def out():
+        return torch.empty(batch, HIDDEN, dtype=torch.bfloat16, device=device)
     steps = []
     for l, L in enumerate(layers):
-        qkv = [torch.empty(batch, HIDDEN, dtype=torch.bfloat16, device=device) for _ in range(3)]
-        steps.append(lr.ChainStep([L["q"], L["k"], L["v"]], -1 if l == 0 else 2 * l - 1, 0, qkv))
-        steps.append(lr.ChainStep([L["o"]], 2 * l, 2,
-                                  [torch.empty(batch, HIDDEN, dtype=torch.bfloat16, device=device)]))
+        if split_v:
+            src = -1 if l == 0 else 3 * l - 1
+            steps.append(lr.ChainStep([L["v"]], src, 0, [out()]))
+            steps.append(lr.ChainStep([L["q"], L["k"]], src, 0, [out(), out()]))
+            steps.append(lr.ChainStep([L["o"]], 3 * l, 0, [out()]))
+        else:
+            steps.append(lr.ChainStep([L["q"], L["k"], L["v"]], -1 if l == 0 else 2 * l - 1, 0,
+                                      [out(), out(), out()]))
+            steps.append(lr.ChainStep([L["o"]], 2 * l, 2, [out()]))
     return steps
 
 
@@ -391,6 +409,10 @@ def run_ours(args) -> None:
     torch.cuda.set_device(device)
     dist_init("nccl")
     batch = args.batch
+    if args.tc_min_batch:
+        lin, ffn = (int(v) for v in args.tc_min_batch.split(","))
+        lr.lr_set_tensor_core_min_batch(lin, ffn)
+        TC_MIN[0], TC_MIN[1] = lin or 9, ffn or 9
     only = set(filter(None, args.only.split(",")))
     want_headline = not only or "headline" in only
     want_cpu = rank == 0 and world == 1 and not args.no_cpu_baseline
@@ -399,7 +421,7 @@ def run_ours(args) -> None:
     out = None
     if want_headline:
         x0 = synth.make_activations(batch, HIDDEN, seed=0, key=(90,)).to(device)
-        steps = stack_steps(lr, layers, batch, device)
+        steps = stack_steps(lr, layers, batch, device, split_v=batch < TC_MIN[0])
         ws = lr.workspace(lr.lr_linear_chain_workspace_size(steps, batch), device)
 
         def step():
@@ -556,12 +578,17 @@ def row_c1(lr, L, synth, device, want_cpu):
 
 def row_c2(lr, L, synth, device, ranks, layers, batch, want_cpu):
     import torch
-    steps = stack_steps(lr, layers, batch, device)
+    steps = stack_steps(lr, layers, batch, device, split_v=batch < TC_MIN[0])
     ws = lr.workspace(lr.lr_linear_chain_workspace_size(steps, batch), device)
     x0 = synth.make_activations(batch, HIDDEN, seed=0, key=(90, batch)).to(device)
     ms = time_graph(lambda i: lr.lr_linear_chain(steps, x0, ws=ws), 20)
     alg = algorithmic_bytes_per_step(ranks, batch, LAYERS)
-    launches = (batch + 7) // 8
+    passes = (batch + 31) // 32
+    tensor_cores = batch >= TC_MIN[0]
+    launches = passes * (3 * len(steps) + 1) if tensor_cores else (batch + 7) // 8
+    note = (f"{launches} launches per step: per dependent step two tcgen05 products (z = x A, y = z B, weights "
+            f"as M, tokens as N) and a finalize; every factor byte streamed once per pass of 32 tokens"
+            if tensor_cores else f"{launches} launch(es) of chain_kernel per step; each streams every factor byte once")
     arr, lib = lr.ops._chain_array(steps), L.load()
     xh = synth.make_activations(batch, HIDDEN, seed=0, key=(90, batch)).pin_memory()
     yh = torch.empty(batch, HIDDEN, dtype=torch.bfloat16).pin_memory()
@@ -575,8 +602,7 @@ def row_c2(lr, L, synth, device, ranks, layers, batch, want_cpu):
     row = {"row": f"c2b{batch}", "workload": f"llama7b-lowrank-qkvo-decode, 32 layers, batch {batch}",
            "value": batch / (ms * 1e-3), "unit": "tokens/s", "higher_is_better": True,
            "ms_per_step": ms, "layer_us": ms * 1e3 / LAYERS, "launches": launches,
-           "roofline": _roof_hbm(alg, ms, f"{launches} launch(es) of chain_kernel per step; each streams every "
-                                          f"factor byte once"),
+           "roofline": _roof_hbm(alg, ms, note),
            "e2e": {"value": batch / (ms_e2e * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": batch * HIDDEN * 2,
                    "d2h_bytes_per_step": batch * HIDDEN * 2, "path": "lr_linear_chain through the C ABI"},
            "l2": "2.58 GB of factors streamed per step"}
@@ -611,13 +637,19 @@ def row_c3(lr, L, synth, device, d, batch, want_cpu):
                                                    ws.data_ptr(), ws.numel(), stream_ptr()))
         yh.copy_(y, non_blocking=True)
     ms_e2e = time_e2e(e2e, 40)
-    pieces = math.ceil(batch / 2)
+    if batch >= TC_MIN[1]:
+        passes = math.ceil(batch / 32)
+        pieces = passes * (5 if d["n_lr"] > 0 else 4)
+        note = (f"{pieces} launches: tcgen05 kind::i8 products (x A' with x D, B'^T z, W_down^T h), SwiGLU, finalize; "
+                f"every weight byte streamed once per pass of 32 tokens")
+    else:
+        pieces = math.ceil(batch / 2) + math.ceil(batch / 4)
+        note = f"{pieces} launch(es) of the CUDA-core decode engine, each streaming its phase's weight bytes"
     row = {"row": f"c3b{batch}", "workload": f"hybrid int8 SwiGLU FFN, 7B shapes (hidden 4096, inter 11008, "
                                              f"n_lr 8192, rank 1536), batch {batch}",
            "value": ms * 1e3, "unit": "µs per layer", "higher_is_better": False,
            "tokens_s_32_layers": batch / (ms * 1e-3 * 32), "launches": pieces,
-           "roofline": _roof_hbm(alg, ms, f"{pieces} launch(es) of the decode engine (2 batch rows each), each "
-                                          f"streaming every weight byte"),
+           "roofline": _roof_hbm(alg, ms, note),
            "e2e": {"value": ms_e2e * 1e3, "unit": "µs per layer", "h2d_bytes_per_step": batch * d["hidden"] * 2,
                    "d2h_bytes_per_step": batch * d["hidden"] * 2, "path": "lr_swiglu_ffn through the C ABI"},
            "l2": f"{copies} weight copies rotate ({copies * w_bytes / 1e6:.0f} MB > L2)"}
@@ -632,13 +664,17 @@ def row_c3(lr, L, synth, device, d, batch, want_cpu):
     return row
 
 
-def row_c4(lr, L, synth, device, ctx, want_cpu):
+def row_c4(lr, L, synth, device, ctx, want_cpu, rope_base: float = 0.0):
+    """Latent-KV decode, batch 8, 32 heads, rank 32: the absorbed form, or (rope_base > 0) keys
+    reconstructed on the tensor cores and rotated (LR_KV_RECONSTRUCT)."""
     import torch
     from oracle import latent_kv as okv
     kvd = synth.make_latent_kv(batch=8, heads=32, ctx=ctx, seed=0)
     cache_bytes = int(kvd["C_K"].numel() * 2 * 2)
     copies = max(1, math.ceil(4 * 126e6 / cache_bytes)) if cache_bytes < 4 * 126e6 else 1
-    kv = lr.LatentKv(8, 32, ctx, kvd["B_K"].to(device), kvd["B_V"].to(device), kvd["scale"])
+    rec = rope_base > 0
+    kv = lr.LatentKv(8, 32, ctx, kvd["B_K"].to(device), kvd["B_V"].to(device), kvd["scale"],
+                     L.LR_KV_RECONSTRUCT if rec else L.LR_KV_ABSORBED, 0, rope_base)
     caches = [(kvd["C_K"].to(device), kvd["C_V"].to(device)) for _ in range(copies)]
     q, sl = kvd["q"].to(device), kvd["seq_lens"].to(device)
     o = torch.empty(8, 32, 128, dtype=torch.bfloat16, device=device)
@@ -657,19 +693,27 @@ def row_c4(lr, L, synth, device, ctx, want_cpu):
                                                                ws.data_ptr(), ws.numel(), stream_ptr()))
         oh.copy_(o, non_blocking=True)
     ms_e2e = time_e2e(e2e, 40)
-    row = {"row": f"c4k{ctx // 1024}", "workload": f"per-head latent-KV flash decoding, batch 8, 32 heads, "
-                                                  f"head_dim 128, rank 32, ctx {ctx} (absorbed form)",
+    form = (f"keys reconstructed on the tensor cores, rotary base {rope_base:g}" if rec else "absorbed form")
+    row = {"row": f"c4{'r' if rec else ''}k{ctx // 1024}",
+           "workload": f"per-head latent-KV flash decoding, batch 8, 32 heads, head_dim 128, rank 32, ctx {ctx} "
+                       f"({form})",
            "value": ms * 1e3, "unit": "µs per call", "higher_is_better": False,
-           "tokens_s_32_layers": 8 / (ms * 1e-3 * 32), "launches": 2,
-           "roofline": _roof_hbm(alg, ms, "split kernel (dominant) + combine kernel"),
+           "tokens_s_32_layers": 8 / (ms * 1e-3 * 32), "launches": 2 if rec else 3,
+           "roofline": _roof_hbm(alg, ms, ("reconstruct-and-rotate split kernel (dominant) + combine kernel" if rec
+                                           else "q projection + split kernel (dominant) + combine kernel")),
            "e2e": {"value": ms_e2e * 1e3, "unit": "µs per call", "h2d_bytes_per_step": int(q.numel() * 2),
                    "d2h_bytes_per_step": int(o.numel() * 2),
                    "path": "lr_latent_kv_decode through the C ABI (the caches stay resident, as a KV cache does)"},
            "l2": f"{copies} cache cop{'y' if copies == 1 else 'ies'} ({copies * cache_bytes / 1e6:.0f} MB > L2)"}
     if want_cpu:
         pairs = [(b, h) for b in range(0, 8, 2) for h in (0, 17)]
-        s, n = cpu_timed(lambda: okv.latent_kv_decode(kvd["q"], kvd["C_K"], kvd["C_V"], kvd["B_K"], kvd["B_V"],
-                                                      kvd["seq_lens"], kvd["scale"], pairs), 2.0, 10)
+        if rec:
+            s, n = cpu_timed(lambda: okv.latent_kv_decode_rope(kvd["q"], kvd["C_K"], kvd["C_V"], kvd["B_K"],
+                                                               kvd["B_V"], kvd["seq_lens"], kvd["scale"], rope_base,
+                                                               pairs), 2.0, 10)
+        else:
+            s, n = cpu_timed(lambda: okv.latent_kv_decode(kvd["q"], kvd["C_K"], kvd["C_V"], kvd["B_K"], kvd["B_V"],
+                                                          kvd["seq_lens"], kvd["scale"], pairs), 2.0, 10)
         row["cpu_baseline"] = {"value": s * 1e6 * 256 / len(pairs), "unit": "µs per call", "cores": host_cores(),
                                "kind": "oracle",
                                "sample": f"{n} call(s) of the float64 oracle on {len(pairs)} of the 256 (batch, head) "
@@ -814,6 +858,51 @@ def row_c2dense(lr, L, synth, device, want_cpu):
     return row
 
 
+def row_c4app(lr, L, synth, device, want_cpu):
+    """The latent producer: one decode token of batch 8 writes its per-head key and value latents
+    (32 heads, rank 32, hidden 4096) into the caches; weights of 32 layers rotate."""
+    import torch
+    from oracle import latent_kv as okv
+    heads, rank, hidden, ctx, batch, layers = 32, 32, 4096, 4096, 8, 32
+    pr = synth.make_latent_producer(heads, rank, hidden, seed=0)
+    A = [pr["A_KV"].to(device) for _ in range(layers)]
+    x = synth.make_activations(batch, hidden, seed=0, key=(42,)).to(device)
+    pos = torch.full((batch,), ctx - 1, dtype=torch.int32, device=device)
+    CK = torch.zeros(batch, heads, ctx, rank, dtype=torch.bfloat16, device=device)
+    CV = torch.zeros_like(CK)
+    kv = lr.LatentKv(batch, heads, ctx, torch.empty(heads, rank, 128, dtype=torch.bfloat16, device=device),
+                     torch.empty(heads, rank, 128, dtype=torch.bfloat16, device=device), 128 ** -0.5)
+    ms = time_graph(lambda i: lr.lr_latent_kv_append(kv, A[i % layers], x, pos, CK, CV), 64)
+    alg = A[0].numel() * 2 + x.numel() * 2 + 2 * batch * heads * rank * 2
+    lib, desc = L.load(), kv.desc()
+    xh = x.cpu().pin_memory()
+    ch = torch.empty(batch, heads, rank, dtype=torch.bfloat16).pin_memory()
+
+    def e2e():
+        x.copy_(xh, non_blocking=True)
+        L.check("lr_latent_kv_append", lib.lr_latent_kv_append(ctypes.byref(desc), A[0].data_ptr(), hidden,
+                                                               x.data_ptr(), pos.data_ptr(), CK.data_ptr(),
+                                                               CV.data_ptr(), stream_ptr()))
+        ch.copy_(CK[:, :, ctx - 1], non_blocking=True)
+    ms_e2e = time_e2e(e2e, 40)
+    row = {"row": "c4app", "workload": "latent producer: x [8, 4096] times the stacked per-head first factors "
+                                       "[2 x 32 heads x rank 32, 4096] bf16, latents written into the caches",
+           "value": ms * 1e3, "unit": "µs per call", "higher_is_better": False, "launches": 1,
+           "roofline": _roof_hbm(alg, ms, "dense GEMV with a cache-scatter epilogue"),
+           "e2e": {"value": ms_e2e * 1e3, "unit": "µs per call", "h2d_bytes_per_step": int(x.numel() * 2),
+                   "d2h_bytes_per_step": int(ch.numel() * 2), "path": "lr_latent_kv_append through the C ABI"},
+           "l2": f"{layers} weight copies ({layers * A[0].numel() * 2 / 1e6:.0f} MB > L2)"}
+    if want_cpu:
+        xc, Ac = x.cpu(), pr["A_KV"]
+        z = torch.zeros(batch, heads, 2, rank, dtype=torch.bfloat16)
+        sec, n = cpu_timed(lambda: okv.append_latents(xc, Ac, heads, rank, z, z, [1] * batch), 2.0, 20)
+        row["cpu_baseline"] = {"value": sec * 1e6, "unit": "µs per call", "cores": host_cores(), "kind": "oracle",
+                               "sample": f"{n} call(s) of the float64 oracle (same weights and batch, 2-position "
+                                         f"caches)"}
+    del A, CK, CV
+    return row
+
+
 def row_c4q8(lr, L, synth, device, ctx, want_cpu):
     """Latent-KV decode over int8 caches (one fp16 scale per position), batch 8, 32 heads, rank 32."""
     import torch
@@ -939,6 +1028,12 @@ def run_rows(args, lr, L, synth, device, ranks, layers, only) -> list:
         if rid.startswith("c4k"):
             rows.append(row_c4(lr, L, synth, device, int(rid[3:]) * 1024, want_cpu))
             torch.cuda.empty_cache()
+        elif rid.startswith("c4rk"):
+            rows.append(row_c4(lr, L, synth, device, int(rid[4:]) * 1024, want_cpu, rope_base=10000.0))
+            torch.cuda.empty_cache()
+        elif rid == "c4app":
+            rows.append(row_c4app(lr, L, synth, device, want_cpu))
+            torch.cuda.empty_cache()
         elif rid.startswith("c4full"):
             rows.append(row_c4full(lr, L, synth, device, int(rid[6:]) * 1024, want_cpu))
             torch.cuda.empty_cache()
@@ -952,6 +1047,7 @@ def run_rows(args, lr, L, synth, device, ranks, layers, only) -> list:
     by = {r["row"]: r for r in rows}
     # speed-up of each low-rank row over its uncompressed baseline (same work, same units)
     for low, base in (("c3b1", "c3dense"), ("c4k4", "c4full4"), ("c4k16", "c4full16"), ("c4k32", "c4full32"),
+                      ("c4rk4", "c4full4"), ("c4rk16", "c4full16"), ("c4rk32", "c4full32"),
                       ("c4q8k4", "c4full4"), ("c4q8k16", "c4full16"), ("c4q8k32", "c4full32")):
         if low in by and base in by:
             by[low]["speedup_vs_uncompressed"] = by[base]["value"] / by[low]["value"]

@@ -51,7 +51,7 @@ class FfnDesc(ctypes.Structure):
 class LatentKvDesc(ctypes.Structure):
     _fields_ = [("batch", c_int), ("heads", c_int), ("head_dim", c_int), ("rank", c_int), ("max_ctx", c_int),
                 ("scale", c_float), ("B_K", c_void_p), ("B_V", c_void_p), ("mode", c_int),
-                ("split_tokens", c_int), ("cache_scale_dtype", c_int)]
+                ("split_tokens", c_int), ("cache_scale_dtype", c_int), ("rope_base", c_float)]
 
 
 class FlashDesc(ctypes.Structure):
@@ -80,6 +80,8 @@ _SIGNATURES = {
     "lr_latent_kv_workspace_size": (c_int, [P(LatentKvDesc), P(c_size_t)]),
     "lr_latent_kv_decode_q8": (c_int, [P(LatentKvDesc), c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                                        c_void_p, c_void_p, c_size_t, c_void_p]),
+    "lr_latent_kv_append": (c_int, [P(LatentKvDesc), c_void_p, c_int, c_void_p, c_void_p, c_void_p, c_void_p,
+                                    c_void_p]),
     "lr_flash_decode": (c_int, [P(FlashDesc), c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_size_t,
                                 c_void_p]),
     "lr_flash_decode_workspace_size": (c_int, [P(FlashDesc), P(c_size_t)]),
@@ -88,6 +90,7 @@ _SIGNATURES = {
     "lr_workspace_init": (c_int, [c_void_p, c_size_t, c_void_p]),
     "lr_check_device_error": (c_int, [c_void_p, P(c_int)]),
     "lr_set_wait_timeout_us": (c_int, [ctypes.c_uint]),
+    "lr_set_tensor_core_min_batch": (c_int, [c_int, c_int]),
     "lr_status_string": (ctypes.c_char_p, [c_int]),
     "lr_version": (c_int, []),
 }

@@ -115,25 +115,58 @@ struct HostStep {
   void* const* y;
 };
 
-// Floats of one accumulator set: the largest step's outputs for one batch chunk.
-size_t chain_acc_set(const HostStep* steps, int n_steps, int batch) {
+// Floats of step s's accumulators for one batch chunk (8-float aligned).
+size_t chain_step_floats(const HostStep& h, int batch) {
   const int chunk = std::min(batch, kMaxDecodeChunk);
-  size_t m = 0;
+  size_t t = 0;
+  for (int p = 0; p < h.n; ++p) t += size_t(chunk) * h.d[p].d_out;
+  return round_up(t, 8);
+}
+
+// ---- batched decode on the tensor cores (bf16 or int8 factors) ----
+// Tokens per pass of the weights, and the accumulator columns of one pass.
+constexpr int kTcMaxPass = 32;
+// Smallest batch that takes the tensor-core path (lr_set_tensor_core_min_batch).
+std::atomic<int> g_tc_min_linear{kMaxDecodeChunk + 1};
+std::atomic<int> g_tc_min_ffn{kMaxDecodeChunk + 1};
+bool use_tc_path(const HostStep* steps, int batch) {
+  return batch >= g_tc_min_linear.load(std::memory_order_relaxed) &&
+         (steps[0].d[0].w_dtype == LR_BF16 || steps[0].d[0].w_dtype == LR_I8);
+}
+bool use_tc_ffn(int batch) { return batch >= g_tc_min_ffn.load(std::memory_order_relaxed); }
+int tc_cols(int batch) { return int(round_up(size_t(std::min(batch, kTcMaxPass)), 8)); }
+
+// Workspace of the tensor-core path: z accumulator [sum of a step's active ranks, cols]
+// and two y accumulator sets [sum of a step's d_out, cols], fp32, zero on entry and exit.
+void tc_sizes(const HostStep* steps, int n_steps, size_t* zmax, size_t* ymax) {
+  *zmax = 0;
+  *ymax = 0;
   for (int s = 0; s < n_steps; ++s) {
-    size_t t = 0;
-    for (int p = 0; p < steps[s].n; ++p) t += size_t(chunk) * steps[s].d[p].d_out;
-    m = std::max(m, t);
+    size_t z = 0, y = 0;
+    for (int p = 0; p < steps[s].n; ++p) {
+      z += size_t(active(&steps[s].d[p]));
+      y += size_t(steps[s].d[p].d_out);
+    }
+    *zmax = std::max(*zmax, z);
+    *ymax = std::max(*ymax, y);
   }
-  return round_up(m, 64);
+}
+size_t tc_ws_bytes(const HostStep* steps, int n_steps, int batch) {
+  size_t zm, ym;
+  tc_sizes(steps, n_steps, &zm, &ym);
+  return kTicketBytes + (zm + 2 * ym) * size_t(tc_cols(batch)) * 4;
 }
 
-size_t chain_ws_bytes(const HostStep* steps, int n_steps, int batch) {
-  return kTicketBytes + 3 * chain_acc_set(steps, n_steps, batch) * 4;
+size_t chain_ws_bytes(const HostStep* steps, int n_steps, int batch, bool allow_tc = true) {
+  size_t b = chain_counter_bytes(n_steps);
+  for (int s = 0; s < n_steps; ++s) b += chain_step_floats(steps[s], batch) * 4;
+  if (allow_tc && use_tc_path(steps, batch)) b = std::max(b, tc_ws_bytes(steps, n_steps, batch));
+  return b;
 }
 
-size_t rank1_ws_bytes(const lr_factor_desc_t* descs, int n, int batch) {
+size_t rank1_ws_bytes(const lr_factor_desc_t* descs, int n, int batch, bool allow_tc = true) {
   HostStep h{descs, n, -1, 0, nullptr};
-  return chain_ws_bytes(&h, 1, batch);
+  return chain_ws_bytes(&h, 1, batch, allow_tc);
 }
 
 lr_status_t check_chain(const HostStep* steps, int n_steps) {
@@ -166,14 +199,195 @@ lr_status_t check_chain(const HostStep* steps, int n_steps) {
   return LR_OK;
 }
 
+// Tensor maps of weight matrices, cached by (address, shape, layout): weights keep
+// their addresses across calls, and encoding a map costs host time on every launch.
+bool weight_map(CUtensorMap* out, const void* W, int rows, int cols, int mn_major, bool i8) {
+  struct Key {
+    const void* W;
+    int rows, cols, mn, i8;
+    bool operator==(const Key& o) const {
+      return W == o.W && rows == o.rows && cols == o.cols && mn == o.mn && i8 == o.i8;
+    }
+  };
+  static std::mutex mu;
+  static std::vector<std::pair<Key, CUtensorMap>> cache;
+  const Key k{W, rows, cols, mn_major, i8 ? 1 : 0};
+  std::lock_guard<std::mutex> lock(mu);
+  for (auto& e : cache)
+    if (e.first == k) {
+      *out = e.second;
+      return true;
+    }
+  if (!tc_make_weight_map(out, W, rows, cols, mn_major, i8)) return false;
+  if (cache.size() >= 4096) cache.clear();
+  cache.push_back({k, *out});
+  return true;
+}
+
+// One product launch over the segments already filled in (maps, seg[].M/K/act/out):
+// split the reduction so that the launch has about two units per SM.
+cudaError_t tc_product(TcMaps& maps, TcGemvParams& g, int sms, bool i8, cudaStream_t stream) {
+  const int kbe = i8 ? 128 : 64;  // reduction elements per k-block
+  int tiles = 0;
+  for (int i = 0; i < g.nseg; ++i) {
+    g.seg[i].m_tiles = (g.seg[i].M + 127) / 128;
+    tiles += g.seg[i].m_tiles;
+  }
+  int ks = std::max(1, (2 * sms + tiles / 2) / std::max(1, tiles));
+  int unit = 0;
+  for (int i = 0; i < g.nseg; ++i) {
+    TcSeg& sg = g.seg[i];
+    int kc = tc_gemv_kc(sg.K, ks, i8);
+    kc = std::max(kc, std::min(4 * kbe, int(round_up(size_t(sg.K), kbe))));  // at least 4 k-blocks per unit
+    while (!tc_gemv_fits(kc, g.N, i8) && kc > kbe) kc -= kbe;
+    sg.kc = kc;
+    sg.k_splits = (sg.K + kc - 1) / kc;   // no empty unit
+    sg.unit0 = unit;
+    unit += sg.m_tiles * sg.k_splits;
+  }
+  int cols = 32;
+  while (cols < g.N + 16) cols *= 2;
+  g.tmem_cols = cols;
+  return launch_tc_gemv(maps, g, i8, stream);
+}
+
+// The chain on the tensor cores, per pass of up to kTcMaxPass tokens and per step:
+//   product 1: z_p += A_p x      (input: the chain input, the previous step's fp32
+//                                 accumulator, or an older step's stored output)
+//   product 2: y_p += B_p^T z_p  (fp32 z split into bf16 high and low parts)
+//   finalize:  y_p (bf16) from the accumulator; zero z and the other y set.
+lr_status_t run_chain_tc(const HostStep* steps, int n_steps, const void* x, int batch, void* ws, cudaStream_t stream) {
+  size_t zmax, ymax;
+  tc_sizes(steps, n_steps, &zmax, &ymax);
+  const int cols = tc_cols(batch);
+  float* zacc = reinterpret_cast<float*>(reinterpret_cast<char*>(ws) + kTicketBytes);
+  float* yacc[2] = {zacc + zmax * cols, zacc + (zmax + ymax) * cols};
+  int* err = device_error_word();
+  const int sms = sm_count_current();
+  const bool i8 = steps[0].d[0].w_dtype == LR_I8;
+  const int scale_f16 = steps[0].d[0].scale_dtype == LR_F16 ? 1 : 0;
+  int x_width = 0;
+  for (int s = 0; s < n_steps; ++s)
+    if (steps[s].input_step < 0) x_width = steps[s].d[0].d_in;
+  for (int b0 = 0; b0 < batch; b0 += kTcMaxPass) {
+    const int nb = std::min(kTcMaxPass, batch - b0);
+    const int nh = int(round_up(size_t(nb), 8));
+    for (int s = 0; s < n_steps; ++s) {
+      const HostStep& h = steps[s];
+      // ---- product 1 ----
+      TcMaps maps;
+      TcGemvParams g;
+      std::memset(&maps, 0, sizeof(maps));
+      std::memset(&g, 0, sizeof(g));
+      g.nseg = h.n;
+      g.nb = nb;
+      g.err = err;
+      const void* act;
+      int act_kind, act_ld;
+      if (h.input_step < 0) {
+        act = reinterpret_cast<const char*>(x) + size_t(b0) * x_width * 2;
+        act_kind = 0;
+        act_ld = x_width;
+      } else if (h.input_step == s - 1) {
+        size_t off = 0;
+        for (int q = 0; q < h.input_proj; ++q) off += size_t(steps[s - 1].d[q].d_out);
+        act = yacc[(s - 1) & 1] + off * cols;
+        act_kind = 1;
+        act_ld = cols;
+      } else {
+        const HostStep& src = steps[h.input_step];
+        act = reinterpret_cast<const char*>(src.y[h.input_proj]) + size_t(b0) * src.d[h.input_proj].d_out * 2;
+        act_kind = 0;
+        act_ld = src.d[h.input_proj].d_out;
+      }
+      g.hilo = (i8 || act_kind == 1) ? 1 : 0;
+      g.N = g.hilo ? std::max(16, 2 * nh) : int(round_up(size_t(nb), 16));
+      size_t zoff = 0;
+      for (int p = 0; p < h.n; ++p) {
+        const lr_factor_desc_t& d = h.d[p];
+        if (!weight_map(&maps.m[p], d.A, active(&d), d.d_in, 0, i8)) return LR_ERR_CUDA;
+        TcSeg& sg = g.seg[p];
+        sg.row_scale = i8 ? d.scale_A : nullptr;
+        sg.row_scale_f16 = scale_f16;
+        sg.M = active(&d);
+        sg.K = d.d_in;
+        sg.a_mn_major = 0;
+        sg.act = act;
+        sg.act_kind = act_kind;
+        sg.act_ld = act_ld;
+        sg.out = zacc + zoff * cols;
+        sg.out_ld = cols;
+        zoff += size_t(sg.M);
+      }
+      cudaError_t e = tc_product(maps, g, sms, i8, stream);
+      if (e != cudaSuccess) return from_cuda(e);
+      // ---- product 2 ----
+      std::memset(&maps, 0, sizeof(maps));
+      g.hilo = 1;
+      g.N = std::max(16, 2 * nh);
+      zoff = 0;
+      size_t yoff = 0;
+      for (int p = 0; p < h.n; ++p) {
+        const lr_factor_desc_t& d = h.d[p];
+        if (!weight_map(&maps.m[p], d.B, active(&d), d.d_out, 1, i8)) return LR_ERR_CUDA;
+        TcSeg& sg = g.seg[p];
+        sg.row_scale = i8 ? d.scale_B : nullptr;
+        sg.row_scale_f16 = scale_f16;
+        sg.M = d.d_out;
+        sg.K = active(&d);
+        sg.a_mn_major = 1;
+        sg.act = zacc + zoff * cols;
+        sg.act_kind = 1;
+        sg.act_ld = cols;
+        sg.out = yacc[s & 1] + yoff * cols;
+        sg.out_ld = cols;
+        zoff += size_t(sg.K);
+        yoff += size_t(sg.M);
+      }
+      e = tc_product(maps, g, sms, i8, stream);
+      if (e != cudaSuccess) return from_cuda(e);
+      // ---- finalize ----
+      TcFinalizeParams f;
+      std::memset(&f, 0, sizeof(f));
+      f.nt = h.n;
+      f.nb = nb;
+      f.ld = cols;
+      yoff = 0;
+      for (int p = 0; p < h.n; ++p) {
+        f.t[p].acc = yacc[s & 1] + yoff * cols;
+        f.t[p].y = reinterpret_cast<char*>(h.y[p]) + size_t(b0) * h.d[p].d_out * 2;
+        f.t[p].M = h.d[p].d_out;
+        yoff += size_t(h.d[p].d_out);
+      }
+      f.zero[0] = zacc;
+      f.zero_floats[0] = zmax * cols;
+      f.zero[1] = yacc[(s + 1) & 1];
+      f.zero_floats[1] = ymax * cols;
+      f.nz = 2;
+      e = launch_tc_finalize(f, sms, stream);
+      if (e != cudaSuccess) return from_cuda(e);
+    }
+    // the last step's accumulator set, now read
+    TcFinalizeParams f;
+    std::memset(&f, 0, sizeof(f));
+    f.zero[0] = yacc[(n_steps - 1) & 1];
+    f.zero_floats[0] = ymax * cols;
+    f.nz = 1;
+    cudaError_t e = launch_tc_finalize(f, sms, stream);
+    if (e != cudaSuccess) return from_cuda(e);
+  }
+  return LR_OK;
+}
+
 lr_status_t run_chain(const HostStep* steps, int n_steps, const void* x, int batch, void* ws, size_t ws_bytes,
-                      cudaStream_t stream) {
+                      cudaStream_t stream, bool allow_tc = true) {
   lr_status_t st = check_chain(steps, n_steps);
   if (st != LR_OK) return st;
   if (!x || batch < 1) return LR_ERR_INVALID_ARG;
   if (!al16(x)) return LR_ERR_MISALIGNED;
-  if (!ws || ws_bytes < chain_ws_bytes(steps, n_steps, batch)) return LR_ERR_WORKSPACE;
+  if (!ws || ws_bytes < chain_ws_bytes(steps, n_steps, batch, allow_tc)) return LR_ERR_WORKSPACE;
   if (!al16(ws)) return LR_ERR_MISALIGNED;
+  if (allow_tc && use_tc_path(steps, batch)) return run_chain_tc(steps, n_steps, x, batch, ws, stream);
   const lr_dtype_t wt = steps[0].d[0].w_dtype;
   const size_t es = (wt == LR_F32) ? 4 : 2;  // activation / output element size
   static ChainParams P;                      // large (kernel parameters); filled under a lock
@@ -183,13 +397,15 @@ lr_status_t run_chain(const HostStep* steps, int n_steps, const void* x, int bat
   P.n_steps = n_steps;
   P.scale_f16 = steps[0].d[0].scale_dtype == LR_F16 ? 1 : 0;
   P.bar = reinterpret_cast<unsigned int*>(ws);
-  P.acc = reinterpret_cast<float*>(reinterpret_cast<char*>(ws) + kTicketBytes);
-  P.acc_set = int(chain_acc_set(steps, n_steps, batch));
+  P.acc = reinterpret_cast<float*>(reinterpret_cast<char*>(ws) + chain_counter_bytes(n_steps));
   P.err = device_error_word();
   P.wait_ns = grid_wait_ns();
   int x_width = 0;
+  size_t acc_off = 0;
   for (int s = 0; s < n_steps; ++s) {
     ChainStep& c = P.step[s];
+    c.acc_off = int(acc_off);
+    acc_off += chain_step_floats(steps[s], batch);
     c.n = steps[s].n;
     c.d_in = steps[s].d[0].d_in;
     c.input_step = steps[s].input_step < 0 ? -1 : steps[s].input_step;
@@ -222,9 +438,9 @@ lr_status_t run_chain(const HostStep* steps, int n_steps, const void* x, int bat
 }
 
 lr_status_t run_rank1(const lr_factor_desc_t* descs, int n, const void* x, int batch, void* const* ys, void* ws,
-                      size_t ws_bytes, cudaStream_t stream) {
+                      size_t ws_bytes, cudaStream_t stream, bool allow_tc = true) {
   HostStep h{descs, n, -1, 0, ys};
-  return run_chain(&h, 1, x, batch, ws, ws_bytes, stream);
+  return run_chain(&h, 1, x, batch, ws, ws_bytes, stream, allow_tc);
 }
 
 // ---------------------------------------------------------------------------
@@ -270,6 +486,13 @@ void noalloc_mark_dirty() {
 
 extern "C" {
 
+lr_status_t lr_set_tensor_core_min_batch(int linear, int ffn) {
+  if (linear < 0 || ffn < 0) return LR_ERR_INVALID_ARG;
+  g_tc_min_linear.store(linear ? linear : kMaxDecodeChunk + 1, std::memory_order_relaxed);
+  g_tc_min_ffn.store(ffn ? ffn : kMaxDecodeChunk + 1, std::memory_order_relaxed);
+  return LR_OK;
+}
+
 lr_status_t lr_set_wait_timeout_us(unsigned int us) {
   g_grid_wait_ns.store(us ? (unsigned long long)us * 1000ull : kGridWaitDefaultNs, std::memory_order_relaxed);
   return LR_OK;
@@ -283,13 +506,14 @@ lr_status_t lr_linear_noalloc(const lr_factor_desc_t* desc, const void* x, int b
   if (!al16(x) || !al16(y)) return LR_ERR_MISALIGNED;
   st = check_rank1_limits(desc);
   if (st != LR_OK) return st;
-  if (rank1_ws_bytes(desc, 1, batch) > size_t(LR_NOALLOC_SCRATCH_BYTES)) return LR_ERR_WORKSPACE;
+  // the CUDA-core path only: its scratch need is what the fixed array is sized for
+  if (rank1_ws_bytes(desc, 1, batch, false) > size_t(LR_NOALLOC_SCRATCH_BYTES)) return LR_ERR_WORKSPACE;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   void* ws = nullptr;
   st = noalloc_scratch(s, &ws);
   if (st != LR_OK) return st;
   void* ys[1] = {y};
-  return run_rank1(desc, 1, x, batch, ys, ws, LR_NOALLOC_SCRATCH_BYTES, s);
+  return run_rank1(desc, 1, x, batch, ys, ws, LR_NOALLOC_SCRATCH_BYTES, s, false);
 }
 
 lr_status_t lr_linear_workspace_size(const lr_factor_desc_t* desc, int batch, int w8a8, size_t* bytes) {
@@ -446,11 +670,122 @@ static lr_status_t check_ffn(const lr_ffn_desc_t* d) {
   return LR_OK;
 }
 
+// Above batch 8 the FFN runs on the tensor cores (int8 weights, kind::i8):
+// accumulators z [rank], gu [2 n_lr], dd [2 n_dense], h [inter], y [hidden],
+// each x cols fp32 (cols = 8-rounded min(batch, 32)), zero on entry and exit.
+static size_t ffn_tc_rows(const lr_ffn_desc_t* d) {
+  return size_t(d->n_lr > 0 ? d->rank : 0) + 2 * size_t(d->inter) + size_t(d->inter) + size_t(d->hidden);
+}
+
 static size_t ffn_ws_bytes(const lr_ffn_desc_t* d, int batch) {
   const int chunk = std::min(batch, kMaxDecodeChunk);
   const int n_dense = d->inter - d->n_lr;
-  return kTicketBytes + round_up(size_t(chunk) * 2 * d->n_lr * 4, 256) + round_up(size_t(chunk) * n_dense * 4, 256) +
-         round_up(size_t(chunk) * d->hidden * 4, 256);
+  size_t b = kTicketBytes + round_up(size_t(chunk) * 2 * d->n_lr * 4, 256) + round_up(size_t(chunk) * n_dense * 4, 256) +
+             round_up(size_t(chunk) * d->hidden * 4, 256);
+  if (use_tc_ffn(batch)) b = std::max(b, kTicketBytes + ffn_tc_rows(d) * size_t(tc_cols(batch)) * 4);
+  return b;
+}
+
+// The hybrid FFN on the tensor cores, per pass of up to kTcMaxPass tokens:
+//   product 1: z += A' x (low-rank latent) and dd += D x (dense gate/up), scaled per row
+//   product 2: gu += B'^T z (low-rank gate/up), scaled per column of B'
+//   SwiGLU:    h = silu(g) u over both branches (clears gu, dd; zeroes z)
+//   product 3: y += W_down^T h, scaled per output column
+//   finalize:  y (bf16), clearing the y accumulator; zeroes h
+static lr_status_t run_ffn_tc(const lr_ffn_desc_t* d, const void* x, int batch, void* y, void* ws,
+                              cudaStream_t stream) {
+  const int cols = tc_cols(batch);
+  const int n_dense = d->inter - d->n_lr;
+  const int rz = d->n_lr > 0 ? d->rank : 0;
+  float* zacc = reinterpret_cast<float*>(reinterpret_cast<char*>(ws) + kTicketBytes);
+  float* gu = zacc + size_t(rz) * cols;
+  float* dd = gu + size_t(2 * d->n_lr) * cols;
+  float* h = dd + size_t(2 * n_dense) * cols;
+  float* yacc = h + size_t(d->inter) * cols;
+  int* err = device_error_word();
+  const int sms = sm_count_current();
+  const int f16 = d->scale_dtype == LR_F16 ? 1 : 0;
+  for (int b0 = 0; b0 < batch; b0 += kTcMaxPass) {
+    const int nb = std::min(kTcMaxPass, batch - b0);
+    const int nh = int(round_up(size_t(nb), 8));
+    const int N = std::max(16, 2 * nh);
+    const void* xb = reinterpret_cast<const char*>(x) + size_t(b0) * d->hidden * 2;
+    auto seg = [&](TcGemvParams& g, TcMaps& maps, int i, const void* W, int rows, int cols_w, int mn, int M, int K,
+                   const void* act, int act_kind, int act_ld, float* out, const void* rs) -> bool {
+      if (!weight_map(&maps.m[i], W, rows, cols_w, mn, true)) return false;
+      TcSeg& sg = g.seg[i];
+      sg.M = M;
+      sg.K = K;
+      sg.a_mn_major = mn;
+      sg.act = act;
+      sg.act_kind = act_kind;
+      sg.act_ld = act_ld;
+      sg.out = out;
+      sg.out_ld = cols;
+      sg.row_scale = rs;
+      sg.row_scale_f16 = f16;
+      g.nseg = i + 1;
+      return true;
+    };
+    TcMaps maps;
+    TcGemvParams g;
+    std::memset(&maps, 0, sizeof(maps));
+    std::memset(&g, 0, sizeof(g));
+    g.nb = nb;
+    g.N = N;
+    g.hilo = 1;
+    g.err = err;
+    int i = 0;
+    if (d->n_lr > 0 && !seg(g, maps, i++, d->A, d->rank, d->hidden, 0, d->rank, d->hidden, xb, 0, d->hidden, zacc, d->s_A))
+      return LR_ERR_CUDA;
+    if (n_dense > 0 &&
+        !seg(g, maps, i++, d->D, 2 * n_dense, d->hidden, 0, 2 * n_dense, d->hidden, xb, 0, d->hidden, dd, d->s_D))
+      return LR_ERR_CUDA;
+    cudaError_t e = tc_product(maps, g, sms, true, stream);
+    if (e != cudaSuccess) return from_cuda(e);
+    if (d->n_lr > 0) {
+      std::memset(&maps, 0, sizeof(maps));
+      if (!seg(g, maps, 0, d->B, d->rank, 2 * d->n_lr, 1, 2 * d->n_lr, d->rank, zacc, 1, cols, gu, d->s_B))
+        return LR_ERR_CUDA;
+      g.nseg = 1;
+      e = tc_product(maps, g, sms, true, stream);
+      if (e != cudaSuccess) return from_cuda(e);
+    }
+    TcSwigluParams sw;
+    std::memset(&sw, 0, sizeof(sw));
+    sw.gu = gu;
+    sw.dd = dd;
+    sw.h = h;
+    sw.n_lr = d->n_lr;
+    sw.n_dense = n_dense;
+    sw.nb = nb;
+    sw.cols = cols;
+    sw.zero = rz ? zacc : nullptr;
+    sw.zero_floats = size_t(rz) * cols;
+    e = launch_tc_swiglu(sw, sms, stream);
+    if (e != cudaSuccess) return from_cuda(e);
+    std::memset(&maps, 0, sizeof(maps));
+    if (!seg(g, maps, 0, d->W_down, d->inter, d->hidden, 1, d->hidden, d->inter, h, 1, cols, yacc, d->s_down))
+      return LR_ERR_CUDA;
+    g.nseg = 1;
+    e = tc_product(maps, g, sms, true, stream);
+    if (e != cudaSuccess) return from_cuda(e);
+    TcFinalizeParams f;
+    std::memset(&f, 0, sizeof(f));
+    f.nt = 1;
+    f.nb = nb;
+    f.ld = cols;
+    f.zero_targets = 1;
+    f.t[0].acc = yacc;
+    f.t[0].y = reinterpret_cast<char*>(y) + size_t(b0) * d->hidden * 2;
+    f.t[0].M = d->hidden;
+    f.zero[0] = h;
+    f.zero_floats[0] = size_t(d->inter) * cols;
+    f.nz = 1;
+    e = launch_tc_finalize(f, sms, stream);
+    if (e != cudaSuccess) return from_cuda(e);
+  }
+  return LR_OK;
 }
 
 lr_status_t lr_dense_linear(const void* W, lr_dtype_t w_dtype, const void* scale, lr_dtype_t scale_dtype, int d_in,
@@ -492,6 +827,7 @@ lr_status_t lr_swiglu_ffn(const lr_ffn_desc_t* d, const void* x, int batch, void
   if (!al16(x) || !al16(y)) return LR_ERR_MISALIGNED;
   if (!ws || ws_bytes < ffn_ws_bytes(d, batch)) return LR_ERR_WORKSPACE;
   if (!al16(ws)) return LR_ERR_MISALIGNED;
+  if (use_tc_ffn(batch)) return run_ffn_tc(d, x, batch, y, ws, reinterpret_cast<cudaStream_t>(stream));
   const int chunk = std::min(batch, kMaxDecodeChunk);
   FfnParams P;
   std::memset(&P, 0, sizeof(P));
@@ -526,11 +862,20 @@ static lr_status_t check_kv(const lr_latent_kv_desc_t* d, int* split) {
   if (!d || !d->B_K || !d->B_V) return LR_ERR_INVALID_ARG;
   if (d->batch <= 0 || d->heads <= 0 || d->max_ctx <= 0 || d->rank <= 0 || d->head_dim <= 0) return LR_ERR_INVALID_ARG;
   if (d->rank != 32 || d->head_dim != 128) return LR_ERR_UNSUPPORTED;
-  if (d->mode != LR_KV_ABSORBED) return LR_ERR_UNSUPPORTED;
+  if (d->mode != LR_KV_ABSORBED && d->mode != LR_KV_RECONSTRUCT) return LR_ERR_UNSUPPORTED;
+  if (!(d->rope_base >= 0.0f) || std::isinf(d->rope_base)) return LR_ERR_INVALID_ARG;
+  // a rotation of the keys makes the absorbed score inexact
+  if (d->mode == LR_KV_ABSORBED && d->rope_base != 0.0f) return LR_ERR_UNSUPPORTED;
   if (d->split_tokens < 0 || (d->split_tokens % 64) != 0 || d->split_tokens > 1024) return LR_ERR_INVALID_ARG;
   if (d->heads > 65535 || d->batch > 65535) return LR_ERR_UNSUPPORTED;
   if (!al16(d->B_K) || !al16(d->B_V)) return LR_ERR_MISALIGNED;
   int t = d->split_tokens;
+  if (d->mode == LR_KV_RECONSTRUCT) {
+    // two 128-position tensor-core tiles per work item; tiled-copy row coordinates are 32-bit
+    if (t != 0 && t != latent_kv_rope_split()) return LR_ERR_UNSUPPORTED;
+    if (double(d->batch) * d->heads * d->max_ctx + 256.0 >= 2147483648.0) return LR_ERR_UNSUPPORTED;
+    t = latent_kv_rope_split();
+  }
   if (t == 0) t = 256;  // measured best at ctx 4K-32K (8 x 32 heads): 32 KiB of cache per CTA, 6 CTAs per SM
   *split = t;
   return LR_OK;
@@ -563,6 +908,7 @@ static lr_status_t run_latent_kv(const lr_latent_kv_desc_t* d, const void* q, co
   if (!q || !C_K || !C_V || !seq_lens || !out) return LR_ERR_INVALID_ARG;
   if (!al16(q) || !al16(C_K) || !al16(C_V) || !al16(seq_lens) || !al16(out)) return LR_ERR_MISALIGNED;
   if (q8) {
+    if (d->mode != LR_KV_ABSORBED) return LR_ERR_UNSUPPORTED;
     if (!s_K || !s_V) return LR_ERR_INVALID_ARG;
     if (d->cache_scale_dtype != LR_F16 && d->cache_scale_dtype != LR_F32) return LR_ERR_UNSUPPORTED;
   }
@@ -582,7 +928,41 @@ static lr_status_t run_latent_kv(const lr_latent_kv_desc_t* d, const void* q, co
   P.cache_scale_f16 = d->cache_scale_dtype == LR_F16 ? 1 : 0;
   P.sK = s_K; P.sV = s_V;
   P.err = device_error_word();
+  if (d->mode == LR_KV_RECONSTRUCT) {
+    KvRopeParams R;
+    std::memset(&R, 0, sizeof(R));
+    R.p = P;
+    for (int i = 0; i < d->head_dim / 2; ++i) {
+      R.theta_d[i] = d->rope_base > 0.0f ? std::pow(double(d->rope_base), -2.0 * i / d->head_dim) : 0.0;
+      R.theta_f[i] = float(R.theta_d[i]);
+    }
+    return from_cuda(launch_latent_kv_rope(R, sm_count_current(), reinterpret_cast<cudaStream_t>(stream)));
+  }
   return from_cuda(launch_latent_kv(P, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+lr_status_t lr_latent_kv_append(const lr_latent_kv_desc_t* d, const void* A_KV, int hidden, const void* x,
+                                const int* pos, void* C_K, void* C_V, lr_stream_t stream) {
+  if (!d || !A_KV || !x || !pos || !C_K || !C_V) return LR_ERR_INVALID_ARG;
+  if (d->batch <= 0 || d->heads <= 0 || d->rank <= 0 || d->max_ctx <= 0 || hidden <= 0) return LR_ERR_INVALID_ARG;
+  if ((hidden % 16) != 0 || size_t(hidden) * 2 > 32768) return LR_ERR_UNSUPPORTED;
+  if (double(2) * d->heads * d->rank > 2147483647.0) return LR_ERR_UNSUPPORTED;
+  if (!al16(A_KV) || !al16(x) || !al16(pos) || !al16(C_K) || !al16(C_V)) return LR_ERR_MISALIGNED;
+  FfnParams P;
+  std::memset(&P, 0, sizeof(P));
+  P.hidden = hidden;
+  P.n_dense = 2 * d->heads * d->rank;
+  P.nb = d->batch;
+  P.D = reinterpret_cast<const int8_t*>(A_KV);
+  P.x = x;
+  P.cache_k = C_K;
+  P.cache_v = C_V;
+  P.cache_pos = pos;
+  P.cache_heads = d->heads;
+  P.cache_rank = d->rank;
+  P.cache_ctx = d->max_ctx;
+  P.err = device_error_word();
+  return from_cuda(launch_dense(P, LR_BF16, sm_count_current(), reinterpret_cast<cudaStream_t>(stream)));
 }
 
 lr_status_t lr_latent_kv_decode(const lr_latent_kv_desc_t* d, const void* q, const void* C_K, const void* C_V,

@@ -12,21 +12,26 @@
 // warp streams the CTA's rows of every step, A rows then B rows, through a
 // ring of shared-memory stages with bulk copies (cp.async.bulk completing on
 // mbarriers).  It never waits for a step boundary, only for a free stage, so
-// DRAM keeps streaming the next step's rows while the CTA waits at a grid
-// barrier.  Sixteen consumer warps, per step:
+// DRAM keeps streaming the next steps' rows while the CTA waits for an input.
+// Sixteen consumer warps, per step:
+//   input    wait until every CTA has finished the step this one reads (one
+//            completion counter per step, bounded in time; every CTA is
+//            resident, which the launch checks), then load x in fp32: the
+//            chain input, or the input step's fp32 accumulator;
 //   phase A  z_j = x_s . a_j: warp w takes line w (512 bytes) of every row in
 //            a stage, keeps x in registers, reduces the stage's rows with one
 //            butterfly and adds its line sums into z in shared memory;
 //   phase B  y_p += z_j b_j: warp w takes line w of every B row and keeps the
-//            output line in registers, adding it into the fp32 accumulator
-//            set s % 3 (red.global.add.v4.f32) when a projection's rows end;
-//   barrier  thread 0 arrives with one release reduction and waits on a
-//            monotonic counter (bounded in time; every CTA is resident, which
-//            the launch checks).
-// The outputs of step s-1 are written during step s (their accumulator loads
-// share the round trip of the step's input loads), and each CTA then zeroes
-// its slice of set (s-2) % 3, which nothing reads any more; the last step's
-// set is zeroed at exit, so the workspace is all zero between calls.
+//            output line in registers, adding it into the step's own fp32
+//            accumulator (red.global.add.v4.f32) when a projection's rows end;
+//   done     thread 0 adds one to the step's completion counter (release).
+// A step waits only for the step it reads: a step whose input is already
+// complete (for example K and Q next to V, which O reads) starts at once, so
+// independent work covers the hand-off of a dependent one.  Every step keeps
+// its own accumulators, so nothing is reused within a launch; after the last
+// step each CTA writes its share of every step's outputs and clears those
+// accumulators, and the last CTA to leave resets the counters, so the
+// workspace is all zero between calls.
 #include <algorithm>
 #include <cstring>
 #include <type_traits>
@@ -212,9 +217,8 @@ LR_DEV int bfly_index(int lane) {
 }
 
 // ---- the step's input for this lane's columns (fp32 registers) ------------
-// Chain input: the caller's x (bf16, or fp32 for fp32 weights).  Previous
-// step: its fp32 accumulator (times the int8 output scale).  Older step: its
-// stored output.
+// Chain input: the caller's x (bf16, or fp32 for fp32 weights).  An earlier
+// step: its fp32 accumulator (times the int8 output scale).
 template <typename WT, int NB, int L>
 LR_DEV void load_x(const ChainParams& P, int s, const WarpMap& m, float (&xr)[L][NB][Lane16<WT>::kElems],
                    int lane) {
@@ -235,9 +239,9 @@ LR_DEV void load_x(const ChainParams& P, int s, const WarpMap& m, float (&xr)[L]
       for (int e = 0; e < EPC; ++e) f[e] = 0.f;
       if (!valid || b >= P.nb) continue;
       const size_t idx = size_t(b) * d_in + col;
-      if (S.input_step == s - 1 && s > 0) {
+      if (S.input_step >= 0) {
         const ChainStep& I = P.step[S.input_step];
-        const float* a = P.acc + size_t((s + 2) % 3) * P.acc_set + acc_offset(I, S.input_proj, P.nb) + idx;
+        const float* a = P.acc + I.acc_off + acc_offset(I, S.input_proj, P.nb) + idx;
 #pragma unroll
         for (int q = 0; q < EPC; q += 4) {
           const float4 v = ld_cg_f4(a + q);
@@ -249,9 +253,7 @@ LR_DEV void load_x(const ChainParams& P, int s, const WarpMap& m, float (&xr)[L]
           for (int e = 0; e < EPC; ++e) f[e] *= load_scale(sB, col + e, f16);
         }
       } else {
-        const XT* src = S.input_step < 0
-                            ? reinterpret_cast<const XT*>(P.x)
-                            : reinterpret_cast<const XT*>(P.step[S.input_step].p[S.input_proj].y);
+        const XT* src = reinterpret_cast<const XT*>(P.x);
         if constexpr (sizeof(XT) == 4) {
           const float4 v = ld_cg_f4(src + idx);
           f[0] = v.x; f[1] = v.y; f[2] = v.z; f[3] = v.w;
@@ -282,32 +284,20 @@ LR_DEV float* out_locate(const ChainParams& P, int t, int c, int* p_out, int* of
   }
   *p_out = p;
   *off_out = off;
-  return P.acc + size_t(t % 3) * P.acc_set + base + off;
+  return P.acc + S.acc_off + base + off;
 }
 
-// Loads of this thread's first chunk (issued early; used by write_outputs).
-LR_DEV void out_preload(const ChainParams& P, int t, float4* v0, float4* v1) {
-  int c0, c1, p, off;
-  out_range(P, t, &c0, &c1);
-  const int c = c0 + int(threadIdx.x);
-  if (c < c1) {
-    const float* a = out_locate(P, t, c, &p, &off);
-    *v0 = ld_cg_f4(a);
-    *v1 = ld_cg_f4(a + 4);
-  }
-}
-
+// This CTA's share of step t's outputs: scale, round, store; clear the accumulators read.
 template <typename YT>
-LR_DEV void write_outputs(const ChainParams& P, int t, bool zero_after, float4 pv0, float4 pv1) {
+LR_DEV void write_outputs(const ChainParams& P, int t) {
   const bool f16 = P.scale_f16 != 0;
   int c0, c1;
   out_range(P, t, &c0, &c1);
-  bool first = true;
-  for (int c = c0 + int(threadIdx.x); c < c1; c += kConsumers, first = false) {
+  for (int c = c0 + int(threadIdx.x); c < c1; c += kConsumers) {
     int p, off;
     float* a = out_locate(P, t, c, &p, &off);
     const ChainProj& pr = P.step[t].p[p];
-    const float4 v0 = first ? pv0 : ld_cg_f4(a), v1 = first ? pv1 : ld_cg_f4(a + 4);
+    const float4 v0 = ld_cg_f4(a), v1 = ld_cg_f4(a + 4);
     float v[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
     if (pr.sB) {
       const int k = off % pr.d_out;
@@ -328,23 +318,8 @@ LR_DEV void write_outputs(const ChainParams& P, int t, bool zero_after, float4 p
       *reinterpret_cast<float4*>(y) = make_float4(v[0], v[1], v[2], v[3]);
       *reinterpret_cast<float4*>(y + 4) = make_float4(v[4], v[5], v[6], v[7]);
     }
-    if (zero_after) {
-      st_cg_f4(a, make_float4(0.f, 0.f, 0.f, 0.f));
-      st_cg_f4(a + 4, make_float4(0.f, 0.f, 0.f, 0.f));
-    }
-  }
-}
-
-// Zero this CTA's share of the region step t used in its accumulator set.
-LR_DEV void zero_set_slice(const ChainParams& P, int t) {
-  const ChainStep& S = P.step[t];
-  float* set = P.acc + size_t(t % 3) * P.acc_set;
-  const int total = acc_offset(S, S.n, P.nb) / 8;
-  int c0, c1;
-  split_range(total, blockIdx.x, gridDim.x, &c0, &c1);
-  for (int c = c0 + int(threadIdx.x); c < c1; c += kConsumers) {
-    st_cg_f4(set + c * 8, make_float4(0.f, 0.f, 0.f, 0.f));
-    st_cg_f4(set + c * 8 + 4, make_float4(0.f, 0.f, 0.f, 0.f));
+    st_cg_f4(a, make_float4(0.f, 0.f, 0.f, 0.f));
+    st_cg_f4(a + 4, make_float4(0.f, 0.f, 0.f, 0.f));
   }
 }
 
@@ -434,12 +409,14 @@ __global__ void __launch_bounds__(kThreads, 1) chain_kernel(const __grid_constan
   bool failed = false;
   for (int s = 0; s < P.n_steps; ++s) {
     const ChainStep& S = P.step[s];
-    // ---- the step's input and the previous step's outputs: one round trip ----
+    // ---- the step's input: wait for the step it reads, then load it ----
+    if (S.input_step >= 0) {
+      if (threadIdx.x == 0) wait_counter_geq(P.bar + S.input_step, gridDim.x, P.wait_ns, P.err);
+      consumer_sync();
+    }
     const WarpMap ma = warp_map(S.d_in * int(sizeof(WT)));
     float xr[L][NB][EPC];
     load_x<WT, NB, L>(P, s, ma, xr, lane);
-    float4 ov0 = make_float4(0.f, 0.f, 0.f, 0.f), ov1 = ov0;
-    if (s >= 1) out_preload(P, s - 1, &ov0, &ov1);
 
     // ---- phase A: z_j = x . a_j ----
     for_segments<WT>(S, 0, [&](int p, const unsigned char*, int row_bytes, int z0, int j0, int rows) {
@@ -488,13 +465,10 @@ __global__ void __launch_bounds__(kThreads, 1) chain_kernel(const __grid_constan
         ++st;
       }
     });
-    // ---- outputs of step s-1; step s-2's set is no longer read ----
-    if (s >= 1) write_outputs<YT>(P, s - 1, false, ov0, ov1);
-    if (s >= 2) zero_set_slice(P, s - 2);
     consumer_sync();  // z complete
 
     // ---- phase B: y += z_j b_j ----
-    float* acc_set = P.acc + size_t(s % 3) * P.acc_set;
+    float* acc_set = P.acc + S.acc_off;
     for_segments<WT>(S, 1, [&](int p, const unsigned char*, int row_bytes, int z0, int, int rows) {
       const WarpMap mb = warp_map(row_bytes);
       const int rps = stage_rows(row_bytes, GR);
@@ -537,29 +511,24 @@ __global__ void __launch_bounds__(kThreads, 1) chain_kernel(const __grid_constan
       if (!failed) flush_lines<WT, NB, L>(acc, acc_set + acc_offset(S, p, nb), row_bytes, nb, mb, lane);
     });
 
-    // ---- barrier s: all partial outputs of step s are in ----
+    // ---- step s done: all of this CTA's partial outputs of step s are issued ----
     consumer_sync();
     for (int i = threadIdx.x; i < rows_cap * NB; i += kConsumers) zs[i] = 0.f;
-    if (threadIdx.x == 0) {
-      red_release_add(P.bar, 1u);
-      wait_counter_geq(P.bar, gridDim.x * unsigned(s + 1), P.wait_ns, P.err);
-    }
+    if (threadIdx.x == 0) red_release_add(P.bar + s, 1u);
     consumer_sync();
   }
 
-  // ---- outputs of the last step; leave the workspace zero ----
-  const int last = P.n_steps - 1;
-  float4 ov0 = make_float4(0.f, 0.f, 0.f, 0.f), ov1 = ov0;
-  out_preload(P, last, &ov0, &ov1);
-  write_outputs<YT>(P, last, true, ov0, ov1);
-  if (last >= 1) zero_set_slice(P, last - 1);
+  // ---- every step's outputs (the last step completes after all others); clear ----
+  if (threadIdx.x == 0) wait_counter_geq(P.bar + (P.n_steps - 1), gridDim.x, P.wait_ns, P.err);
+  consumer_sync();
+  for (int t = 0; t < P.n_steps; ++t) write_outputs<YT>(P, t);
   consumer_sync();
   if (threadIdx.x == 0) {
     __threadfence();
-    const unsigned prev = atomicAdd(P.bar + 1, 1u);
+    unsigned int* exit_count = P.bar + P.n_steps;
+    const unsigned prev = atomicAdd(exit_count, 1u);
     if (prev == gridDim.x - 1) {
-      atomicExch(P.bar, 0u);
-      atomicExch(P.bar + 1, 0u);
+      for (int t = 0; t <= P.n_steps; ++t) atomicExch(P.bar + t, 0u);
     }
   }
 }
@@ -649,7 +618,6 @@ cudaError_t launch_chain_w(const ChainParams& p0, int sm_count, cudaStream_t s) 
 
 }  // namespace
 
-size_t chain_workspace_bytes(const ChainParams& p) { return kTicketBytes + size_t(3) * p.acc_set * 4; }
 
 cudaError_t launch_chain(const ChainParams& p, lr_dtype_t w_dtype, int sm_count, cudaStream_t s) {
   switch (w_dtype) {

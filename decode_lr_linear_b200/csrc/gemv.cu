@@ -549,8 +549,20 @@ __global__ void __launch_bounds__(kThreads, (NB <= 1 && LPW <= 2 ? 2 : 1)) strea
           float v = 0.f;
 #pragma unroll 4
           for (int w = 0; w < kConsumerWarps; ++w) v += part[(r * kConsumerWarps + w) * NB + b];
-          reinterpret_cast<__nv_bfloat16*>(K.f.y)[size_t(b) * K.f.n_dense + pl.row_base + r] =
-              __float2bfloat16_rn(v * row_scale<MODE>(K, pl, r));
+          const __nv_bfloat16 o = __float2bfloat16_rn(v * row_scale<MODE>(K, pl, r));
+          const int row = pl.row_base + r;
+          if (!K.f.cache_k) {
+            reinterpret_cast<__nv_bfloat16*>(K.f.y)[size_t(b) * K.f.n_dense + row] = o;
+          } else {
+            // latent producer: row (kv, head, j) of token b goes to its cache position
+            const int hr = K.f.cache_heads * K.f.cache_rank, ps = K.f.cache_pos[b];
+            const int kv = row >= hr ? 1 : 0, rr = row - kv * hr;
+            if (ps >= 0 && ps < K.f.cache_ctx) {
+              __nv_bfloat16* c = reinterpret_cast<__nv_bfloat16*>(kv ? K.f.cache_v : K.f.cache_k);
+              c[((size_t(b) * K.f.cache_heads + rr / K.f.cache_rank) * K.f.cache_ctx + ps) * K.f.cache_rank +
+                rr % K.f.cache_rank] = o;
+            }
+          }
         }
       }
     }
@@ -723,7 +735,14 @@ cudaError_t launch_dense_impl(const FfnParams& p0, int sm_count, cudaStream_t s)
     FfnParams f = p0;
     f.nb = std::min(kMaxDecodeChunk, p0.nb - b0);
     f.x = reinterpret_cast<const __nv_bfloat16*>(p0.x) + size_t(b0) * p0.hidden;
-    f.y = reinterpret_cast<__nv_bfloat16*>(p0.y) + size_t(b0) * p0.n_dense;
+    if (p0.cache_k) {
+      const size_t per_b = size_t(p0.cache_heads) * p0.cache_ctx * p0.cache_rank;
+      f.cache_k = reinterpret_cast<__nv_bfloat16*>(p0.cache_k) + size_t(b0) * per_b;
+      f.cache_v = reinterpret_cast<__nv_bfloat16*>(p0.cache_v) + size_t(b0) * per_b;
+      f.cache_pos = p0.cache_pos + b0;
+    } else {
+      f.y = reinterpret_cast<__nv_bfloat16*>(p0.y) + size_t(b0) * p0.n_dense;
+    }
     K.f = f;
     cudaError_t e = dispatch<WT, __nv_bfloat16, __nv_bfloat16, kDense>(K, f.nb, 1, grid, sm_count, s);
     if (e != cudaSuccess) return e;

@@ -1,6 +1,7 @@
 // Internal launch interface between the C ABI (api.cu) and the kernel files.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -50,6 +51,7 @@ struct ChainStep {
   int total_rows;
   int input_step;     // -1: chain input
   int input_proj;
+  int acc_off;        // first float of this step's accumulators in ChainParams::acc
 };
 
 struct ChainParams {
@@ -57,16 +59,16 @@ struct ChainParams {
   int n_steps;
   int nb;             // batch rows in this launch (<= kMaxDecodeChunk)
   const void* x;      // chain input [nb, d_in of step 0], offset to the chunk
-  float* acc;         // 3 accumulator sets of acc_set floats (zero on entry and exit)
-  int acc_set;        // floats per set
-  unsigned int* bar;  // 2 barrier counters (zero on entry and exit)
+  float* acc;         // every step's fp32 output accumulators (zero on entry and exit)
+  unsigned int* bar;  // n_steps completion counters + one exit counter (zero on entry and exit)
   int scale_f16;
   int* err;
-  unsigned long long wait_ns;  // bound of the grid-barrier waits
+  unsigned long long wait_ns;  // bound of the waits on other CTAs
 };
 
 static_assert(sizeof(ChainParams) < 32000, "chain parameters must fit the kernel parameter space");
-size_t chain_workspace_bytes(const ChainParams& p);
+// Bytes of the chain's counters (the accumulators follow them in the workspace).
+inline size_t chain_counter_bytes(int n_steps) { return (size_t(n_steps + 1) * 4 + 255) / 256 * 256; }
 cudaError_t launch_chain(const ChainParams& p, lr_dtype_t w_dtype, int sm_count, cudaStream_t s);
 
 struct FfnParams {
@@ -85,6 +87,13 @@ struct FfnParams {
   unsigned int* ticket;
   unsigned long long wait_ns;  // bound of the grid-barrier wait
   int* err;                    // device error word
+  // dense mode only: when cache_k is set, output row j of token b is not written
+  // to y but to the latent caches [batch, heads, ctx, rank] at position cache_pos[b]
+  // (rows [0, heads*rank) -> cache_k, the next heads*rank rows -> cache_v), bf16
+  void* cache_k;
+  void* cache_v;
+  const int* cache_pos;
+  int cache_heads, cache_rank, cache_ctx;
 };
 
 cudaError_t launch_ffn(const FfnParams& p, int sm_count, cudaStream_t s);
@@ -110,6 +119,75 @@ struct LatentKvParams {
 };
 
 cudaError_t launch_latent_kv(const LatentKvParams& p, cudaStream_t s);
+// The merge of the splits and o = a B_V (the last launch of launch_latent_kv).
+cudaError_t launch_latent_kv_combine(const LatentKvParams& p, cudaStream_t s);
+
+// Keys reconstructed on chip, with an optional rotary embedding: p.split_tokens
+// must be latent_kv_rope_split(); theta = 0 everywhere means no rotation.
+struct KvRopeParams {
+  LatentKvParams p;
+  float theta_f[64];   // rotary frequencies theta_i = base^(-2i/head_dim)
+  double theta_d[64];
+};
+int latent_kv_rope_split();
+cudaError_t launch_latent_kv_rope(const KvRopeParams& r, int sm_count, cudaStream_t s);
+
+// ---- batched decode on the tensor cores (tc_gemv.cu) ----
+// One product out[m][n] += sum_k W[m][k] act[n][k] over up to four weight
+// matrices ("segments"), each split into units of 128 rows x kc of the reduction.
+struct TcSeg {
+  int M, K;           // weight rows (outputs) and reduction length
+  int a_mn_major;     // 0: W stored [M, K]; 1: W stored [K, M] (its tensor map in TcMaps)
+  int m_tiles, k_splits, kc, unit0;
+  const void* act;    // act_kind 0: bf16 [nb, K] (row stride act_ld); 1: fp32 [K, act_ld]
+  int act_kind, act_ld;
+  float* out;         // fp32 [M, out_ld], added into
+  int out_ld;
+  const void* row_scale;  // int8 weights: one scale per weight row (output channel), or null
+  int row_scale_f16;
+};
+struct TcGemvParams {
+  TcSeg seg[4];
+  int nseg;
+  int N;              // MMA N: token rows of the operand (x2 with hilo)
+  int nb;             // tokens
+  int hilo;           // split each fp32 activation into bf16 high and low parts (rows nb.. of the operand)
+  int tmem_cols;
+  int* err;
+};
+struct alignas(64) TcMaps {
+  CUtensorMap m[4];
+};
+struct TcFinalTarget {
+  const float* acc;   // [M, ld]
+  void* y;            // bf16 [nb, M]
+  int M;
+};
+struct TcFinalizeParams {
+  TcFinalTarget t[4];
+  int nt;
+  int nb, ld;
+  int zero_targets;   // clear each accumulator element after reading it
+  float* zero[2];
+  size_t zero_floats[2];  // multiples of 4
+  int nz;
+};
+// i8: int8 weights (kind::i8, activations as high and low int8 codes; hilo must be set)
+int tc_gemv_kc(int K, int k_splits, bool i8);
+size_t tc_gemv_smem(int kc, int N, bool i8);
+bool tc_gemv_fits(int kc, int N, bool i8);
+bool tc_make_weight_map(CUtensorMap* m, const void* W, int rows, int cols, int a_mn_major, bool i8);
+cudaError_t launch_tc_gemv(const TcMaps& maps, const TcGemvParams& p, bool i8, cudaStream_t s);
+cudaError_t launch_tc_finalize(const TcFinalizeParams& f, int sm_count, cudaStream_t s);
+struct TcSwigluParams {
+  float* gu;          // [2 n_lr, cols] gate/up accumulators of the low-rank channels (interleaved rows)
+  float* dd;          // [2 n_dense, cols] of the dense channels
+  float* h;           // [n_lr + n_dense, cols]
+  int n_lr, n_dense, nb, cols;
+  float* zero;        // region zeroed afterwards (or null)
+  size_t zero_floats; // multiple of 4
+};
+cudaError_t launch_tc_swiglu(const TcSwigluParams& p, int sm_count, cudaStream_t s);
 
 // Full-K/V flash decoding (the uncompressed baseline).
 struct FlashParams {

@@ -261,8 +261,20 @@ cudaError_t launch_latent_kv(const LatentKvParams& p, cudaStream_t s) {
   e = q8 ? cudaLaunchKernelEx(&c1, latent_kv_split_kernel<true>, p)
          : cudaLaunchKernelEx(&c1, latent_kv_split_kernel<false>, p);
   if (e != cudaSuccess) return e;
-  cudaLaunchConfig_t c2 = c0;
-  return cudaLaunchKernelEx(&c2, latent_kv_combine_kernel, p);
+  return launch_latent_kv_combine(p, s);
+}
+
+cudaError_t launch_latent_kv_combine(const LatentKvParams& p, cudaStream_t s) {
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t c = {};
+  c.gridDim = dim3(p.heads, p.batch);
+  c.blockDim = dim3(kThreads);
+  c.stream = s;
+  c.attrs = attr;
+  c.numAttrs = 1;
+  return cudaLaunchKernelEx(&c, latent_kv_combine_kernel, p);
 }
 
 }  // namespace lr

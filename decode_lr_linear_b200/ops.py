@@ -95,6 +95,7 @@ class LatentKv:
     scale: float
     mode: int = L.LR_KV_ABSORBED
     split_tokens: int = 0
+    rope_base: float = 0.0
     rank: int = field(init=False)
     head_dim: int = field(init=False)
 
@@ -103,7 +104,8 @@ class LatentKv:
 
     def desc(self, cache_scale_dtype: int = L.LR_F16) -> L.LatentKvDesc:
         return L.LatentKvDesc(self.batch, self.heads, self.head_dim, self.rank, self.max_ctx, self.scale,
-                              _ptr(self.B_K), _ptr(self.B_V), self.mode, self.split_tokens, cache_scale_dtype)
+                              _ptr(self.B_K), _ptr(self.B_V), self.mode, self.split_tokens, cache_scale_dtype,
+                              self.rope_base)
 
 
 def workspace(nbytes: int, device) -> torch.Tensor:
@@ -253,6 +255,15 @@ def lr_latent_kv_decode(kv: LatentKv, q: torch.Tensor, C_K: torch.Tensor, C_V: t
     return out
 
 
+def lr_latent_kv_append(kv: LatentKv, A_KV: torch.Tensor, x: torch.Tensor, pos: torch.Tensor, C_K: torch.Tensor,
+                        C_V: torch.Tensor, stream=None) -> None:
+    """Write the new token's per-head latents x A_Kh, x A_Vh into C_K, C_V at position pos[b]."""
+    d = kv.desc()
+    L.check("lr_latent_kv_append",
+            L.load().lr_latent_kv_append(ctypes.byref(d), _ptr(A_KV), A_KV.shape[1], _ptr(x), _ptr(pos), _ptr(C_K),
+                                         _ptr(C_V), _stream(stream)))
+
+
 def lr_quantize_per_token(x: torch.Tensor, x_q: Optional[torch.Tensor] = None, s: Optional[torch.Tensor] = None,
                           stream=None):
     rows, cols = x.shape
@@ -292,6 +303,11 @@ def lr_check_device_error(stream=None) -> int:
 def lr_set_wait_timeout_us(us: int) -> None:
     """Bound of a persistent kernel's waits on its other CTAs, in microseconds (0: default, 1 s)."""
     L.check("lr_set_wait_timeout_us", L.load().lr_set_wait_timeout_us(int(us)))
+
+
+def lr_set_tensor_core_min_batch(linear: int = 0, ffn: int = 0) -> None:
+    """Smallest batch that takes the tensor-core path (0: the default, 9)."""
+    L.check("lr_set_tensor_core_min_batch", L.load().lr_set_tensor_core_min_batch(int(linear), int(ffn)))
 
 
 def _rank_vec(values):

@@ -382,6 +382,14 @@ def make_latent_kv_int8(batch: int = 8, heads: int = 32, ctx: int = 4096, rank: 
     return out
 
 
+def make_latent_producer(heads: int = 32, rank: int = 32, hidden: int = 4096, seed: int = 0) -> dict:
+    """First factors of the per-head key/value projections, latent-major and stacked:
+    A_KV [2 * heads * rank, hidden] bf16 ~ N(0, 1/hidden) (rows h*rank + j: A_Kh column j;
+    rows (heads + h)*rank + j: A_Vh column j), so a latent of an N(0,1) token is O(1)."""
+    A = normals((2 * heads * rank, hidden), seed, (7, heads, rank, hidden)) / math.sqrt(hidden)
+    return {"A_KV": to_bf16(A), "heads": heads, "rank": rank, "hidden": hidden}
+
+
 # --------------------------------------------------------------------------
 # W8A8 prefill (LLaMA-13B shapes).
 # --------------------------------------------------------------------------

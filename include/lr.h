@@ -115,6 +115,12 @@ typedef struct lr_factor_desc {
  *   w_dtype LR_BF16: x bf16 [batch, d_in] -> y bf16 [batch, d_out]
  *   w_dtype LR_I8:   x bf16 [batch, d_in] -> y bf16 [batch, d_out]
  *   accumulation in fp32; the r-dim latent z = x A stays on chip in fp32.
+ *   Up to batch 8 (and always for f32 and int8 weights) the CUDA cores
+ *   stream the factors; bf16 factors above batch 8 run on the tensor cores
+ *   (tcgen05, weights as the M operand, tokens as N), streaming every factor
+ *   once per pass of up to 32 tokens; there the latent goes through an fp32
+ *   accumulator in the workspace, split into bf16 high and low parts for the
+ *   second product (fp32 accuracy).
  * W8A8 path (x_scale != NULL; w_dtype LR_I8, scale_dtype LR_F32):
  *   x int8 [batch, d_in] with per-token scales x_scale f32 [batch] (from
  *   lr_quantize_per_token), y bf16 [batch, d_out]; int8 x int8 -> int32 tensor
@@ -126,7 +132,11 @@ typedef struct lr_factor_desc {
  *   weights and activations quantised, e.g. W8A8).
  * Weight-only limits: d_in and d_out multiples of 8 (of 16 for int8 weights)
  * and at most 32 KiB per factor row (d <= 16384 for bf16, 8192 for f32).
- * ws: workspace of at least lr_linear_workspace_size(...) bytes.
+ * ws: workspace of at least lr_linear_workspace_size(...) bytes: 256 +
+ * 8-rounded(min(batch, 8) * d_out) * 4, and for bf16 or int8 factors above
+ * batch 8 at least 256 + (r + 2 d_out) * c * 4 with c = 8-rounded
+ * min(batch, 32) (r the active rank).  Zero on entry (lr_workspace_init);
+ * every call leaves it zero.
  * Errors: LR_ERR_INVALID_ARG (null pointers, batch < 1, bad shape or rank),
  * LR_ERR_UNSUPPORTED (dtype combination), LR_ERR_MISALIGNED,
  * LR_ERR_WORKSPACE, LR_ERR_CUDA.
@@ -160,22 +170,28 @@ LR_API lr_status_t lr_linear_grouped_workspace_size(const lr_factor_desc_t* desc
  * Step s computes y[s][p] = (x_s A[s][p]) B[s][p] for p < n, with
  *   x_s = x                      when input_step < 0,
  *   x_s = y[input_step][input_proj] otherwise (input_step < s).
- * An input taken from the step right before is read at fp32 (its accumulator
- * times the int8 output scale, before the output rounding to bf16); an older
- * one is read from its stored output.  Every step's outputs are written.  All
+ * An input taken from an earlier step is read at fp32 (its accumulator times
+ * the int8 output scale, before the output rounding to bf16).  Every step's
+ * outputs are written.  A step waits only for the step it reads, so steps
+ * whose inputs are ready (for example Q and K next to V, which O reads)
+ * overlap the hand-off of a dependent one.  All
  * descriptors of a step share d_in, which must equal d_out of the projection
  * its input comes from; all steps share w_dtype (weight-only paths) and
  * scale_dtype; any batch >= 1 (one launch per 8 rows or fewer, depending on
  * the widest row); at most LR_MAX_CHAIN steps.
- * One persistent CTA per SM (all resident: checked before the launch,
- * LR_ERR_UNSUPPORTED otherwise) streams the factors of all steps back to back
- * through shared memory, so the loads of step s+1 proceed while step s is
- * finishing; the CTAs meet at one grid-wide barrier per step, bounded in time
- * (lr_set_wait_timeout_us).  LASER "System Implementation" fuses the stages
+ * bf16 and int8 factors above batch 8 run on the tensor cores instead (as
+ * lr_linear: three launches per step and pass of up to 32 tokens; there the
+ * step right before is read at fp32 from its accumulator and an older step
+ * from its stored output).
+ * Up to batch 8, one persistent CTA per SM (all resident: checked before the
+ * launch, LR_ERR_UNSUPPORTED otherwise) streams the factors of all steps back
+ * to back through shared memory, so the loads of later steps proceed while a
+ * step waits for its input; that wait on the CTAs producing the input is
+ * bounded in time (lr_set_wait_timeout_us).  LASER "System Implementation" fuses the stages
  * of a layer to cut memory movement and kernel-launch overhead; this is that
  * fusion across consecutive factorised projections.
  */
-#define LR_MAX_CHAIN 64
+#define LR_MAX_CHAIN 128
 typedef struct lr_chain_step {
   int n;
   int input_step;
@@ -241,8 +257,8 @@ LR_API lr_status_t lr_linear_chain_ranked(const lr_chain_step_t* steps, int n_st
  * LR_NOALLOC_SCRATCH_BYTES bytes per device, which every GPU that loads the
  * library keeps until the process exits.  The caller still passes x and y.
  *
- *   - The scratch a call needs is what lr_linear_workspace_size reports,
- *     256 + 3 * 64-rounded(min(batch, 8) * d_out) * 4 bytes; a call that needs
+ *   - The scratch a call needs is 256 + 8-rounded(min(batch, 8) * d_out) * 4
+ *     bytes (this call stays on the CUDA-core path at every batch); a call that needs
  *     more returns LR_ERR_WORKSPACE and launches nothing.  Shapes lr_linear
  *     refuses are refused the same way (LR_ERR_UNSUPPORTED) before that.
  *   - The first call on a device (in a CUDA context) looks the array up and
@@ -339,12 +355,21 @@ LR_API lr_status_t lr_swiglu_ffn_workspace_size(const lr_ffn_desc_t* desc, int b
  *             K_t = C_K[b,h,t,:] B_K[h], value V_t = C_V[b,h,t,:] B_V[h]
  *   scale     softmax scale (1/sqrt(head_dim) for standard attention)
  *   mode      LR_KV_ABSORBED: scores s_t = C_K[t] (B_K q) * scale, latent
- *             values accumulated and reconstructed once per split (the only
- *             mode implemented);
- *             LR_KV_RECONSTRUCT: reserved for on-chip reconstruction of the
- *             key tiles (needed once a position-dependent rotation is applied
- *             to keys); returns LR_ERR_UNSUPPORTED
+ *             values accumulated and reconstructed once per split; exact
+ *             only without a rotary embedding (rope_base must be 0);
+ *             LR_KV_RECONSTRUCT: keys reconstructed on chip, 128 cached
+ *             positions at a time on the tensor cores, and rotated before the
+ *             score: with rope_base > 0, K_t is rotated to position t and q to
+ *             position seq_lens[b] - 1 (LLaMA convention: theta_i =
+ *             rope_base^(-2i/head_dim), dimension i turns with i + head_dim/2
+ *             by pos * theta_i; the pages' models are LLaMA-family, the pages do
+ *             not write the embedding out); values carry no rotation.  bf16
+ *             caches only (lr_latent_kv_decode); split_tokens 0 or 256;
+ *             batch * heads * max_ctx < 2^31 - 256.  Scores use the query and
+ *             B_K folded into one bf16 operand per tile (error well inside the
+ *             1e-2 normwise bar).
  *   split_tokens  tokens per split-K chunk (multiple of 64), 0 = library choice
+ *   rope_base     0: no rotary embedding; > 0: its base (e.g. 10000)
  * Supported: rank 32, head_dim 128.
  */
 #define LR_KV_ABSORBED 0
@@ -361,6 +386,7 @@ typedef struct lr_latent_kv_desc {
   int mode;
   int split_tokens;
   lr_dtype_t cache_scale_dtype;  /* lr_latent_kv_decode_q8 only: LR_F16 or LR_F32 */
+  float rope_base;               /* LR_KV_RECONSTRUCT only; 0 = no rotary embedding */
 } lr_latent_kv_desc_t;
 
 /*
@@ -389,6 +415,26 @@ LR_API lr_status_t lr_latent_kv_workspace_size(const lr_latent_kv_desc_t* desc, 
 LR_API lr_status_t lr_latent_kv_decode_q8(const lr_latent_kv_desc_t* desc, const void* q, const int8_t* C_K,
                                           const void* s_K, const int8_t* C_V, const void* s_V, const int* seq_lens,
                                           void* out, void* ws, size_t ws_bytes, lr_stream_t stream);
+
+/*
+ * The latent producer of the per-head caches (WSVD "Fine-Grained Per-Head
+ * SVD": the cache keeps the latent x A_Kh of each head instead of its key, and
+ * x A_Vh instead of its value): one GEMV over all heads' first factors at
+ * once, whose outputs are written straight into the caches at each
+ * sequence's new position.
+ *   A_KV  bf16 [2 * heads * rank, hidden], latent-major: row h * rank + j is
+ *         column j of A_Kh, row (heads + h) * rank + j column j of A_Vh
+ *   x     bf16 [batch, hidden], the new token of each sequence
+ *   pos   int32 [batch] (device): the position written for sequence b
+ *         (normally seq_lens[b] before it is incremented); a position outside
+ *         [0, max_ctx) writes nothing for that sequence
+ *   C_K, C_V  bf16 [batch, heads, max_ctx, rank], updated in place at
+ *         [b, :, pos[b], :]; nothing else is written
+ * Only desc->batch, heads, rank and max_ctx are read.  Limits: hidden a
+ * multiple of 16 with hidden * 2 <= 32 KiB.  No workspace.
+ */
+LR_API lr_status_t lr_latent_kv_append(const lr_latent_kv_desc_t* desc, const void* A_KV, int hidden, const void* x,
+                                       const int* pos, void* C_K, void* C_V, lr_stream_t stream);
 
 /*
  * Standard single-query flash decoding over full K/V caches: the uncompressed
@@ -479,6 +525,17 @@ LR_API lr_status_t lr_check_device_error(lr_stream_t stream, int* err);
  * hanging.  Process-wide.
  */
 LR_API lr_status_t lr_set_wait_timeout_us(unsigned int us);
+
+/*
+ * Smallest batch at which lr_linear, lr_linear_grouped, lr_linear_chain (bf16
+ * or int8 factors, weight-only) and lr_swiglu_ffn switch from the CUDA-core
+ * decode kernels to the tensor-core path; 0 restores the default (9 for both:
+ * the CUDA-core kernels take at most 8 tokens per pass of the weights).
+ * Process-wide, for calls issued after this one; the workspace sizes reported
+ * afterwards follow the setting.  A tuning knob: both paths compute the same
+ * products (see lr_linear and lr_swiglu_ffn for their precision).
+ */
+LR_API lr_status_t lr_set_tensor_core_min_batch(int linear, int ffn);
 
 /* Static string for a status code. */
 LR_API const char* lr_status_string(lr_status_t status);

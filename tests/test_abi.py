@@ -42,13 +42,21 @@ def _ws(lib, d, batch, w8a8=0):
 
 
 def test_linear_workspace_sizes(lib):
-    # barrier words + three accumulator sets of min(batch, 8) x d_out floats (64-rounded)
+    # completion counters (256 bytes) + min(batch, 8) x d_out fp32 accumulators (8-rounded)
     st, n = _ws(lib, _desc(), 1)
-    assert st == L.LR_OK and n == 256 + 3 * 4096 * 4
-    st, n8 = _ws(lib, _desc(), 16)
-    assert st == L.LR_OK and n8 == 256 + 3 * 8 * 4096 * 4
+    assert st == L.LR_OK and n == 256 + 4096 * 4
+    st, n8 = _ws(lib, _desc(), 8)
+    assert st == L.LR_OK and n8 == 256 + 8 * 4096 * 4
+    # bf16 above batch 8 (tensor cores): z [rank, cols] and two y sets [d_out, cols], cols = 8-rounded
+    # min(batch, 32); the larger of the two paths' needs
+    st, n16 = _ws(lib, _desc(), 16)
+    assert st == L.LR_OK and n16 == 256 + (1024 + 2 * 4096) * 16 * 4
+    st, n40 = _ws(lib, _desc(), 40)
+    assert st == L.LR_OK and n40 == 256 + (1024 + 2 * 4096) * 32 * 4
+    st, n16f = _ws(lib, _desc(w_dtype=L.LR_F32), 16)
+    assert st == L.LR_OK and n16f == 256 + 8 * 4096 * 4
     st, n3 = _ws(lib, _desc(d_out=8), 3)
-    assert st == L.LR_OK and n3 == 256 + 3 * 64 * 4
+    assert st == L.LR_OK and n3 == 256 + 24 * 4
     st, _ = _ws(lib, _desc(w_dtype=L.LR_I8), 1)
     assert st == L.LR_ERR_INVALID_ARG  # int8 needs scales
     st, n = _ws(lib, _desc(w_dtype=L.LR_I8, scale_A=FAKE, scale_B=FAKE), 2048, 1)
@@ -86,7 +94,7 @@ def test_grouped_validation(lib):
     arr = (L.FactorDesc * 3)(_desc(), _desc(d_out=1024), _desc(rank=512))
     n = ctypes.c_size_t(0)
     assert lib.lr_linear_grouped_workspace_size(arr, 3, 1, ctypes.byref(n)) == L.LR_OK
-    assert n.value == 256 + 3 * (4096 + 1024 + 4096) * 4
+    assert n.value == 256 + (4096 + 1024 + 4096) * 4
 
 
 def _ffn(**kw):
@@ -116,7 +124,7 @@ def test_ffn_validation_and_workspace(lib):
 
 def _kv(**kw):
     d = dict(batch=8, heads=32, head_dim=128, rank=32, max_ctx=4096, scale=128 ** -0.5, B_K=FAKE, B_V=FAKE,
-             mode=L.LR_KV_ABSORBED, split_tokens=0, cache_scale_dtype=L.LR_F16)
+             mode=L.LR_KV_ABSORBED, split_tokens=0, cache_scale_dtype=L.LR_F16, rope_base=0.0)
     d.update(kw)
     return L.LatentKvDesc(**d)
 
@@ -154,7 +162,7 @@ def test_chain_validation_and_workspace(lib):
     arr = (L.ChainStep * 3)(_step(3), _step(1, 0, 2), _step(3, 1, 0))
     n = ctypes.c_size_t(0)
     assert lib.lr_linear_chain_workspace_size(arr, 3, 1, ctypes.byref(n)) == L.LR_OK
-    assert n.value == 256 + 3 * 3 * 4096 * 4
+    assert n.value == 256 + (3 + 1 + 3) * 4096 * 4     # counters + every step's own accumulators
     bad = (L.ChainStep * 2)(_step(1), _step(1, 1, 0))            # input from itself
     assert lib.lr_linear_chain(bad, 2, FAKE, 1, FAKE, 1 << 24, None) == L.LR_ERR_INVALID_ARG
     bad = (L.ChainStep * 2)(_step(1), _step(1, 0, 3))            # no such output
@@ -244,3 +252,35 @@ def test_latent_kv_q8_validation(lib):
                                       None) == L.LR_ERR_UNSUPPORTED
     assert lib.lr_latent_kv_decode_q8(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 16,
                                       None) == L.LR_ERR_WORKSPACE
+
+
+def test_latent_kv_reconstruct_mode_validation(lib):
+    # the on-chip reconstruction mode takes a rotary base; the absorbed form refuses one
+    n = ctypes.c_size_t(0)
+    rec = _kv(mode=L.LR_KV_RECONSTRUCT, rope_base=10000.0)
+    assert lib.lr_latent_kv_workspace_size(ctypes.byref(rec), ctypes.byref(n)) == L.LR_OK
+    assert n.value == 8 * 32 * (4096 // 256) * 34 * 4 + 8 * 32 * 32 * 4
+    for bad, code in ((_kv(rope_base=10000.0), L.LR_ERR_UNSUPPORTED),
+                      (_kv(mode=L.LR_KV_RECONSTRUCT, rope_base=-1.0), L.LR_ERR_INVALID_ARG),
+                      (_kv(mode=L.LR_KV_RECONSTRUCT, rope_base=float("nan")), L.LR_ERR_INVALID_ARG),
+                      (_kv(mode=L.LR_KV_RECONSTRUCT, split_tokens=512), L.LR_ERR_UNSUPPORTED),
+                      (_kv(mode=L.LR_KV_RECONSTRUCT, batch=4096, heads=1024, max_ctx=1024), L.LR_ERR_UNSUPPORTED),
+                      (_kv(mode=7), L.LR_ERR_UNSUPPORTED)):
+        assert lib.lr_latent_kv_decode(ctypes.byref(bad), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1 << 30,
+                                       None) == code
+    # int8 caches have no reconstruct mode
+    assert lib.lr_latent_kv_decode_q8(ctypes.byref(rec), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1 << 30,
+                                      None) == L.LR_ERR_UNSUPPORTED
+    assert lib.lr_latent_kv_decode(ctypes.byref(rec), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 16,
+                                   None) == L.LR_ERR_WORKSPACE
+
+
+def test_latent_kv_append_validation(lib):
+    d = _kv()
+    assert lib.lr_latent_kv_append(ctypes.byref(d), None, 4096, FAKE, FAKE, FAKE, FAKE, None) == L.LR_ERR_INVALID_ARG
+    assert lib.lr_latent_kv_append(ctypes.byref(d), FAKE, 0, FAKE, FAKE, FAKE, FAKE, None) == L.LR_ERR_INVALID_ARG
+    assert lib.lr_latent_kv_append(ctypes.byref(d), FAKE, 4100, FAKE, FAKE, FAKE, FAKE, None) == L.LR_ERR_UNSUPPORTED
+    assert lib.lr_latent_kv_append(ctypes.byref(d), FAKE, 32768, FAKE, FAKE, FAKE, FAKE, None) == L.LR_ERR_UNSUPPORTED
+    assert lib.lr_latent_kv_append(ctypes.byref(d), FAKE, 4096, FAKE, MIS, FAKE, FAKE, None) == L.LR_ERR_MISALIGNED
+    assert lib.lr_latent_kv_append(ctypes.byref(_kv(batch=0)), FAKE, 4096, FAKE, FAKE, FAKE, FAKE,
+                                   None) == L.LR_ERR_INVALID_ARG

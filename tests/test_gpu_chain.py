@@ -53,8 +53,8 @@ def test_decode_stack_chain(cuda_device, layers4, batch):
 def test_chain_older_inputs_against_oracle(cuda_device, layers4):
     L0, L1 = layers4[0], layers4[1]
     x = synth.make_activations(2, 4096, seed=6, key=(71,))
-    # step 1 reads step 0's second output (at fp32, the step right before);
-    # step 2 reads step 0's first output two steps back (its stored bf16 output)
+    # step 1 reads step 0's second output, step 2 step 0's first output two steps
+    # back (both at fp32, from step 0's accumulators)
     steps = [lr.ChainStep([_fac(L0["q"]), _fac(L0["v"])]), lr.ChainStep([_fac(L0["o"])], 0, 1),
              lr.ChainStep([_fac(L1["k"])], 0, 0)]
     outs = lr.lr_linear_chain(steps, dev(x))

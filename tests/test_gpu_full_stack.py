@@ -1,7 +1,9 @@
 """GPU parity at full size, in the launch the bench times: the 32-layer
 Llama-2-7B-shaped low-rank Q/K/V/O decode stack as one lr_linear_chain call
-(64 dependent steps, batch 1), every output of every layer against the fp64
-oracle run layer by layer on the same stored factors.
+at batch 1 (CUDA cores: 96 steps, V / Q and K / O per layer, as the bench
+times it) and 16 (tensor cores: 64 steps, Q/K/V / O per layer), every
+output of every layer against the fp64 oracle run layer by layer on the same
+stored factors.
 """
 import pytest
 import torch
@@ -24,18 +26,31 @@ def _oracle(f, x64):
     return lowrank.lr_linear(x64, f["At"].double().numpy().T, f["B"].double().numpy())
 
 
-def test_full_decode_stack_chain(cuda_device):
+@pytest.fixture(scope="module")
+def layers32():
     ranks = synth.attention_ranks(0)
-    layers = [synth.make_attention_layer(l, ranks, seed=0) for l in range(LAYERS)]
-    x = synth.make_activations(1, HIDDEN, seed=0, key=(90,))
-    qkv = [[torch.empty(1, HIDDEN, dtype=torch.bfloat16, device="cuda") for _ in range(3)] for _ in range(LAYERS)]
-    outs = [torch.empty(1, HIDDEN, dtype=torch.bfloat16, device="cuda") for _ in range(LAYERS)]
+    return [synth.make_attention_layer(l, ranks, seed=0) for l in range(LAYERS)]
+
+
+@pytest.mark.parametrize("batch", [1, 16])
+def test_full_decode_stack_chain(cuda_device, layers32, batch):
+    layers = layers32
+    x = synth.make_activations(batch, HIDDEN, seed=0, key=(90,) if batch == 1 else (90, batch))
+    qkv = [[torch.empty(batch, HIDDEN, dtype=torch.bfloat16, device="cuda") for _ in range(3)] for _ in range(LAYERS)]
+    outs = [torch.empty(batch, HIDDEN, dtype=torch.bfloat16, device="cuda") for _ in range(LAYERS)]
     steps = []
     for l, L in enumerate(layers):
-        steps.append(lr.ChainStep([_fac(L["q"]), _fac(L["k"]), _fac(L["v"])], -1 if l == 0 else 2 * l - 1, 0,
-                                  qkv[l]))
-        steps.append(lr.ChainStep([_fac(L["o"])], 2 * l, 2, [outs[l]]))
-    ws = lr.workspace(lr.lr_linear_chain_workspace_size(steps, 1), torch.device("cuda"))
+        if batch < 9:
+            # the bench's layout on the CUDA-core path: V, then Q and K, then O (reads V)
+            src = -1 if l == 0 else 3 * l - 1
+            steps.append(lr.ChainStep([_fac(L["v"])], src, 0, [qkv[l][2]]))
+            steps.append(lr.ChainStep([_fac(L["q"]), _fac(L["k"])], src, 0, qkv[l][:2]))
+            steps.append(lr.ChainStep([_fac(L["o"])], 3 * l, 0, [outs[l]]))
+        else:
+            steps.append(lr.ChainStep([_fac(L["q"]), _fac(L["k"]), _fac(L["v"])], -1 if l == 0 else 2 * l - 1, 0,
+                                      qkv[l]))
+            steps.append(lr.ChainStep([_fac(L["o"])], 2 * l, 2, [outs[l]]))
+    ws = lr.workspace(lr.lr_linear_chain_workspace_size(steps, batch), torch.device("cuda"))
     lr.lr_linear_chain(steps, dev(x), ws=ws)
     torch.cuda.synchronize()
     assert lr.lr_check_device_error() == 0
@@ -51,4 +66,4 @@ def test_full_decode_stack_chain(cuda_device):
             assert err < NORMWISE_TOL, (l, err)
         x64 = o                          # the next layer reads O (fp64 here, fp32 in the chain)
     assert int(ws.count_nonzero()) == 0
-    print(f"worst normwise error over 128 outputs: {worst:.2e}")
+    print(f"batch {batch}: worst normwise error over 128 outputs: {worst:.2e}")
