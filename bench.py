@@ -7,8 +7,8 @@ stack of 32 layers whose Q/K/V/O projections are truncated-SVD factorised
 reduction, batch 1).  Per layer, Q, K and V are computed from the layer input
 x; the O projection reads the V output (single-token attention returns V
 exactly) and its output is the next layer's input.  The whole stack is one
-lr_linear_chain call, one persistent launch per step, of three chain steps per
-layer (V; Q and K; O), each waiting only for the step it reads.
+lr_linear_chain call: one persistent launch per step, two chain steps per
+layer (Q/K/V; O), each waiting only for the step it reads.
 
 The 32 layers hold 2.58 GB of factors, far above the 126 MB L2, so every step
 streams them from HBM (no L2 flush needed).  Timing: W untimed warm-up steps,
@@ -60,7 +60,7 @@ METRIC = "decode-layer µs & achieved HBM GB/s (% of B200 roofline) at batch 1; 
 LAYERS, HIDDEN = 32, 4096
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
-TC_MIN = [9, 9]   # smallest batch on the tensor-core path (linears, FFN): the library's default
+TC_MIN = [4, 1]   # smallest batch on the tensor-core path (linears, FFN): the library's defaults
 ROW_IDS = ("c1", "c2b4", "c2b16", "c2dense", "c3b1", "c3b8", "c3b32", "c3dense", "c4k4", "c4k16", "c4k32",
            "c4rk4", "c4rk16", "c4rk32", "c4app", "c4full4", "c4full16", "c4full32", "c4q8k4", "c4q8k16", "c4q8k32",
            "c5")
@@ -337,11 +337,11 @@ def build_layers(device, layers: int):
     return ranks, out
 
 
-def stack_steps(lr, layers, batch, device, split_v: bool = True):
-    """The decode stack as one chain.  split_v (the CUDA-core path, one persistent launch): three
-    steps per layer, V (input: the previous O), then Q and K (same input), then O (input: V); O waits
-    only for V, so Q and K stream while V's result is handed over, and the next layer's V waits for
-    O.  Otherwise (the tensor-core path, a sequence of launches): Q/K/V in one step, then O."""
+def stack_steps(lr, layers, batch, device, split_v: bool = False):
+    """The decode stack as one chain: per layer Q/K/V in one step (input: the previous O), then O
+    (input: V).  split_v: three steps per layer instead, V, then Q and K, then O (reads V), so O waits
+    only for V; measured slower on B200 (0.97 against 0.80 ms per step at batch 1: the third step's
+    input round trip and latent hand-off cost more than the wait it hides), kept for comparison."""
     import torch
 
     def out():
@@ -412,7 +412,7 @@ def run_ours(args) -> None:
     if args.tc_min_batch:
         lin, ffn = (int(v) for v in args.tc_min_batch.split(","))
         lr.lr_set_tensor_core_min_batch(lin, ffn)
-        TC_MIN[0], TC_MIN[1] = lin or 9, ffn or 9
+        TC_MIN[0], TC_MIN[1] = lin or 4, ffn or 1
     only = set(filter(None, args.only.split(",")))
     want_headline = not only or "headline" in only
     want_cpu = rank == 0 and world == 1 and not args.no_cpu_baseline
@@ -421,7 +421,7 @@ def run_ours(args) -> None:
     out = None
     if want_headline:
         x0 = synth.make_activations(batch, HIDDEN, seed=0, key=(90,)).to(device)
-        steps = stack_steps(lr, layers, batch, device, split_v=batch < TC_MIN[0])
+        steps = stack_steps(lr, layers, batch, device)
         ws = lr.workspace(lr.lr_linear_chain_workspace_size(steps, batch), device)
 
         def step():
@@ -578,16 +578,17 @@ def row_c1(lr, L, synth, device, want_cpu):
 
 def row_c2(lr, L, synth, device, ranks, layers, batch, want_cpu):
     import torch
-    steps = stack_steps(lr, layers, batch, device, split_v=batch < TC_MIN[0])
+    steps = stack_steps(lr, layers, batch, device)
     ws = lr.workspace(lr.lr_linear_chain_workspace_size(steps, batch), device)
     x0 = synth.make_activations(batch, HIDDEN, seed=0, key=(90, batch)).to(device)
     ms = time_graph(lambda i: lr.lr_linear_chain(steps, x0, ws=ws), 20)
     alg = algorithmic_bytes_per_step(ranks, batch, LAYERS)
     passes = (batch + 31) // 32
     tensor_cores = batch >= TC_MIN[0]
-    launches = passes * (3 * len(steps) + 1) if tensor_cores else (batch + 7) // 8
+    launches = passes * (2 * len(steps) + 1) if tensor_cores else (batch + 7) // 8
     note = (f"{launches} launches per step: per dependent step two tcgen05 products (z = x A, y = z B, weights "
-            f"as M, tokens as N) and a finalize; every factor byte streamed once per pass of 32 tokens"
+            f"as M, tokens as N; the first also finalizes the step before), one finalize at the end; every "
+            f"factor byte streamed once per pass of 32 tokens"
             if tensor_cores else f"{launches} launch(es) of chain_kernel per step; each streams every factor byte once")
     arr, lib = lr.ops._chain_array(steps), L.load()
     xh = synth.make_activations(batch, HIDDEN, seed=0, key=(90, batch)).pin_memory()
@@ -993,6 +994,21 @@ def row_c4full(lr, L, synth, device, ctx, want_cpu):
     return row
 
 
+class _Nvtx:
+    """An NVTX range around one row (visible in a profiler's timeline; free without one)."""
+
+    def __init__(self, name):
+        self.name = name
+
+    def __enter__(self):
+        import torch
+        torch.cuda.nvtx.range_push(self.name)
+
+    def __exit__(self, *exc):
+        import torch
+        torch.cuda.nvtx.range_pop()
+
+
 def run_rows(args, lr, L, synth, device, ranks, layers, only) -> list:
     import torch
     want_cpu = not args.no_cpu_baseline
@@ -1002,19 +1018,22 @@ def run_rows(args, lr, L, synth, device, ranks, layers, only) -> list:
     clocks.wait_first_sample()
     for rid in sel:
         if rid.startswith("c2b"):
-            rows.append(row_c2(lr, L, synth, device, ranks, layers, int(rid[3:]), want_cpu))
+            with _Nvtx(rid):
+                rows.append(row_c2(lr, L, synth, device, ranks, layers, int(rid[3:]), want_cpu))
     del layers
     torch.cuda.empty_cache()
     if "c1" in sel:
         rows.insert(0, row_c1(lr, L, synth, device, want_cpu))
     if "c2dense" in sel:
-        rows.append(row_c2dense(lr, L, synth, device, want_cpu))
+        with _Nvtx("c2dense"):
+            rows.append(row_c2dense(lr, L, synth, device, want_cpu))
         torch.cuda.empty_cache()
     ffn = None
     for rid in sel:
         if rid.startswith("c3b"):
             ffn = ffn or synth.make_hybrid_ffn(seed=0)
-            rows.append(row_c3(lr, L, synth, device, ffn, int(rid[3:]), want_cpu))
+            with _Nvtx(rid):
+                rows.append(row_c3(lr, L, synth, device, ffn, int(rid[3:]), want_cpu))
             torch.cuda.empty_cache()
     if "c3dense" in sel:
         dense = synth.make_hybrid_ffn(seed=0, n_lr=0, rotate=False)
@@ -1026,22 +1045,28 @@ def run_rows(args, lr, L, synth, device, ranks, layers, only) -> list:
         torch.cuda.empty_cache()
     for rid in sel:
         if rid.startswith("c4k"):
-            rows.append(row_c4(lr, L, synth, device, int(rid[3:]) * 1024, want_cpu))
+            with _Nvtx(rid):
+                rows.append(row_c4(lr, L, synth, device, int(rid[3:]) * 1024, want_cpu))
             torch.cuda.empty_cache()
         elif rid.startswith("c4rk"):
-            rows.append(row_c4(lr, L, synth, device, int(rid[4:]) * 1024, want_cpu, rope_base=10000.0))
+            with _Nvtx(rid):
+                rows.append(row_c4(lr, L, synth, device, int(rid[4:]) * 1024, want_cpu, rope_base=10000.0))
             torch.cuda.empty_cache()
         elif rid == "c4app":
-            rows.append(row_c4app(lr, L, synth, device, want_cpu))
+            with _Nvtx("c4app"):
+                rows.append(row_c4app(lr, L, synth, device, want_cpu))
             torch.cuda.empty_cache()
         elif rid.startswith("c4full"):
-            rows.append(row_c4full(lr, L, synth, device, int(rid[6:]) * 1024, want_cpu))
+            with _Nvtx(rid):
+                rows.append(row_c4full(lr, L, synth, device, int(rid[6:]) * 1024, want_cpu))
             torch.cuda.empty_cache()
         elif rid.startswith("c4q8k"):
-            rows.append(row_c4q8(lr, L, synth, device, int(rid[5:]) * 1024, want_cpu))
+            with _Nvtx(rid):
+                rows.append(row_c4q8(lr, L, synth, device, int(rid[5:]) * 1024, want_cpu))
             torch.cuda.empty_cache()
     if "c5" in sel:
-        rows.append(row_c5(lr, L, synth, device, want_cpu))
+        with _Nvtx("c5"):
+            rows.append(row_c5(lr, L, synth, device, want_cpu))
     clk = clocks.stop()
     check_device(lr)
     by = {r["row"]: r for r in rows}

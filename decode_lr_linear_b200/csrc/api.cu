@@ -127,8 +127,14 @@ size_t chain_step_floats(const HostStep& h, int batch) {
 // Tokens per pass of the weights, and the accumulator columns of one pass.
 constexpr int kTcMaxPass = 32;
 // Smallest batch that takes the tensor-core path (lr_set_tensor_core_min_batch).
-std::atomic<int> g_tc_min_linear{kMaxDecodeChunk + 1};
-std::atomic<int> g_tc_min_ffn{kMaxDecodeChunk + 1};
+// Measured on B200 (7B shapes): from batch 4 the tensor-core path streams the
+// factorised linears faster (stack 0.43 against 0.32 of HBM); the int8 FFN is
+// faster there at every batch (batch 1: 41 against 47.5 us; batch 8: 46 against
+// 217 us), its CUDA-core kernels being bound by int8-to-float conversion.
+constexpr int kTcDefaultMinBatchLinear = 4;
+constexpr int kTcDefaultMinBatchFfn = 1;
+std::atomic<int> g_tc_min_linear{kTcDefaultMinBatchLinear};
+std::atomic<int> g_tc_min_ffn{kTcDefaultMinBatchFfn};
 bool use_tc_path(const HostStep* steps, int batch) {
   return batch >= g_tc_min_linear.load(std::memory_order_relaxed) &&
          (steps[0].d[0].w_dtype == LR_BF16 || steps[0].d[0].w_dtype == LR_I8);
@@ -138,23 +144,28 @@ int tc_cols(int batch) { return int(round_up(size_t(std::min(batch, kTcMaxPass))
 
 // Workspace of the tensor-core path: z accumulator [sum of a step's active ranks, cols]
 // and two y accumulator sets [sum of a step's d_out, cols], fp32, zero on entry and exit.
+// Row length of projection p's latent accumulator (token-major, 8-float aligned rows).
+inline size_t tc_zld(const lr_factor_desc_t& d) { return round_up(size_t(active(&d)), 8); }
+
 void tc_sizes(const HostStep* steps, int n_steps, size_t* zmax, size_t* ymax) {
   *zmax = 0;
   *ymax = 0;
   for (int s = 0; s < n_steps; ++s) {
     size_t z = 0, y = 0;
     for (int p = 0; p < steps[s].n; ++p) {
-      z += size_t(active(&steps[s].d[p]));
+      z += tc_zld(steps[s].d[p]);
       y += size_t(steps[s].d[p].d_out);
     }
     *zmax = std::max(*zmax, z);
     *ymax = std::max(*ymax, y);
   }
 }
+// + per-token maxima of a step's input and of its latents (int8 factors)
+constexpr size_t kTcAmaxBytes = 5 * kTcMaxPass * 4 + 96;
 size_t tc_ws_bytes(const HostStep* steps, int n_steps, int batch) {
   size_t zm, ym;
   tc_sizes(steps, n_steps, &zm, &ym);
-  return kTicketBytes + (zm + 2 * ym) * size_t(tc_cols(batch)) * 4;
+  return kTicketBytes + kTcAmaxBytes + (2 * zm + 2 * ym) * size_t(tc_cols(batch)) * 4;
 }
 
 size_t chain_ws_bytes(const HostStep* steps, int n_steps, int batch, bool allow_tc = true) {
@@ -256,12 +267,24 @@ cudaError_t tc_product(TcMaps& maps, TcGemvParams& g, int sms, bool i8, cudaStre
 //                                 accumulator, or an older step's stored output)
 //   product 2: y_p += B_p^T z_p  (fp32 z split into bf16 high and low parts)
 //   finalize:  y_p (bf16) from the accumulator; zero z and the other y set.
+// The chain on the tensor cores, per pass of up to kTcMaxPass tokens and per step s:
+//   (int8 factors: per-token max of the input)
+//   product 1: z_p += x A_p into latent set s % 2; its units first finalize step
+//              s-1 (bf16 outputs from y set (s-1) % 2) and clear y set s % 2,
+//              latent set (s-1) % 2 and the latent maxima, none of which it reads
+//   (int8 factors: per-token max of each latent)
+//   product 2: y_p += z_p B_p into y set s % 2 (units first clear the input maximum)
+// and after the last step one finalize launch.  All accumulators are token-major
+// fp32; the input is the chain input, the previous step's y set (fp32), or an
+// older step's stored bf16 output.
 lr_status_t run_chain_tc(const HostStep* steps, int n_steps, const void* x, int batch, void* ws, cudaStream_t stream) {
   size_t zmax, ymax;
   tc_sizes(steps, n_steps, &zmax, &ymax);
   const int cols = tc_cols(batch);
-  float* zacc = reinterpret_cast<float*>(reinterpret_cast<char*>(ws) + kTicketBytes);
-  float* yacc[2] = {zacc + zmax * cols, zacc + (zmax + ymax) * cols};
+  float* amax = reinterpret_cast<float*>(reinterpret_cast<char*>(ws) + kTicketBytes);  // [5][kTcMaxPass]
+  float* acc0 = reinterpret_cast<float*>(reinterpret_cast<char*>(ws) + kTicketBytes + kTcAmaxBytes);
+  float* zacc[2] = {acc0, acc0 + zmax * cols};
+  float* yacc[2] = {acc0 + 2 * zmax * cols, acc0 + (2 * zmax + ymax) * cols};
   int* err = device_error_word();
   const int sms = sm_count_current();
   const bool i8 = steps[0].d[0].w_dtype == LR_I8;
@@ -269,19 +292,26 @@ lr_status_t run_chain_tc(const HostStep* steps, int n_steps, const void* x, int 
   int x_width = 0;
   for (int s = 0; s < n_steps; ++s)
     if (steps[s].input_step < 0) x_width = steps[s].d[0].d_in;
+  // finalize of step t of this pass: its bf16 outputs from y set t % 2
+  auto set_targets = [&](TcFinalizeParams& f, int t, int b0, int nb) {
+    const HostStep& h = steps[t];
+    f.nt = h.n;
+    f.nb = nb;
+    size_t yoff = 0;
+    for (int p = 0; p < h.n; ++p) {
+      f.t[p].acc = yacc[t & 1] + yoff * cols;
+      f.t[p].y = reinterpret_cast<char*>(h.y[p]) + size_t(b0) * h.d[p].d_out * 2;
+      f.t[p].M = h.d[p].d_out;
+      yoff += size_t(h.d[p].d_out);
+    }
+  };
   for (int b0 = 0; b0 < batch; b0 += kTcMaxPass) {
     const int nb = std::min(kTcMaxPass, batch - b0);
     const int nh = int(round_up(size_t(nb), 8));
     for (int s = 0; s < n_steps; ++s) {
       const HostStep& h = steps[s];
-      // ---- product 1 ----
-      TcMaps maps;
-      TcGemvParams g;
-      std::memset(&maps, 0, sizeof(maps));
-      std::memset(&g, 0, sizeof(g));
-      g.nseg = h.n;
-      g.nb = nb;
-      g.err = err;
+      float* z = zacc[s & 1];
+      // ---- the step's input ----
       const void* act;
       int act_kind, act_ld;
       if (h.input_step < 0) {
@@ -293,15 +323,43 @@ lr_status_t run_chain_tc(const HostStep* steps, int n_steps, const void* x, int 
         for (int q = 0; q < h.input_proj; ++q) off += size_t(steps[s - 1].d[q].d_out);
         act = yacc[(s - 1) & 1] + off * cols;
         act_kind = 1;
-        act_ld = cols;
+        act_ld = steps[s - 1].d[h.input_proj].d_out;
       } else {
         const HostStep& src = steps[h.input_step];
         act = reinterpret_cast<const char*>(src.y[h.input_proj]) + size_t(b0) * src.d[h.input_proj].d_out * 2;
         act_kind = 0;
         act_ld = src.d[h.input_proj].d_out;
       }
+      cudaError_t e;
+      if (i8) {  // per-token scales of the input's int8 codes (zero on entry)
+        TcAmaxParams a;
+        std::memset(&a, 0, sizeof(a));
+        a.nsrc = 1;
+        a.nb = nb;
+        a.src[0] = TcAmaxSrc{act, act_kind, h.d[0].d_in, act_ld, amax};
+        e = launch_tc_amax(a, stream);
+        if (e != cudaSuccess) return from_cuda(e);
+      }
+      // ---- product 1: z_p = x A_p ----
+      TcMaps maps;
+      TcGemvParams g;
+      std::memset(&maps, 0, sizeof(maps));
+      std::memset(&g, 0, sizeof(g));
+      g.nseg = h.n;
+      g.nb = nb;
+      g.err = err;
       g.hilo = (i8 || act_kind == 1) ? 1 : 0;
       g.N = g.hilo ? std::max(16, 2 * nh) : int(round_up(size_t(nb), 16));
+      if (s > 0) {
+        set_targets(g.pre, s - 1, b0, nb);
+        g.pre.zero[0] = yacc[s & 1];                 // step s-2's set, finalized by the previous launch
+        g.pre.zero_floats[0] = ymax * cols;
+        g.pre.zero[1] = zacc[(s - 1) & 1];           // consumed by step s-1's second product
+        g.pre.zero_floats[1] = zmax * cols;
+        g.pre.zero[2] = amax + kTcMaxPass;           // the latent maxima of step s-1
+        g.pre.zero_floats[2] = 4 * kTcMaxPass;
+        g.pre.nz = 3;
+      }
       size_t zoff = 0;
       for (int p = 0; p < h.n; ++p) {
         const lr_factor_desc_t& d = h.d[p];
@@ -309,20 +367,40 @@ lr_status_t run_chain_tc(const HostStep* steps, int n_steps, const void* x, int 
         TcSeg& sg = g.seg[p];
         sg.row_scale = i8 ? d.scale_A : nullptr;
         sg.row_scale_f16 = scale_f16;
+        sg.tok_amax = amax;
         sg.M = active(&d);
         sg.K = d.d_in;
         sg.a_mn_major = 0;
         sg.act = act;
         sg.act_kind = act_kind;
         sg.act_ld = act_ld;
-        sg.out = zacc + zoff * cols;
-        sg.out_ld = cols;
-        zoff += size_t(sg.M);
+        sg.out = z + zoff * cols;
+        sg.out_ld = int(tc_zld(d));
+        zoff += tc_zld(d);
       }
-      cudaError_t e = tc_product(maps, g, sms, i8, stream);
+      e = tc_product(maps, g, sms, i8, stream);
       if (e != cudaSuccess) return from_cuda(e);
-      // ---- product 2 ----
+      if (i8) {  // per-token scales of each projection's latent
+        TcAmaxParams a;
+        std::memset(&a, 0, sizeof(a));
+        a.nsrc = h.n;
+        a.nb = nb;
+        zoff = 0;
+        for (int p = 0; p < h.n; ++p) {
+          a.src[p] = TcAmaxSrc{z + zoff * cols, 1, active(&h.d[p]), int(tc_zld(h.d[p])), amax + (p + 1) * kTcMaxPass};
+          zoff += tc_zld(h.d[p]);
+        }
+        e = launch_tc_amax(a, stream);
+        if (e != cudaSuccess) return from_cuda(e);
+      }
+      // ---- product 2: y_p = z_p B_p ----
       std::memset(&maps, 0, sizeof(maps));
+      std::memset(&g.pre, 0, sizeof(g.pre));
+      if (i8) {
+        g.pre.zero[0] = amax;                        // the input maximum, read by product 1 only
+        g.pre.zero_floats[0] = kTcMaxPass;
+        g.pre.nz = 1;
+      }
       g.hilo = 1;
       g.N = std::max(16, 2 * nh);
       zoff = 0;
@@ -333,46 +411,34 @@ lr_status_t run_chain_tc(const HostStep* steps, int n_steps, const void* x, int 
         TcSeg& sg = g.seg[p];
         sg.row_scale = i8 ? d.scale_B : nullptr;
         sg.row_scale_f16 = scale_f16;
+        sg.tok_amax = amax + (p + 1) * kTcMaxPass;
         sg.M = d.d_out;
         sg.K = active(&d);
         sg.a_mn_major = 1;
-        sg.act = zacc + zoff * cols;
+        sg.act = z + zoff * cols;
         sg.act_kind = 1;
-        sg.act_ld = cols;
+        sg.act_ld = int(tc_zld(d));
         sg.out = yacc[s & 1] + yoff * cols;
-        sg.out_ld = cols;
-        zoff += size_t(sg.K);
-        yoff += size_t(sg.M);
+        sg.out_ld = d.d_out;
+        zoff += tc_zld(d);
+        yoff += size_t(d.d_out);
       }
       e = tc_product(maps, g, sms, i8, stream);
       if (e != cudaSuccess) return from_cuda(e);
-      // ---- finalize ----
-      TcFinalizeParams f;
-      std::memset(&f, 0, sizeof(f));
-      f.nt = h.n;
-      f.nb = nb;
-      f.ld = cols;
-      yoff = 0;
-      for (int p = 0; p < h.n; ++p) {
-        f.t[p].acc = yacc[s & 1] + yoff * cols;
-        f.t[p].y = reinterpret_cast<char*>(h.y[p]) + size_t(b0) * h.d[p].d_out * 2;
-        f.t[p].M = h.d[p].d_out;
-        yoff += size_t(h.d[p].d_out);
-      }
-      f.zero[0] = zacc;
-      f.zero_floats[0] = zmax * cols;
-      f.zero[1] = yacc[(s + 1) & 1];
-      f.zero_floats[1] = ymax * cols;
-      f.nz = 2;
-      e = launch_tc_finalize(f, sms, stream);
-      if (e != cudaSuccess) return from_cuda(e);
     }
-    // the last step's accumulator set, now read
+    // the last step: outputs (clearing its y set), its latent set, the other y set, the maxima
+    const int last = n_steps - 1;
     TcFinalizeParams f;
     std::memset(&f, 0, sizeof(f));
-    f.zero[0] = yacc[(n_steps - 1) & 1];
-    f.zero_floats[0] = ymax * cols;
-    f.nz = 1;
+    set_targets(f, last, b0, nb);
+    f.zero_targets = 1;
+    f.zero[0] = zacc[last & 1];
+    f.zero_floats[0] = zmax * cols;
+    f.zero[1] = yacc[(last + 1) & 1];
+    f.zero_floats[1] = ymax * cols;
+    f.zero[2] = amax;
+    f.zero_floats[2] = 5 * kTcMaxPass;
+    f.nz = 3;
     cudaError_t e = launch_tc_finalize(f, sms, stream);
     if (e != cudaSuccess) return from_cuda(e);
   }
@@ -488,8 +554,8 @@ extern "C" {
 
 lr_status_t lr_set_tensor_core_min_batch(int linear, int ffn) {
   if (linear < 0 || ffn < 0) return LR_ERR_INVALID_ARG;
-  g_tc_min_linear.store(linear ? linear : kMaxDecodeChunk + 1, std::memory_order_relaxed);
-  g_tc_min_ffn.store(ffn ? ffn : kMaxDecodeChunk + 1, std::memory_order_relaxed);
+  g_tc_min_linear.store(linear ? linear : kTcDefaultMinBatchLinear, std::memory_order_relaxed);
+  g_tc_min_ffn.store(ffn ? ffn : kTcDefaultMinBatchFfn, std::memory_order_relaxed);
   return LR_OK;
 }
 
@@ -670,11 +736,12 @@ static lr_status_t check_ffn(const lr_ffn_desc_t* d) {
   return LR_OK;
 }
 
-// Above batch 8 the FFN runs on the tensor cores (int8 weights, kind::i8):
-// accumulators z [rank], gu [2 n_lr], dd [2 n_dense], h [inter], y [hidden],
-// each x cols fp32 (cols = 8-rounded min(batch, 32)), zero on entry and exit.
-static size_t ffn_tc_rows(const lr_ffn_desc_t* d) {
-  return size_t(d->n_lr > 0 ? d->rank : 0) + 2 * size_t(d->inter) + size_t(d->inter) + size_t(d->hidden);
+// On the tensor-core path the FFN keeps token-major fp32 accumulators: z [rank],
+// gu [2 n_lr], dd [2 n_dense], h [inter], y [hidden] per token (rows 8-float
+// aligned) for cols tokens, zero on entry and exit, and three per-token maxima.
+static size_t ffn_tc_floats_per_token(const lr_ffn_desc_t* d) {
+  return round_up(size_t(d->n_lr > 0 ? d->rank : 0), 8) + 2 * size_t(d->inter) + round_up(size_t(d->inter), 8) +
+         size_t(d->hidden);
 }
 
 static size_t ffn_ws_bytes(const lr_ffn_desc_t* d, int batch) {
@@ -682,26 +749,33 @@ static size_t ffn_ws_bytes(const lr_ffn_desc_t* d, int batch) {
   const int n_dense = d->inter - d->n_lr;
   size_t b = kTicketBytes + round_up(size_t(chunk) * 2 * d->n_lr * 4, 256) + round_up(size_t(chunk) * n_dense * 4, 256) +
              round_up(size_t(chunk) * d->hidden * 4, 256);
-  if (use_tc_ffn(batch)) b = std::max(b, kTicketBytes + ffn_tc_rows(d) * size_t(tc_cols(batch)) * 4);
+  if (use_tc_ffn(batch))
+    b = std::max(b, kTicketBytes + kTcAmaxBytes + ffn_tc_floats_per_token(d) * size_t(tc_cols(batch)) * 4);
   return b;
 }
 
-// The hybrid FFN on the tensor cores, per pass of up to kTcMaxPass tokens:
+// The hybrid FFN on the tensor cores (int8 weights, kind::i8), per pass of up
+// to kTcMaxPass tokens:
+//   max |x|    per token (scales of x's int8 codes)
 //   product 1: z += A' x (low-rank latent) and dd += D x (dense gate/up), scaled per row
+//   max |z|    per token
 //   product 2: gu += B'^T z (low-rank gate/up), scaled per column of B'
-//   SwiGLU:    h = silu(g) u over both branches (clears gu, dd; zeroes z)
+//   SwiGLU:    h = silu(g) u over both branches and max |h| per token (clears gu, dd; zeroes z)
 //   product 3: y += W_down^T h, scaled per output column
 //   finalize:  y (bf16), clearing the y accumulator; zeroes h
 static lr_status_t run_ffn_tc(const lr_ffn_desc_t* d, const void* x, int batch, void* y, void* ws,
                               cudaStream_t stream) {
   const int cols = tc_cols(batch);
   const int n_dense = d->inter - d->n_lr;
-  const int rz = d->n_lr > 0 ? d->rank : 0;
-  float* zacc = reinterpret_cast<float*>(reinterpret_cast<char*>(ws) + kTicketBytes);
+  const int rz = d->n_lr > 0 ? int(round_up(size_t(d->rank), 8)) : 0;
+  const int hld = int(round_up(size_t(d->inter), 8));
+  float* amax = reinterpret_cast<float*>(reinterpret_cast<char*>(ws) + kTicketBytes);  // x, z, h
+  float* zacc = reinterpret_cast<float*>(reinterpret_cast<char*>(ws) + kTicketBytes + kTcAmaxBytes);
   float* gu = zacc + size_t(rz) * cols;
   float* dd = gu + size_t(2 * d->n_lr) * cols;
   float* h = dd + size_t(2 * n_dense) * cols;
-  float* yacc = h + size_t(d->inter) * cols;
+  float* yacc = h + size_t(hld) * cols;
+  float *ax = amax, *az = amax + kTcMaxPass, *ah = amax + 2 * kTcMaxPass;
   int* err = device_error_word();
   const int sms = sm_count_current();
   const int f16 = d->scale_dtype == LR_F16 ? 1 : 0;
@@ -711,7 +785,8 @@ static lr_status_t run_ffn_tc(const lr_ffn_desc_t* d, const void* x, int batch, 
     const int N = std::max(16, 2 * nh);
     const void* xb = reinterpret_cast<const char*>(x) + size_t(b0) * d->hidden * 2;
     auto seg = [&](TcGemvParams& g, TcMaps& maps, int i, const void* W, int rows, int cols_w, int mn, int M, int K,
-                   const void* act, int act_kind, int act_ld, float* out, const void* rs) -> bool {
+                   const void* act, int act_kind, int act_ld, float* out, int out_ld, const void* rs,
+                   const float* am) -> bool {
       if (!weight_map(&maps.m[i], W, rows, cols_w, mn, true)) return false;
       TcSeg& sg = g.seg[i];
       sg.M = M;
@@ -721,12 +796,20 @@ static lr_status_t run_ffn_tc(const lr_ffn_desc_t* d, const void* x, int batch, 
       sg.act_kind = act_kind;
       sg.act_ld = act_ld;
       sg.out = out;
-      sg.out_ld = cols;
+      sg.out_ld = out_ld;
       sg.row_scale = rs;
       sg.row_scale_f16 = f16;
+      sg.tok_amax = am;
       g.nseg = i + 1;
       return true;
     };
+    TcAmaxParams am;
+    std::memset(&am, 0, sizeof(am));
+    am.nsrc = 1;
+    am.nb = nb;
+    am.src[0] = TcAmaxSrc{xb, 0, d->hidden, d->hidden, ax};
+    cudaError_t e = launch_tc_amax(am, stream);
+    if (e != cudaSuccess) return from_cuda(e);
     TcMaps maps;
     TcGemvParams g;
     std::memset(&maps, 0, sizeof(maps));
@@ -736,16 +819,21 @@ static lr_status_t run_ffn_tc(const lr_ffn_desc_t* d, const void* x, int batch, 
     g.hilo = 1;
     g.err = err;
     int i = 0;
-    if (d->n_lr > 0 && !seg(g, maps, i++, d->A, d->rank, d->hidden, 0, d->rank, d->hidden, xb, 0, d->hidden, zacc, d->s_A))
+    if (d->n_lr > 0 &&
+        !seg(g, maps, i++, d->A, d->rank, d->hidden, 0, d->rank, d->hidden, xb, 0, d->hidden, zacc, rz, d->s_A, ax))
       return LR_ERR_CUDA;
-    if (n_dense > 0 &&
-        !seg(g, maps, i++, d->D, 2 * n_dense, d->hidden, 0, 2 * n_dense, d->hidden, xb, 0, d->hidden, dd, d->s_D))
+    if (n_dense > 0 && !seg(g, maps, i++, d->D, 2 * n_dense, d->hidden, 0, 2 * n_dense, d->hidden, xb, 0,
+                            d->hidden, dd, 2 * n_dense, d->s_D, ax))
       return LR_ERR_CUDA;
-    cudaError_t e = tc_product(maps, g, sms, true, stream);
+    e = tc_product(maps, g, sms, true, stream);
     if (e != cudaSuccess) return from_cuda(e);
     if (d->n_lr > 0) {
+      am.src[0] = TcAmaxSrc{zacc, 1, d->rank, rz, az};
+      e = launch_tc_amax(am, stream);
+      if (e != cudaSuccess) return from_cuda(e);
       std::memset(&maps, 0, sizeof(maps));
-      if (!seg(g, maps, 0, d->B, d->rank, 2 * d->n_lr, 1, 2 * d->n_lr, d->rank, zacc, 1, cols, gu, d->s_B))
+      if (!seg(g, maps, 0, d->B, d->rank, 2 * d->n_lr, 1, 2 * d->n_lr, d->rank, zacc, 1, rz, gu, 2 * d->n_lr, d->s_B,
+               az))
         return LR_ERR_CUDA;
       g.nseg = 1;
       e = tc_product(maps, g, sms, true, stream);
@@ -756,16 +844,18 @@ static lr_status_t run_ffn_tc(const lr_ffn_desc_t* d, const void* x, int batch, 
     sw.gu = gu;
     sw.dd = dd;
     sw.h = h;
+    sw.h_ld = hld;
+    sw.h_amax = ah;
     sw.n_lr = d->n_lr;
     sw.n_dense = n_dense;
     sw.nb = nb;
-    sw.cols = cols;
     sw.zero = rz ? zacc : nullptr;
-    sw.zero_floats = size_t(rz) * cols;
+    sw.zero_row = rz;
     e = launch_tc_swiglu(sw, sms, stream);
     if (e != cudaSuccess) return from_cuda(e);
     std::memset(&maps, 0, sizeof(maps));
-    if (!seg(g, maps, 0, d->W_down, d->inter, d->hidden, 1, d->hidden, d->inter, h, 1, cols, yacc, d->s_down))
+    if (!seg(g, maps, 0, d->W_down, d->inter, d->hidden, 1, d->hidden, d->inter, h, 1, hld, yacc, d->hidden,
+             d->s_down, ah))
       return LR_ERR_CUDA;
     g.nseg = 1;
     e = tc_product(maps, g, sms, true, stream);
@@ -774,14 +864,15 @@ static lr_status_t run_ffn_tc(const lr_ffn_desc_t* d, const void* x, int batch, 
     std::memset(&f, 0, sizeof(f));
     f.nt = 1;
     f.nb = nb;
-    f.ld = cols;
     f.zero_targets = 1;
     f.t[0].acc = yacc;
     f.t[0].y = reinterpret_cast<char*>(y) + size_t(b0) * d->hidden * 2;
     f.t[0].M = d->hidden;
     f.zero[0] = h;
-    f.zero_floats[0] = size_t(d->inter) * cols;
-    f.nz = 1;
+    f.zero_floats[0] = size_t(hld) * cols;
+    f.zero[1] = amax;   // the per-token maxima are raised with atomicMax: zero for the next pass
+    f.zero_floats[1] = 3 * kTcMaxPass;
+    f.nz = 2;
     e = launch_tc_finalize(f, sms, stream);
     if (e != cudaSuccess) return from_cuda(e);
   }

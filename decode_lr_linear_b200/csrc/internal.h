@@ -139,13 +139,29 @@ struct TcSeg {
   int M, K;           // weight rows (outputs) and reduction length
   int a_mn_major;     // 0: W stored [M, K]; 1: W stored [K, M] (its tensor map in TcMaps)
   int m_tiles, k_splits, kc, unit0;
-  const void* act;    // act_kind 0: bf16 [nb, K] (row stride act_ld); 1: fp32 [K, act_ld]
+  const void* act;    // token-major [nb, K], row stride act_ld (a multiple of 8): act_kind 0 bf16, 1 fp32
   int act_kind, act_ld;
-  float* out;         // fp32 [M, out_ld], added into
+  float* out;         // token-major fp32 [nb, out_ld], out[n][m] += product
   int out_ld;
   const void* row_scale;  // int8 weights: one scale per weight row (output channel), or null
   int row_scale_f16;
+  const float* tok_amax;  // int8 weights: per-token max |act| over the whole row
 };
+struct TcFinalTarget {
+  const float* acc;   // token-major fp32 [nb, M]
+  void* y;            // bf16 [nb, M]
+  int M;              // a multiple of 8
+};
+struct TcFinalizeParams {
+  TcFinalTarget t[4];
+  int nt;
+  int nb;
+  int zero_targets;   // clear each accumulator element after reading it
+  float* zero[3];
+  size_t zero_floats[3];  // multiples of 4
+  int nz;
+};
+// i8: int8 weights (kind::i8, activations as high and low int8 codes; hilo must be set)
 struct TcGemvParams {
   TcSeg seg[4];
   int nseg;
@@ -154,25 +170,11 @@ struct TcGemvParams {
   int hilo;           // split each fp32 activation into bf16 high and low parts (rows nb.. of the operand)
   int tmem_cols;
   int* err;
+  TcFinalizeParams pre;  // finalize work of the preceding step, spread over the units (after the dependency wait)
 };
 struct alignas(64) TcMaps {
   CUtensorMap m[4];
 };
-struct TcFinalTarget {
-  const float* acc;   // [M, ld]
-  void* y;            // bf16 [nb, M]
-  int M;
-};
-struct TcFinalizeParams {
-  TcFinalTarget t[4];
-  int nt;
-  int nb, ld;
-  int zero_targets;   // clear each accumulator element after reading it
-  float* zero[2];
-  size_t zero_floats[2];  // multiples of 4
-  int nz;
-};
-// i8: int8 weights (kind::i8, activations as high and low int8 codes; hilo must be set)
 int tc_gemv_kc(int K, int k_splits, bool i8);
 size_t tc_gemv_smem(int kc, int N, bool i8);
 bool tc_gemv_fits(int kc, int N, bool i8);
@@ -180,14 +182,26 @@ bool tc_make_weight_map(CUtensorMap* m, const void* W, int rows, int cols, int a
 cudaError_t launch_tc_gemv(const TcMaps& maps, const TcGemvParams& p, bool i8, cudaStream_t s);
 cudaError_t launch_tc_finalize(const TcFinalizeParams& f, int sm_count, cudaStream_t s);
 struct TcSwigluParams {
-  float* gu;          // [2 n_lr, cols] gate/up accumulators of the low-rank channels (interleaved rows)
-  float* dd;          // [2 n_dense, cols] of the dense channels
-  float* h;           // [n_lr + n_dense, cols]
-  int n_lr, n_dense, nb, cols;
-  float* zero;        // region zeroed afterwards (or null)
-  size_t zero_floats; // multiple of 4
+  float* gu;          // token-major [nb, 2 n_lr] gate/up accumulators of the low-rank channels (interleaved)
+  float* dd;          // token-major [nb, 2 n_dense] of the dense channels
+  float* h;           // token-major [nb, h_ld], h_ld >= n_lr + n_dense
+  int h_ld;
+  float* h_amax;      // [nb] max |h| per token (fp32 bits raised with atomicMax; zero on entry)
+  int n_lr, n_dense, nb;
+  float* zero;        // token-major rows of zero_row floats zeroed afterwards (or null)
+  int zero_row;
 };
 cudaError_t launch_tc_swiglu(const TcSwigluParams& p, int sm_count, cudaStream_t s);
+struct TcAmaxSrc {
+  const void* act;    // token-major [nb, K], row stride ld: kind 0 bf16, 1 fp32
+  int kind, K, ld;
+  float* amax;        // [nb], raised with atomicMax (zero on entry)
+};
+struct TcAmaxParams {
+  TcAmaxSrc src[4];
+  int nsrc, nb;
+};
+cudaError_t launch_tc_amax(const TcAmaxParams& p, cudaStream_t s);
 
 // Full-K/V flash decoding (the uncompressed baseline).
 struct FlashParams {

@@ -38,6 +38,8 @@ constexpr int kThreads = 128;
 constexpr int kATile = kBM * kKBytes;    // 16 KiB
 constexpr size_t kSmemCap = 200 * 1024;
 constexpr int kMaxTokens = 64;           // operand rows (tokens, or high and low parts)
+constexpr int kSwigluChunk = 1024;       // channels per SwiGLU CTA
+constexpr int kAmaxChunk = 2048;         // row elements per max CTA
 
 // Byte offset of byte `kb` of row n in a K-major, 128-byte-swizzled operand block
 // (rows of 128 bytes; the 16-byte chunk index is XORed with row bits 0..2).
@@ -62,41 +64,35 @@ LR_DEV void tmem_ld16(uint32_t taddr, uint32_t (&v)[16]) {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
-// Element e of a unit's activations for token n at reduction index k (0 outside [.., k1)).
-LR_DEV void load_act(const TcSeg& g, int n, int k, int k1, int cnt, float* v) {
+// Eight activations of token n from reduction index k (0 at k >= k1).  Both
+// sources are token-major: bf16 [nb, K] or fp32 [nb, K], row stride act_ld
+// (a multiple of 8 elements, so k..k+7 is one aligned 16- or 32-byte piece).
+LR_DEV void load_act8(const TcSeg& g, int n, int k, int k1, float* v) {
   if (g.act_kind == 0) {
     const __nv_bfloat16* src = reinterpret_cast<const __nv_bfloat16*>(g.act) + size_t(n) * g.act_ld + k;
-    if (k + cnt <= k1 && cnt == 8) {
-      bf16x8_to_f32(*reinterpret_cast<const uint4*>(src), v);
+    if (k + 8 <= k1) {
+      bf16x8_to_f32(ld_cg_u4(src), v);
     } else {
-      for (int e = 0; e < cnt; ++e) v[e] = k + e < k1 ? __bfloat162float(src[e]) : 0.f;
+      for (int e = 0; e < 8; ++e) v[e] = k + e < k1 ? __bfloat162float(src[e]) : 0.f;
     }
   } else {
-    const float* src = reinterpret_cast<const float*>(g.act) + size_t(k) * g.act_ld + n;
-    for (int e = 0; e < cnt; ++e) v[e] = k + e < k1 ? __ldcg(src + size_t(e) * g.act_ld) : 0.f;
+    const float* src = reinterpret_cast<const float*>(g.act) + size_t(n) * g.act_ld + k;
+    if (k + 8 <= k1) {
+      const float4 a = ld_cg_f4(src), b = ld_cg_f4(src + 4);
+      v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+    } else {
+      for (int e = 0; e < 8; ++e) v[e] = k + e < k1 ? __ldcg(src + e) : 0.f;
+    }
   }
 }
 
-// Chunk c of a unit's operand (k-block kb, token n, 16-byte chunk kci of the
-// 128-byte row): tokens vary fastest for an fp32 [K, ld] source (a warp then
-// reads 32 consecutive tokens of one row), reduction chunks vary fastest for a
-// bf16 [nb, K] source (a thread reads 16 contiguous bytes).
-LR_DEV void chunk_coords(int c, int nh, int act_kind, int* kb, int* n, int* kci) {
-  *kb = c / (nh * 8);
-  const int rem = c % (nh * 8);
-  if (act_kind == 0) {
-    *n = rem / 8;
-    *kci = rem % 8;
-  } else {
-    *kci = rem / nh;
-    *n = rem % nh;
-  }
-}
+LR_DEV void finalize_part(const TcFinalizeParams& F, int part, int parts, int t, int nt);
 
 // I8 = false: bf16 weights, kind::f16, bf16 operand rows (fp32 sources as high +
 // low parts).  I8 = true: int8 weights, kind::i8, every activation as two int8
-// codes with this unit's per-token scales s1 = max|x| / 127 over the unit's
-// reduction slice and s2 = s1 / 254: x ~ s1 hi + s2 lo with |error| <= s1 / 508.
+// codes with per-token scales s1 = max|x| / 127 over the token's whole input
+// (tok_amax, from tc_amax_kernel or the kernel that produced the input) and
+// s2 = s1 / 254: x ~ s1 hi + s2 lo with |error| <= s1 / 508.
 template <bool I8>
 __global__ void __launch_bounds__(kThreads) tc_gemv_kernel(const __grid_constant__ TcMaps maps,
                                                            const __grid_constant__ TcGemvParams P) {
@@ -107,7 +103,7 @@ __global__ void __launch_bounds__(kThreads) tc_gemv_kernel(const __grid_constant
   __shared__ __align__(8) uint64_t accum;
   __shared__ uint32_t tmem_slot;
   __shared__ float s_scale[2][kMaxTokens];   // I8: per-token scales of the high and low codes
-  __shared__ int s_amax[kMaxTokens];
+  __shared__ float s_inv[2][kMaxTokens];     // and their reciprocals (codes by multiplication)
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;      // ring: 1024-byte aligned tiles
   unsigned char* gbase = smem_raw + (base - raw);
@@ -135,7 +131,6 @@ __global__ void __launch_bounds__(kThreads) tc_gemv_kernel(const __grid_constant
     mbar_init(&accum, 1);
     fence_mbar_init();
   }
-  if (threadIdx.x < kMaxTokens) s_amax[threadIdx.x] = 0;
   if (warp == 1) tc::tmem_alloc(&tmem_slot, P.tmem_cols);
   tc::fence_before();
   __syncthreads();
@@ -162,84 +157,66 @@ __global__ void __launch_bounds__(kThreads) tc_gemv_kernel(const __grid_constant
 
   // ---- the activations of this unit as the N x K operand (zero outside the data) ----
   pdl_wait();
-  if constexpr (!I8) {
-    const int chunks = nkb * nh * 8;              // 8 consecutive k (16 bytes) of one token
-    for (int c = threadIdx.x; c < chunks; c += kThreads) {
-      int kb, n, kci;
-      chunk_coords(c, nh, g.act_kind, &kb, &n, &kci);
-      const int kc8 = kci * 8;
-      const int k = k0 + kb * kKB + kc8;
-      float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-      if (n < P.nb && k < k1) load_act(g, n, k, k1, 8, v);
-      uint32_t hi[4], lo[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * e], v[2 * e + 1]);
-        hi[e] = *reinterpret_cast<const uint32_t*>(&h);
-        const float2 hf = __bfloat1622float2(h);
-        const __nv_bfloat162 l = __floats2bfloat162_rn(v[2 * e] - hf.x, v[2 * e + 1] - hf.y);
-        lo[e] = *reinterpret_cast<const uint32_t*>(&l);
-      }
-      unsigned char* blk = act_g + size_t(kb) * N * 128;
-      *reinterpret_cast<uint4*>(blk + sw128_offset(n, kc8 * 2)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-      if (P.hilo) *reinterpret_cast<uint4*>(blk + sw128_offset(nh + n, kc8 * 2)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
-    }
-  } else {
-    // pass 1: per-token max |x| over the unit's slice
-    const int chunks = nkb * nh * 8;              // 16 consecutive k (16 codes) of one token
-    for (int c = threadIdx.x; c < chunks; c += kThreads) {
-      int kb, n, kci;
-      chunk_coords(c, nh, g.act_kind, &kb, &n, &kci);
-      const int k = k0 + kb * kKB + kci * 16;
-      if (n < P.nb && k < k1) {
-        float v[16];
-        load_act(g, n, k, k1, 8, v);
-        load_act(g, n, k + 8, k1, 8, v + 8);
-        float m = 0.f;
-#pragma unroll
-        for (int e = 0; e < 16; ++e) m = fmaxf(m, fabsf(v[e]));
-        atomicMax(&s_amax[n], __float_as_int(m));
-      }
-    }
-    __syncthreads();
+  // the preceding step's finalize, spread over this launch's units (outputs and clearing)
+  if (P.pre.nt > 0 || P.pre.nz > 0) finalize_part(P.pre, blockIdx.x, gridDim.x, threadIdx.x, kThreads);
+  if constexpr (I8) {
     if (threadIdx.x < nh) {
-      const float a = __int_as_float(s_amax[threadIdx.x]);
+      const float a = threadIdx.x < P.nb ? g.tok_amax[threadIdx.x] : 0.f;
       const float s1 = a > 0.f ? a / 127.f : 1.f;
       s_scale[0][threadIdx.x] = s1;
       s_scale[1][threadIdx.x] = s1 / 254.f;
+      s_inv[0][threadIdx.x] = 1.f / s1;
+      s_inv[1][threadIdx.x] = 254.f / s1;
     }
     __syncthreads();
-    // pass 2: the codes
+  }
+  {
+    // chunk c: k-block kb, token n, 16 bytes of the 128-byte operand row (8 bf16 or 16 int8 codes);
+    // the reduction index varies fastest, so a thread's loads are contiguous
+    constexpr int kPer = I8 ? 16 : 8;
+    const int chunks = nkb * nh * 8;
     for (int c = threadIdx.x; c < chunks; c += kThreads) {
-      int kb, n, kci;
-      chunk_coords(c, nh, g.act_kind, &kb, &n, &kci);
-      const int kc = kci * 16, k = k0 + kb * kKB + kc;
-      float v[16];
+      const int kb = c / (nh * 8), rem = c % (nh * 8), n = rem / 8, kci = rem % 8;
+      const int k = k0 + kb * kKB + kci * kPer;
+      float v[kPer];
 #pragma unroll
-      for (int e = 0; e < 16; ++e) v[e] = 0.f;
+      for (int e = 0; e < kPer; ++e) v[e] = 0.f;
       if (n < P.nb && k < k1) {
-        load_act(g, n, k, k1, 8, v);
-        load_act(g, n, k + 8, k1, 8, v + 8);
+        load_act8(g, n, k, k1, v);
+        if constexpr (I8) load_act8(g, n, k + 8, k1, v + 8);
       }
-      const float s1 = s_scale[0][n], s2 = s_scale[1][n];
       uint32_t hi[4], lo[4];
+      if constexpr (I8) {
+        // codes by multiplication with the reciprocal scales: the result is any integer pair whose
+        // error against x stays within s2 / 2 plus rounding; the epilogue uses s1, s2 themselves
+        const float s1 = s_scale[0][n], i1 = s_inv[0][n], i2 = s_inv[1][n];
 #pragma unroll
-      for (int w = 0; w < 4; ++w) {
-        uint32_t ph = 0, pl = 0;
+        for (int w = 0; w < 4; ++w) {
+          uint32_t ph = 0, pl = 0;
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float x = v[4 * w + e];
+            const float qh = fminf(fmaxf(rintf(x * i1), -127.f), 127.f);
+            const float ql = fminf(fmaxf(rintf(fmaf(-qh, s1, x) * i2), -127.f), 127.f);
+            ph |= (uint32_t(int(qh)) & 0xffu) << (8 * e);
+            pl |= (uint32_t(int(ql)) & 0xffu) << (8 * e);
+          }
+          hi[w] = ph;
+          lo[w] = pl;
+        }
+      } else {
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const float x = v[4 * w + e];
-          const float qh = fminf(fmaxf(rintf(x / s1), -127.f), 127.f);
-          const float ql = fminf(fmaxf(rintf((x - qh * s1) / s2), -127.f), 127.f);
-          ph |= (uint32_t(int(qh)) & 0xffu) << (8 * e);
-          pl |= (uint32_t(int(ql)) & 0xffu) << (8 * e);
+          const __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * e], v[2 * e + 1]);
+          hi[e] = *reinterpret_cast<const uint32_t*>(&h);
+          const float2 hf = __bfloat1622float2(h);
+          const __nv_bfloat162 l = __floats2bfloat162_rn(v[2 * e] - hf.x, v[2 * e + 1] - hf.y);
+          lo[e] = *reinterpret_cast<const uint32_t*>(&l);
         }
-        hi[w] = ph;
-        lo[w] = pl;
       }
       unsigned char* blk = act_g + size_t(kb) * N * 128;
-      *reinterpret_cast<uint4*>(blk + sw128_offset(n, kc)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-      *reinterpret_cast<uint4*>(blk + sw128_offset(nh + n, kc)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+      *reinterpret_cast<uint4*>(blk + sw128_offset(n, kci * 16)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+      if (P.hilo) *reinterpret_cast<uint4*>(blk + sw128_offset(nh + n, kci * 16)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
     }
   }
   fence_proxy_async();  // generic-proxy writes of the operand before the tensor cores read it
@@ -293,21 +270,18 @@ __global__ void __launch_bounds__(kThreads) tc_gemv_kernel(const __grid_constant
       tmem_ld16(tmem + (uint32_t(warp * 32) << 16) + uint32_t(c0), v);
       if (P.hilo) tmem_ld16(tmem + (uint32_t(warp * 32) << 16) + uint32_t(nh + c0), w);
       if (row < g.M) {
-        float* out = g.out + size_t(row) * g.out_ld + c0;
+        // token-major accumulator: out[n * out_ld + row]; a warp's 32 rows are contiguous for each n
 #pragma unroll
-        for (int e = 0; e < 16; e += 4) {
-          if (c0 + e < P.nb) {
-            float a[4];
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              if constexpr (I8) {
-                const int n = c0 + e + q;
-                a[q] = (float(int(v[e + q])) * s_scale[0][n] + float(int(w[e + q])) * s_scale[1][n]) * rs;
-              } else {
-                a[q] = (__uint_as_float(v[e + q]) + (P.hilo ? __uint_as_float(w[e + q]) : 0.f)) * rs;
-              }
+        for (int e = 0; e < 16; ++e) {
+          const int n = c0 + e;
+          if (n < P.nb) {
+            float a;
+            if constexpr (I8) {
+              a = (float(int(v[e])) * s_scale[0][n] + float(int(w[e])) * s_scale[1][n]) * rs;
+            } else {
+              a = (__uint_as_float(v[e]) + (P.hilo ? __uint_as_float(w[e]) : 0.f)) * rs;
             }
-            red_add_f4(out + e, a[0], a[1], a[2], a[3]);
+            atomicAdd(g.out + size_t(n) * g.out_ld + row, a);
           }
         }
       }
@@ -322,52 +296,117 @@ __global__ void __launch_bounds__(kThreads) tc_gemv_kernel(const __grid_constant
 }
 
 // y[n][m] = bf16(acc[m][n]) for every target; then zero the listed accumulator regions.
-__global__ void __launch_bounds__(256) tc_finalize_kernel(const __grid_constant__ TcFinalizeParams F) {
-  pdl_launch_dependents();
-  pdl_wait();
-  const int stride = gridDim.x * blockDim.x;
-  const int tid = blockIdx.x * blockDim.x + threadIdx.x;
-  for (int t = 0; t < F.nt; ++t) {
-    const TcFinalTarget& f = F.t[t];
-    for (int m = tid; m < f.M; m += stride) {
-      float* a = const_cast<float*>(f.acc) + size_t(m) * F.ld;
-      __nv_bfloat16* y = reinterpret_cast<__nv_bfloat16*>(f.y) + m;
-      for (int n = 0; n < F.nb; ++n) {
-        y[size_t(n) * f.M] = __float2bfloat16_rn(__ldcg(a + n));
-        if (F.zero_targets) __stcg(a + n, 0.f);   // read and cleared by the same thread
+// Finalize work for part `part` of `parts` (each part takes its share of every
+// target's 8-float chunks and of every zero region), thread `t` of `nt` within
+// the part: y[n][m] = bf16(acc[n][m]) for each target (token-major, M a
+// multiple of 8), clearing what it read when zero_targets is set; then the
+// zero regions, which no part reads.
+LR_DEV void finalize_part(const TcFinalizeParams& F, int part, int parts, int t, int nt) {
+  for (int q = 0; q < F.nt; ++q) {
+    const TcFinalTarget& f = F.t[q];
+    float* a = const_cast<float*>(f.acc);
+    __nv_bfloat16* y = reinterpret_cast<__nv_bfloat16*>(f.y);
+    const long long n8 = (long long)F.nb * f.M / 8;
+    const long long c0 = n8 * part / parts, c1 = n8 * (part + 1) / parts;
+    for (long long i = c0 + t; i < c1; i += nt) {
+      const float4 v0 = ld_cg_f4(a + 8 * i), v1 = ld_cg_f4(a + 8 * i + 4);
+      uint4 o;
+      uint32_t* ow = reinterpret_cast<uint32_t*>(&o);
+      const float v[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * e], v[2 * e + 1]);
+        ow[e] = *reinterpret_cast<const uint32_t*>(&h);
+      }
+      *reinterpret_cast<uint4*>(y + 8 * i) = o;
+      if (F.zero_targets) {   // read and cleared by the same thread
+        st_cg_f4(a + 8 * i, make_float4(0.f, 0.f, 0.f, 0.f));
+        st_cg_f4(a + 8 * i + 4, make_float4(0.f, 0.f, 0.f, 0.f));
       }
     }
   }
   for (int z = 0; z < F.nz; ++z) {
     float4* p = reinterpret_cast<float4*>(F.zero[z]);
-    const size_t n4 = F.zero_floats[z] / 4;
-    for (size_t i = tid; i < n4; i += stride) __stcg(p + i, make_float4(0.f, 0.f, 0.f, 0.f));
+    const long long n4 = (long long)(F.zero_floats[z] / 4);
+    const long long c0 = n4 * part / parts, c1 = n4 * (part + 1) / parts;
+    for (long long i = c0 + t; i < c1; i += nt) __stcg(p + i, make_float4(0.f, 0.f, 0.f, 0.f));
   }
 }
 
-// SwiGLU of the hybrid FFN between its two tensor-core products:
-// h[c][n] = silu(g) u for channel c, from the gate/up accumulators of the
-// low-rank channels (c < n_lr, rows 2c and 2c+1 of gu) or of the dense ones
-// (rows 2(c - n_lr), +1 of dd); each accumulator element is read and cleared by
-// the thread that uses it.  Then the listed region (the latent accumulator,
-// consumed by the preceding product) is zeroed.
+__global__ void __launch_bounds__(256) tc_finalize_kernel(const __grid_constant__ TcFinalizeParams F) {
+  pdl_launch_dependents();
+  pdl_wait();
+  finalize_part(F, blockIdx.x, gridDim.x, threadIdx.x, blockDim.x);
+}
+
+// SwiGLU of the hybrid FFN between its tensor-core products (token-major
+// accumulators), grid (tokens, channel chunks): h[n][c] = silu(g) u for
+// channel c, from the gate/up pair of the low-rank channels (c < n_lr:
+// gu[n][2c], gu[n][2c+1]) or of the dense ones (dd[n][2(c - n_lr)], +1); each
+// accumulator element is read and cleared by the thread that uses it.  The
+// token's max |h| (the scale of its int8 codes in the down projection) is
+// raised with atomicMax on its fp32 bits (non-negative, zero on entry), and the
+// chunk-0 CTA zeroes the token's latent row (consumed by the preceding product).
 __global__ void __launch_bounds__(256) tc_swiglu_kernel(const __grid_constant__ TcSwigluParams S) {
   pdl_launch_dependents();
   pdl_wait();
-  const int stride = gridDim.x * blockDim.x;
-  const int tid = blockIdx.x * blockDim.x + threadIdx.x;
+  __shared__ float red[8];
+  const int n = blockIdx.x;
   const int inter = S.n_lr + S.n_dense;
-  for (int i = tid; i < inter * S.nb; i += stride) {
-    const int c = i / S.nb, n = i % S.nb;
-    float* src = c < S.n_lr ? S.gu + size_t(2 * c) * S.cols : S.dd + size_t(2 * (c - S.n_lr)) * S.cols;
-    const float gt = __ldcg(src + n), up = __ldcg(src + S.cols + n);
-    __stcg(src + n, 0.f);
-    __stcg(src + S.cols + n, 0.f);
-    S.h[size_t(c) * S.cols + n] = silu(gt) * up;
+  float* gu = S.gu + size_t(n) * 2 * S.n_lr;
+  float* dd = S.dd + size_t(n) * 2 * S.n_dense;
+  float m = 0.f;
+  const int c0 = blockIdx.y * kSwigluChunk, c1 = min(inter, c0 + kSwigluChunk);
+  for (int c = c0 + int(threadIdx.x); c < c1; c += blockDim.x) {
+    float2* src = reinterpret_cast<float2*>(c < S.n_lr ? gu + 2 * c : dd + 2 * (c - S.n_lr));
+    const float2 gv = __ldcg(src);
+    __stcg(src, make_float2(0.f, 0.f));
+    const float hv = silu(gv.x) * gv.y;
+    S.h[size_t(n) * S.h_ld + c] = hv;
+    m = fmaxf(m, fabsf(hv));
   }
-  if (S.zero) {
-    float4* p = reinterpret_cast<float4*>(S.zero);
-    for (size_t i = tid; i < S.zero_floats / 4; i += stride) __stcg(p + i, make_float4(0.f, 0.f, 0.f, 0.f));
+  m = warp_max(m);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float a = red[0];
+    for (int w = 1; w < int(blockDim.x >> 5); ++w) a = fmaxf(a, red[w]);
+    atomicMax(reinterpret_cast<int*>(S.h_amax) + n, __float_as_int(a));
+  }
+  if (S.zero && blockIdx.y == 0) {
+    float* z = S.zero + size_t(n) * S.zero_row;
+    for (int i = threadIdx.x; i < S.zero_row; i += blockDim.x) __stcg(z + i, 0.f);
+  }
+}
+
+// Per-token max |x| over the row of each source (token-major, bf16 or fp32):
+// grid (tokens, sources); the scale of the token's int8 codes in the next product.
+__global__ void __launch_bounds__(256) tc_amax_kernel(const __grid_constant__ TcAmaxParams A) {
+  pdl_launch_dependents();
+  pdl_wait();
+  __shared__ float red[8];
+  const int n = blockIdx.x, s = blockIdx.y;
+  const TcAmaxSrc& src = A.src[s];
+  float m = 0.f;
+  // grid z: chunks of kAmaxChunk elements of the row, combined with atomicMax (zero on entry)
+  const int kend = min(src.K, int(blockIdx.z + 1) * kAmaxChunk);
+  for (int k = int(blockIdx.z) * kAmaxChunk + threadIdx.x * 8; k < kend; k += blockDim.x * 8) {
+    float v[8];
+    TcSeg g;
+    g.act = src.act;
+    g.act_kind = src.kind;
+    g.act_ld = src.ld;
+    load_act8(g, n, k, src.K, v);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) m = fmaxf(m, fabsf(v[e]));
+  }
+  m = warp_max(m);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float a = red[0];
+    for (int w = 1; w < int(blockDim.x >> 5); ++w) a = fmaxf(a, red[w]);
+    atomicMax(reinterpret_cast<int*>(src.amax) + n, __float_as_int(a));
   }
 }
 
@@ -420,12 +459,27 @@ cudaError_t launch_tc_gemv(const TcMaps& maps, const TcGemvParams& p, bool i8, c
   return cudaLaunchKernelEx(&c, kern, maps, p);
 }
 
-cudaError_t launch_tc_swiglu(const TcSwigluParams& p, int sm_count, cudaStream_t s) {
+cudaError_t launch_tc_amax(const TcAmaxParams& p, cudaStream_t s) {
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cudaLaunchConfig_t c = {};
-  c.gridDim = dim3(sm_count);
+  int kmax = 0;
+  for (int i = 0; i < p.nsrc; ++i) kmax = std::max(kmax, p.src[i].K);
+  c.gridDim = dim3(p.nb, p.nsrc, (kmax + kAmaxChunk - 1) / kAmaxChunk);
+  c.blockDim = dim3(256);
+  c.stream = s;
+  c.attrs = attr;
+  c.numAttrs = 1;
+  return cudaLaunchKernelEx(&c, tc_amax_kernel, p);
+}
+
+cudaError_t launch_tc_swiglu(const TcSwigluParams& p, int /*sm_count*/, cudaStream_t s) {
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t c = {};
+  c.gridDim = dim3(p.nb, (p.n_lr + p.n_dense + kSwigluChunk - 1) / kSwigluChunk);
   c.blockDim = dim3(256);
   c.stream = s;
   c.attrs = attr;

@@ -115,12 +115,14 @@ typedef struct lr_factor_desc {
  *   w_dtype LR_BF16: x bf16 [batch, d_in] -> y bf16 [batch, d_out]
  *   w_dtype LR_I8:   x bf16 [batch, d_in] -> y bf16 [batch, d_out]
  *   accumulation in fp32; the r-dim latent z = x A stays on chip in fp32.
- *   Up to batch 8 (and always for f32 and int8 weights) the CUDA cores
- *   stream the factors; bf16 factors above batch 8 run on the tensor cores
- *   (tcgen05, weights as the M operand, tokens as N), streaming every factor
- *   once per pass of up to 32 tokens; there the latent goes through an fp32
- *   accumulator in the workspace, split into bf16 high and low parts for the
- *   second product (fp32 accuracy).
+ *   Below batch 4 (and always for f32 weights) the CUDA cores stream the
+ *   factors; from batch 4 (lr_set_tensor_core_min_batch) bf16 and int8
+ *   factors run on the tensor cores (tcgen05, weights as the M operand,
+ *   tokens as N), streaming every factor once per pass of up to 32 tokens;
+ *   there the latent goes through an fp32 accumulator in the workspace and
+ *   enters the second product as bf16 high and low parts (bf16 factors,
+ *   fp32 accuracy) or as int8 high and low codes with a per-token scale
+ *   (int8 factors, error within max|z| / 64516 per element).
  * W8A8 path (x_scale != NULL; w_dtype LR_I8, scale_dtype LR_F32):
  *   x int8 [batch, d_in] with per-token scales x_scale f32 [batch] (from
  *   lr_quantize_per_token), y bf16 [batch, d_out]; int8 x int8 -> int32 tensor
@@ -133,10 +135,10 @@ typedef struct lr_factor_desc {
  * Weight-only limits: d_in and d_out multiples of 8 (of 16 for int8 weights)
  * and at most 32 KiB per factor row (d <= 16384 for bf16, 8192 for f32).
  * ws: workspace of at least lr_linear_workspace_size(...) bytes: 256 +
- * 8-rounded(min(batch, 8) * d_out) * 4, and for bf16 or int8 factors above
- * batch 8 at least 256 + (r + 2 d_out) * c * 4 with c = 8-rounded
- * min(batch, 32) (r the active rank).  Zero on entry (lr_workspace_init);
- * every call leaves it zero.
+ * 8-rounded(min(batch, 8) * d_out) * 4, and for bf16 or int8 factors on the
+ * tensor-core path at least 992 + (2 r8 + 2 d_out) * c * 4 with c = 8-rounded
+ * min(batch, 32) and r8 the 8-rounded active rank.  Zero on entry
+ * (lr_workspace_init); every call leaves it zero.
  * Errors: LR_ERR_INVALID_ARG (null pointers, batch < 1, bad shape or rank),
  * LR_ERR_UNSUPPORTED (dtype combination), LR_ERR_MISALIGNED,
  * LR_ERR_WORKSPACE, LR_ERR_CUDA.
@@ -179,11 +181,12 @@ LR_API lr_status_t lr_linear_grouped_workspace_size(const lr_factor_desc_t* desc
  * its input comes from; all steps share w_dtype (weight-only paths) and
  * scale_dtype; any batch >= 1 (one launch per 8 rows or fewer, depending on
  * the widest row); at most LR_MAX_CHAIN steps.
- * bf16 and int8 factors above batch 8 run on the tensor cores instead (as
- * lr_linear: three launches per step and pass of up to 32 tokens; there the
+ * bf16 and int8 factors from batch 4 run on the tensor cores instead (as
+ * lr_linear: two launches per step and pass of up to 32 tokens, four with
+ * int8 factors, plus one at the end; there the
  * step right before is read at fp32 from its accumulator and an older step
  * from its stored output).
- * Up to batch 8, one persistent CTA per SM (all resident: checked before the
+ * On the CUDA-core path, one persistent CTA per SM (all resident: checked before the
  * launch, LR_ERR_UNSUPPORTED otherwise) streams the factors of all steps back
  * to back through shared memory, so the loads of later steps proceed while a
  * step waits for its input; that wait on the CTAs producing the input is
@@ -529,8 +532,10 @@ LR_API lr_status_t lr_set_wait_timeout_us(unsigned int us);
 /*
  * Smallest batch at which lr_linear, lr_linear_grouped, lr_linear_chain (bf16
  * or int8 factors, weight-only) and lr_swiglu_ffn switch from the CUDA-core
- * decode kernels to the tensor-core path; 0 restores the default (9 for both:
- * the CUDA-core kernels take at most 8 tokens per pass of the weights).
+ * decode kernels to the tensor-core path; 0 restores the defaults, measured on
+ * B200: 4 for the linears (the CUDA-core kernels stream the weights once per
+ * 2 to 8 tokens, the tensor cores once per 32) and 1 for the FFN (its
+ * CUDA-core kernels are bound by int8-to-float conversion).
  * Process-wide, for calls issued after this one; the workspace sizes reported
  * afterwards follow the setting.  A tuning knob: both paths compute the same
  * products (see lr_linear and lr_swiglu_ffn for their precision).

@@ -45,18 +45,18 @@ def test_linear_workspace_sizes(lib):
     # completion counters (256 bytes) + min(batch, 8) x d_out fp32 accumulators (8-rounded)
     st, n = _ws(lib, _desc(), 1)
     assert st == L.LR_OK and n == 256 + 4096 * 4
-    st, n8 = _ws(lib, _desc(), 8)
-    assert st == L.LR_OK and n8 == 256 + 8 * 4096 * 4
-    # bf16 above batch 8 (tensor cores): z [rank, cols] and two y sets [d_out, cols], cols = 8-rounded
-    # min(batch, 32); the larger of the two paths' needs
+    st, n3 = _ws(lib, _desc(), 3)
+    assert st == L.LR_OK and n3 == 256 + 3 * 4096 * 4
+    # bf16 from batch 4 (tensor cores): 736 bytes of per-token maxima, two latent sets [cols, rank] and
+    # two y sets [cols, d_out], cols = 8-rounded min(batch, 32); the larger of the two paths' needs
     st, n16 = _ws(lib, _desc(), 16)
-    assert st == L.LR_OK and n16 == 256 + (1024 + 2 * 4096) * 16 * 4
+    assert st == L.LR_OK and n16 == 256 + 736 + (2 * 1024 + 2 * 4096) * 16 * 4
     st, n40 = _ws(lib, _desc(), 40)
-    assert st == L.LR_OK and n40 == 256 + (1024 + 2 * 4096) * 32 * 4
+    assert st == L.LR_OK and n40 == 256 + 736 + (2 * 1024 + 2 * 4096) * 32 * 4
     st, n16f = _ws(lib, _desc(w_dtype=L.LR_F32), 16)
     assert st == L.LR_OK and n16f == 256 + 8 * 4096 * 4
-    st, n3 = _ws(lib, _desc(d_out=8), 3)
-    assert st == L.LR_OK and n3 == 256 + 24 * 4
+    st, n3s = _ws(lib, _desc(d_out=8), 3)
+    assert st == L.LR_OK and n3s == 256 + 24 * 4
     st, _ = _ws(lib, _desc(w_dtype=L.LR_I8), 1)
     assert st == L.LR_ERR_INVALID_ARG  # int8 needs scales
     st, n = _ws(lib, _desc(w_dtype=L.LR_I8, scale_A=FAKE, scale_B=FAKE), 2048, 1)
@@ -108,7 +108,16 @@ def test_ffn_validation_and_workspace(lib):
     n = ctypes.c_size_t(0)
     d = _ffn()
     assert lib.lr_swiglu_ffn_workspace_size(ctypes.byref(d), 1, ctypes.byref(n)) == L.LR_OK
-    assert n.value == 256 + 16384 * 4 + 2816 * 4 + 4096 * 4
+    # tensor-core path (every batch by default): 256 + 736 bytes, then per token (8 columns at batch 1)
+    # z [rank], gate/up [2 inter], h [inter], y [hidden] fp32
+    assert n.value == 256 + 736 + (1536 + 2 * 11008 + 11008 + 4096) * 8 * 4
+    # the CUDA-core path's need: gate/up of the low-rank channels, h of the dense ones, y
+    try:
+        assert lib.lr_set_tensor_core_min_batch(64, 64) == L.LR_OK
+        assert lib.lr_swiglu_ffn_workspace_size(ctypes.byref(d), 1, ctypes.byref(n)) == L.LR_OK
+        assert n.value == 256 + 16384 * 4 + 2816 * 4 + 4096 * 4
+    finally:
+        lib.lr_set_tensor_core_min_batch(0, 0)
     bad = _ffn(n_lr=12000)
     assert lib.lr_swiglu_ffn(ctypes.byref(bad), FAKE, 1, FAKE, FAKE, 1 << 20, None) == L.LR_ERR_INVALID_ARG
     bad = _ffn(n_lr=8196)

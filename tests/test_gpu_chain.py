@@ -133,3 +133,26 @@ def test_ranked_chain_progressive_schedule(cuda_device, layers4):
                 assert normwise_rel(got, ref[n]) < NORMWISE_TOL, (t, l, n)
             x64 = ref["o"]
     assert int(ws.count_nonzero()) == 0
+
+
+def test_chain_split_layout_waits_only_for_inputs(cuda_device, layers4):
+    # V, then Q and K, then O (reads V two steps back) per layer: O waits only for V
+    x = synth.make_activations(2, 4096, seed=12, key=(76,))
+    steps = []
+    for l, L in enumerate(layers4):
+        src = -1 if l == 0 else 3 * l - 1
+        steps.append(lr.ChainStep([_fac(L["v"])], src, 0))
+        steps.append(lr.ChainStep([_fac(L["q"]), _fac(L["k"])], src, 0))
+        steps.append(lr.ChainStep([_fac(L["o"])], 3 * l, 0))
+    ws = lr.workspace(lr.lr_linear_chain_workspace_size(steps, 2), torch.device("cuda"))
+    outs = lr.lr_linear_chain(steps, dev(x), ws=ws)
+    torch.cuda.synchronize()
+    x64 = x.double().numpy()
+    for l, L in enumerate(layers4):
+        v, q, k = (_oracle(L[n], x64) for n in ("v", "q", "k"))
+        o = _oracle(L["o"], v)
+        for got, ref in zip(outs[3 * l] + outs[3 * l + 1] + outs[3 * l + 2], (v, q, k, o)):
+            assert normwise_rel(got, ref) < NORMWISE_TOL, l
+        x64 = o
+    assert int(ws.count_nonzero()) == 0
+    assert lr.lr_check_device_error() == 0

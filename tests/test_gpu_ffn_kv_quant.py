@@ -38,6 +38,20 @@ def test_hybrid_ffn_llama7b(cuda_device, ffn7b, batch):
     assert err < NORMWISE_TOL, err
 
 
+@pytest.mark.parametrize("batch", [1, 5])
+def test_hybrid_ffn_cuda_core_path(cuda_device, ffn7b, batch):
+    # the CUDA-core FFN kernels (the tensor cores take every batch by default)
+    lr.lr_set_tensor_core_min_batch(64, 64)
+    try:
+        x = synth.make_activations(batch, 4096, seed=0, key=(32, batch), outliers=4)
+        assert normwise_rel(lr.lr_swiglu_ffn(_ffn_dev(ffn7b), dev(x)), _ffn_oracle(ffn7b, x)) < NORMWISE_TOL
+        d = synth.make_hybrid_ffn(seed=1, hidden=512, inter=1000, n_lr=512, rank=512)
+        xs = synth.make_activations(batch, 512, seed=1, key=(33, batch), outliers=1)
+        assert normwise_rel(lr.lr_swiglu_ffn(_ffn_dev(d), dev(xs)), _ffn_oracle(d, xs)) < NORMWISE_TOL
+    finally:
+        lr.lr_set_tensor_core_min_batch(0, 0)
+
+
 @pytest.mark.parametrize("n_lr", [0, 512, 1000])
 def test_hybrid_ffn_small_and_degenerate(cuda_device, n_lr):
     d = synth.make_hybrid_ffn(seed=1, hidden=512, inter=1000, n_lr=n_lr, rank=512, rotate=n_lr > 0)

@@ -1,7 +1,7 @@
 """GPU parity at full size, in the launch the bench times: the 32-layer
 Llama-2-7B-shaped low-rank Q/K/V/O decode stack as one lr_linear_chain call
-at batch 1 (CUDA cores: 96 steps, V / Q and K / O per layer, as the bench
-times it) and 16 (tensor cores: 64 steps, Q/K/V / O per layer), every
+(64 dependent steps, Q/K/V then O per layer, as the bench times it) at batch
+1 (CUDA cores) and 16 (tensor cores), every
 output of every layer against the fp64 oracle run layer by layer on the same
 stored factors.
 """
@@ -40,16 +40,9 @@ def test_full_decode_stack_chain(cuda_device, layers32, batch):
     outs = [torch.empty(batch, HIDDEN, dtype=torch.bfloat16, device="cuda") for _ in range(LAYERS)]
     steps = []
     for l, L in enumerate(layers):
-        if batch < 9:
-            # the bench's layout on the CUDA-core path: V, then Q and K, then O (reads V)
-            src = -1 if l == 0 else 3 * l - 1
-            steps.append(lr.ChainStep([_fac(L["v"])], src, 0, [qkv[l][2]]))
-            steps.append(lr.ChainStep([_fac(L["q"]), _fac(L["k"])], src, 0, qkv[l][:2]))
-            steps.append(lr.ChainStep([_fac(L["o"])], 3 * l, 0, [outs[l]]))
-        else:
-            steps.append(lr.ChainStep([_fac(L["q"]), _fac(L["k"]), _fac(L["v"])], -1 if l == 0 else 2 * l - 1, 0,
-                                      qkv[l]))
-            steps.append(lr.ChainStep([_fac(L["o"])], 2 * l, 2, [outs[l]]))
+        steps.append(lr.ChainStep([_fac(L["q"]), _fac(L["k"]), _fac(L["v"])], -1 if l == 0 else 2 * l - 1, 0,
+                                  qkv[l]))
+        steps.append(lr.ChainStep([_fac(L["o"])], 2 * l, 2, [outs[l]]))
     ws = lr.workspace(lr.lr_linear_chain_workspace_size(steps, batch), torch.device("cuda"))
     lr.lr_linear_chain(steps, dev(x), ws=ws)
     torch.cuda.synchronize()

@@ -132,3 +132,17 @@ def test_errors_raise(cuda_device, layer0):
     with pytest.raises(lr.LrError):
         lr.lr_linear(f, x, ws=ws)
     assert lr.lr_check_device_error() == 0
+
+
+@pytest.mark.parametrize("batch", [5, 8])
+def test_cuda_core_path_multi_row(cuda_device, layer0, batch):
+    # the CUDA-core kernels at several rows per pass (the tensor cores take these batches by default)
+    lr.lr_set_tensor_core_min_batch(64, 64)
+    try:
+        x = synth.make_activations(batch, 4096, seed=13, key=(26, batch))
+        fs = [_factor_dev(layer0[n]) for n in ("q", "k", "v")]
+        ys = lr.lr_linear_grouped(fs, dev(x))
+        for y, n in zip(ys, ("q", "k", "v")):
+            assert normwise_rel(y, _oracle(layer0[n], x.double().numpy())) < NORMWISE_TOL
+    finally:
+        lr.lr_set_tensor_core_min_batch(0, 0)
