@@ -10,7 +10,7 @@ from .ops import (  # noqa: F401
     lr_swiglu_ffn, lr_swiglu_ffn_workspace_size, lr_latent_kv_decode, lr_latent_kv_workspace_size,
     lr_quantize_per_token, lr_gemm_s8s32, lr_workspace_init, lr_check_device_error, lr_set_wait_timeout_us,
     lr_rank_allocate, lr_linear_chain_ranked, lr_dense_linear, lr_flash_decode,
-    lr_latent_kv_decode_q8, lr_latent_kv_append, lr_set_tensor_core_min_batch,
+    lr_latent_kv_decode_q8, lr_latent_kv_append, lr_latent_kv_append_workspace_size, lr_set_tensor_core_min_batch,
 )
 from ._lib import LrError, load  # noqa: F401
 

@@ -81,7 +81,8 @@ _SIGNATURES = {
     "lr_latent_kv_decode_q8": (c_int, [P(LatentKvDesc), c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                                        c_void_p, c_void_p, c_size_t, c_void_p]),
     "lr_latent_kv_append": (c_int, [P(LatentKvDesc), c_void_p, c_int, c_void_p, c_void_p, c_void_p, c_void_p,
-                                    c_void_p]),
+                                    c_void_p, c_size_t, c_void_p]),
+    "lr_latent_kv_append_workspace_size": (c_int, [P(LatentKvDesc), c_int, P(c_size_t)]),
     "lr_flash_decode": (c_int, [P(FlashDesc), c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_size_t,
                                 c_void_p]),
     "lr_flash_decode_workspace_size": (c_int, [P(FlashDesc), P(c_size_t)]),

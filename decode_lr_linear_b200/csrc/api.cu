@@ -1032,17 +1032,83 @@ static lr_status_t run_latent_kv(const lr_latent_kv_desc_t* d, const void* q, co
   return from_cuda(launch_latent_kv(P, reinterpret_cast<cudaStream_t>(stream)));
 }
 
-lr_status_t lr_latent_kv_append(const lr_latent_kv_desc_t* d, const void* A_KV, int hidden, const void* x,
-                                const int* pos, void* C_K, void* C_V, lr_stream_t stream) {
-  if (!d || !A_KV || !x || !pos || !C_K || !C_V) return LR_ERR_INVALID_ARG;
+static lr_status_t check_append(const lr_latent_kv_desc_t* d, const void* A_KV, int hidden) {
+  if (!d || !A_KV) return LR_ERR_INVALID_ARG;
   if (d->batch <= 0 || d->heads <= 0 || d->rank <= 0 || d->max_ctx <= 0 || hidden <= 0) return LR_ERR_INVALID_ARG;
   if ((hidden % 16) != 0 || size_t(hidden) * 2 > 32768) return LR_ERR_UNSUPPORTED;
   if (double(2) * d->heads * d->rank > 2147483647.0) return LR_ERR_UNSUPPORTED;
+  return LR_OK;
+}
+
+// The tensor-core path needs 8-float aligned accumulator rows (2 H r a multiple of 8).
+static bool append_tc(const lr_latent_kv_desc_t* d) { return (size_t(d->heads) * d->rank) % 4 == 0; }
+
+lr_status_t lr_latent_kv_append_workspace_size(const lr_latent_kv_desc_t* d, int hidden, size_t* bytes) {
+  if (!bytes) return LR_ERR_INVALID_ARG;
+  lr_status_t st = check_append(d, reinterpret_cast<const void*>(16), hidden);
+  if (st != LR_OK) return st;
+  *bytes = append_tc(d) ? kTicketBytes + size_t(2) * d->heads * d->rank * size_t(tc_cols(d->batch)) * 4 : 0;
+  return LR_OK;
+}
+
+lr_status_t lr_latent_kv_append(const lr_latent_kv_desc_t* d, const void* A_KV, int hidden, const void* x,
+                                const int* pos, void* C_K, void* C_V, void* ws, size_t ws_bytes,
+                                lr_stream_t stream) {
+  lr_status_t st = check_append(d, A_KV, hidden);
+  if (st != LR_OK) return st;
+  if (!x || !pos || !C_K || !C_V) return LR_ERR_INVALID_ARG;
   if (!al16(A_KV) || !al16(x) || !al16(pos) || !al16(C_K) || !al16(C_V)) return LR_ERR_MISALIGNED;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int width = 2 * d->heads * d->rank;
+  if (ws && append_tc(d)) {
+    // tensor cores: latents = x A_KV^T into a token-major fp32 accumulator, then scattered
+    size_t need = 0;
+    lr_latent_kv_append_workspace_size(d, hidden, &need);
+    if (ws_bytes < need) return LR_ERR_WORKSPACE;
+    if (!al16(ws)) return LR_ERR_MISALIGNED;
+    float* acc = reinterpret_cast<float*>(reinterpret_cast<char*>(ws) + kTicketBytes);
+    const int sms = sm_count_current();
+    const size_t per_seq = size_t(d->heads) * d->max_ctx * d->rank * 2;  // bytes of one sequence's cache
+    for (int b0 = 0; b0 < d->batch; b0 += kTcMaxPass) {
+      const int nb = std::min(kTcMaxPass, d->batch - b0);
+      TcMaps maps;
+      TcGemvParams g;
+      std::memset(&maps, 0, sizeof(maps));
+      std::memset(&g, 0, sizeof(g));
+      if (!weight_map(&maps.m[0], A_KV, width, hidden, 0, false)) return LR_ERR_CUDA;
+      g.nseg = 1;
+      g.nb = nb;
+      g.N = int(round_up(size_t(nb), 16));
+      g.hilo = 0;
+      g.err = device_error_word();
+      TcSeg& sg = g.seg[0];
+      sg.M = width;
+      sg.K = hidden;
+      sg.act = reinterpret_cast<const char*>(x) + size_t(b0) * hidden * 2;
+      sg.act_kind = 0;
+      sg.act_ld = hidden;
+      sg.out = acc;
+      sg.out_ld = width;
+      cudaError_t e = tc_product(maps, g, sms, false, s);
+      if (e != cudaSuccess) return from_cuda(e);
+      TcScatterParams sp;
+      sp.acc = acc;
+      sp.cache_k = reinterpret_cast<char*>(C_K) + size_t(b0) * per_seq;
+      sp.cache_v = reinterpret_cast<char*>(C_V) + size_t(b0) * per_seq;
+      sp.pos = pos + b0;
+      sp.nb = nb;
+      sp.heads = d->heads;
+      sp.rank = d->rank;
+      sp.ctx = d->max_ctx;
+      e = launch_tc_cache_scatter(sp, s);
+      if (e != cudaSuccess) return from_cuda(e);
+    }
+    return LR_OK;
+  }
   FfnParams P;
   std::memset(&P, 0, sizeof(P));
   P.hidden = hidden;
-  P.n_dense = 2 * d->heads * d->rank;
+  P.n_dense = width;
   P.nb = d->batch;
   P.D = reinterpret_cast<const int8_t*>(A_KV);
   P.x = x;
@@ -1053,7 +1119,7 @@ lr_status_t lr_latent_kv_append(const lr_latent_kv_desc_t* d, const void* A_KV, 
   P.cache_rank = d->rank;
   P.cache_ctx = d->max_ctx;
   P.err = device_error_word();
-  return from_cuda(launch_dense(P, LR_BF16, sm_count_current(), reinterpret_cast<cudaStream_t>(stream)));
+  return from_cuda(launch_dense(P, LR_BF16, sm_count_current(), s));
 }
 
 lr_status_t lr_latent_kv_decode(const lr_latent_kv_desc_t* d, const void* q, const void* C_K, const void* C_V,

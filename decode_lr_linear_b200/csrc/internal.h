@@ -202,6 +202,14 @@ struct TcAmaxParams {
   int nsrc, nb;
 };
 cudaError_t launch_tc_amax(const TcAmaxParams& p, cudaStream_t s);
+struct TcScatterParams {
+  float* acc;         // token-major fp32 [nb, 2 heads rank], cleared
+  void* cache_k;      // bf16 [nb, heads, ctx, rank], offset to the pass's first sequence
+  void* cache_v;
+  const int* pos;     // [nb]
+  int nb, heads, rank, ctx;
+};
+cudaError_t launch_tc_cache_scatter(const TcScatterParams& p, cudaStream_t s);
 
 // Full-K/V flash decoding (the uncompressed baseline).
 struct FlashParams {

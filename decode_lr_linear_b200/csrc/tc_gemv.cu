@@ -410,6 +410,29 @@ __global__ void __launch_bounds__(256) tc_amax_kernel(const __grid_constant__ Tc
   }
 }
 
+// The latent producer's scatter after its tensor-core product: token n's row of
+// the token-major fp32 accumulator [nb, 2 H r] (keys then values, head-major)
+// goes to the caches at position pos[n] as bf16 and is cleared (read and
+// cleared by the same thread); a position outside [0, ctx) writes nothing.
+__global__ void __launch_bounds__(256) tc_cache_scatter_kernel(const __grid_constant__ TcScatterParams S) {
+  pdl_launch_dependents();
+  pdl_wait();
+  const int n = blockIdx.y;
+  const int hr = S.heads * S.rank, width = 2 * hr;
+  const int ps = S.pos[n];
+  const bool keep = ps >= 0 && ps < S.ctx;
+  float* a = S.acc + size_t(n) * width;
+  for (int j = blockIdx.x * blockDim.x + threadIdx.x; j < width; j += gridDim.x * blockDim.x) {
+    const float v = __ldcg(a + j);
+    __stcg(a + j, 0.f);
+    if (keep) {
+      const int kv = j >= hr ? 1 : 0, rr = j - kv * hr;
+      __nv_bfloat16* c = reinterpret_cast<__nv_bfloat16*>(kv ? S.cache_v : S.cache_k);
+      c[((size_t(n) * S.heads + rr / S.rank) * S.ctx + ps) * S.rank + rr % S.rank] = __float2bfloat16_rn(v);
+    }
+  }
+}
+
 int kb_elems(bool i8) { return i8 ? 128 : 64; }
 
 }  // namespace
@@ -472,6 +495,19 @@ cudaError_t launch_tc_amax(const TcAmaxParams& p, cudaStream_t s) {
   c.attrs = attr;
   c.numAttrs = 1;
   return cudaLaunchKernelEx(&c, tc_amax_kernel, p);
+}
+
+cudaError_t launch_tc_cache_scatter(const TcScatterParams& p, cudaStream_t s) {
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t c = {};
+  c.gridDim = dim3((2 * p.heads * p.rank + 255) / 256, p.nb);
+  c.blockDim = dim3(256);
+  c.stream = s;
+  c.attrs = attr;
+  c.numAttrs = 1;
+  return cudaLaunchKernelEx(&c, tc_cache_scatter_kernel, p);
 }
 
 cudaError_t launch_tc_swiglu(const TcSwigluParams& p, int /*sm_count*/, cudaStream_t s) {

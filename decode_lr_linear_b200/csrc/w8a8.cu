@@ -41,6 +41,7 @@ constexpr int kATileBytes = kBM * kBK;         // 16 KB
 constexpr int kBTileBytes = kBN * kBK;         // 32 KB
 constexpr int kStageBytes = kATileBytes + kBTileBytes;
 constexpr int kTmemCols = 256;
+constexpr int kEpiStageBytes = 4 * 32 * 33 * 4;  // a 32 x 32 fp32 chunk per epilogue warp (padded rows)
 
 // 2-D int8 tensor [rows, cols] (row stride `ld` bytes), box [box_rows, box_cols],
 // 128-byte swizzle, zero fill outside the tensor.
@@ -156,37 +157,79 @@ __global__ void __launch_bounds__(kThreads, 1) w8a8_gemm_kernel(const __grid_con
       // the raw int32 mode has no scales (s_row, s_col are null there)
       const float sr = (P.mode != 2 && row < P.M) ? P.s_row[row] : 0.f;
       float rmax = 0.f;
+      // Each 32 x 32 chunk (lane = row) goes through this warp's shared-memory
+      // stage, so that global stores are whole 16-byte pieces of rows (a warp
+      // instruction covers 4 rows of fp32 or 8 rows of bf16) instead of one
+      // partial 32-byte sector per element.
+      float* stage = reinterpret_cast<float*>(smem_raw + (base - smem_u32(smem_raw)) + size_t(kStages) * kStageBytes) +
+                     q * 32 * 33;
+      const bool vec = (P.N % 8) == 0;
       for (int c = 0; c < kBN / 32; ++c) {
         uint32_t v[32];
         tmem_ld32(tmem + (uint32_t(q * 32) << 16) + uint32_t(c * 32), v);
         const int col0 = n0 + c * 32;
-        if (row >= P.M || col0 >= P.N) continue;
+        if (col0 >= P.N) continue;
+        float f[32];
         if (P.mode == 2) {
-          int32_t* cr = P.c + size_t(row) * P.N + col0;
 #pragma unroll
-          for (int i = 0; i < 32; ++i)
-            if (col0 + i < P.N) cr[i] = int32_t(v[i]);
-        } else if (P.mode == 0) {
-          float* zr = P.z + size_t(row) * P.N + col0;
+          for (int i = 0; i < 32; ++i) f[i] = __uint_as_float(v[i]);
+        } else {
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
-            if (col0 + i < P.N) {
-              const float zv = __fmul_rn(__fmul_rn(__int2float_rn(int(v[i])), sr), P.s_col[col0 + i]);
-              zr[i] = zv;
-              rmax = fmaxf(rmax, fabsf(zv));
+            const float sc = col0 + i < P.N ? P.s_col[col0 + i] : 0.f;
+            f[i] = __fmul_rn(__fmul_rn(__int2float_rn(int(v[i])), sr), sc);
+          }
+          if (P.mode == 0 && row < P.M) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              if (col0 + i < P.N) rmax = fmaxf(rmax, fabsf(f[i]));
+          }
+        }
+        if (vec && col0 + 32 <= P.N) {
+          __syncwarp();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) stage[lane * 33 + i] = f[i];
+          __syncwarp();
+          const int rbase = m0 + q * 32;
+          if (P.mode == 1) {
+            // 4 lanes per row, 8 bf16 (16 bytes) each; 8 rows per instruction
+#pragma unroll
+            for (int it = 0; it < 4; ++it) {
+              const int r = it * 8 + (lane >> 2), cc = (lane & 3) * 8;
+              if (rbase + r < P.M) {
+                const float* sp = stage + r * 33 + cc;
+                uint4 o;
+                uint32_t* ow = reinterpret_cast<uint32_t*>(&o);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                  const __nv_bfloat162 h = __floats2bfloat162_rn(sp[2 * e], sp[2 * e + 1]);
+                  ow[e] = *reinterpret_cast<const uint32_t*>(&h);
+                }
+                *reinterpret_cast<uint4*>(P.y + size_t(rbase + r) * P.N + col0 + cc) = o;
+              }
+            }
+          } else {
+            // 8 lanes per row, 4 words (16 bytes) each; 4 rows per instruction
+            uint32_t* dst = P.mode == 0 ? reinterpret_cast<uint32_t*>(P.z) : reinterpret_cast<uint32_t*>(P.c);
+#pragma unroll
+            for (int it = 0; it < 8; ++it) {
+              const int r = it * 4 + (lane >> 3), cc = (lane & 7) * 4;
+              if (rbase + r < P.M) {
+                const float* sp = stage + r * 33 + cc;
+                *reinterpret_cast<uint4*>(dst + size_t(rbase + r) * P.N + col0 + cc) =
+                    make_uint4(__float_as_uint(sp[0]), __float_as_uint(sp[1]), __float_as_uint(sp[2]),
+                               __float_as_uint(sp[3]));
+              }
             }
           }
-        } else {
-          __nv_bfloat16* yr = P.y + size_t(row) * P.N + col0;
-#pragma unroll
-          for (int i = 0; i < 32; i += 2) {
-            if (col0 + i + 1 < P.N) {
-              const float a = __fmul_rn(__fmul_rn(__int2float_rn(int(v[i])), sr), P.s_col[col0 + i]);
-              const float b = __fmul_rn(__fmul_rn(__int2float_rn(int(v[i + 1])), sr), P.s_col[col0 + i + 1]);
-              *reinterpret_cast<__nv_bfloat162*>(yr + i) = __floats2bfloat162_rn(a, b);
-            } else if (col0 + i < P.N) {
-              yr[i] = __float2bfloat16_rn(__fmul_rn(__fmul_rn(__int2float_rn(int(v[i])), sr), P.s_col[col0 + i]));
-            }
+        } else if (row < P.M) {
+          // a ragged last chunk: element stores
+          for (int i = 0; i < 32; ++i) {
+            if (col0 + i >= P.N) break;
+            const size_t o = size_t(row) * P.N + col0 + i;
+            if (P.mode == 0) P.z[o] = f[i];
+            else if (P.mode == 2) P.c[o] = int32_t(__float_as_uint(f[i]));
+            else P.y[o] = __float2bfloat16_rn(f[i]);
           }
         }
       }
@@ -239,7 +282,7 @@ __global__ void __launch_bounds__(256) requant_kernel(const float* __restrict__ 
 }
 
 cudaError_t launch_gemm(const CUtensorMap& a, const CUtensorMap& b, const GemmParams& p, cudaStream_t s) {
-  const size_t smem = size_t(kStages) * kStageBytes + 1024;
+  const size_t smem = size_t(kStages) * kStageBytes + 1024 + kEpiStageBytes;
   cudaError_t e = ensure_smem(w8a8_gemm_kernel, smem);
   if (e != cudaSuccess) return e;
   cudaLaunchAttribute attr[1];

@@ -255,13 +255,30 @@ def lr_latent_kv_decode(kv: LatentKv, q: torch.Tensor, C_K: torch.Tensor, C_V: t
     return out
 
 
+def lr_latent_kv_append_workspace_size(kv: LatentKv, hidden: int) -> int:
+    n = ctypes.c_size_t(0)
+    d = kv.desc()
+    L.check("lr_latent_kv_append_workspace_size",
+            L.load().lr_latent_kv_append_workspace_size(ctypes.byref(d), int(hidden), ctypes.byref(n)))
+    return n.value
+
+
 def lr_latent_kv_append(kv: LatentKv, A_KV: torch.Tensor, x: torch.Tensor, pos: torch.Tensor, C_K: torch.Tensor,
-                        C_V: torch.Tensor, stream=None) -> None:
-    """Write the new token's per-head latents x A_Kh, x A_Vh into C_K, C_V at position pos[b]."""
+                        C_V: torch.Tensor, ws: Optional[torch.Tensor] = None, use_ws: bool = True,
+                        stream=None) -> None:
+    """Write the new token's per-head latents x A_Kh, x A_Vh into C_K, C_V at position pos[b].
+
+    With a workspace (allocated here when ``ws`` is None and ``use_ws``) the product runs on the tensor
+    cores; ``use_ws=False`` keeps the CUDA-core GEMV."""
+    hidden = A_KV.shape[1]
+    if ws is None and use_ws:
+        n = lr_latent_kv_append_workspace_size(kv, hidden)
+        ws = workspace(n, x.device) if n else None
     d = kv.desc()
     L.check("lr_latent_kv_append",
-            L.load().lr_latent_kv_append(ctypes.byref(d), _ptr(A_KV), A_KV.shape[1], _ptr(x), _ptr(pos), _ptr(C_K),
-                                         _ptr(C_V), _stream(stream)))
+            L.load().lr_latent_kv_append(ctypes.byref(d), _ptr(A_KV), hidden, _ptr(x), _ptr(pos), _ptr(C_K),
+                                         _ptr(C_V), _ptr(ws), 0 if ws is None else ws.numel() * ws.element_size(),
+                                         _stream(stream)))
 
 
 def lr_quantize_per_token(x: torch.Tensor, x_q: Optional[torch.Tensor] = None, s: Optional[torch.Tensor] = None,

@@ -433,11 +433,20 @@ LR_API lr_status_t lr_latent_kv_decode_q8(const lr_latent_kv_desc_t* desc, const
  *         [0, max_ctx) writes nothing for that sequence
  *   C_K, C_V  bf16 [batch, heads, max_ctx, rank], updated in place at
  *         [b, :, pos[b], :]; nothing else is written
+ *   ws    lr_latent_kv_append_workspace_size bytes, zero on entry and left
+ *         zero: the product then runs on the tensor cores (tcgen05, the stacked
+ *         factors as the M operand, the tokens as N, split over the reduction
+ *         into an fp32 accumulator) and a scatter writes the bf16 latents; NULL
+ *         (or heads * rank not a multiple of 4) keeps the CUDA-core GEMV, which
+ *         writes the caches from its epilogue and needs no workspace
  * Only desc->batch, heads, rank and max_ctx are read.  Limits: hidden a
- * multiple of 16 with hidden * 2 <= 32 KiB.  No workspace.
+ * multiple of 16 with hidden * 2 <= 32 KiB.
  */
 LR_API lr_status_t lr_latent_kv_append(const lr_latent_kv_desc_t* desc, const void* A_KV, int hidden, const void* x,
-                                       const int* pos, void* C_K, void* C_V, lr_stream_t stream);
+                                       const int* pos, void* C_K, void* C_V, void* ws, size_t ws_bytes,
+                                       lr_stream_t stream);
+
+LR_API lr_status_t lr_latent_kv_append_workspace_size(const lr_latent_kv_desc_t* desc, int hidden, size_t* bytes);
 
 /*
  * Standard single-query flash decoding over full K/V caches: the uncompressed

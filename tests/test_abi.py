@@ -286,10 +286,17 @@ def test_latent_kv_reconstruct_mode_validation(lib):
 
 def test_latent_kv_append_validation(lib):
     d = _kv()
-    assert lib.lr_latent_kv_append(ctypes.byref(d), None, 4096, FAKE, FAKE, FAKE, FAKE, None) == L.LR_ERR_INVALID_ARG
-    assert lib.lr_latent_kv_append(ctypes.byref(d), FAKE, 0, FAKE, FAKE, FAKE, FAKE, None) == L.LR_ERR_INVALID_ARG
-    assert lib.lr_latent_kv_append(ctypes.byref(d), FAKE, 4100, FAKE, FAKE, FAKE, FAKE, None) == L.LR_ERR_UNSUPPORTED
-    assert lib.lr_latent_kv_append(ctypes.byref(d), FAKE, 32768, FAKE, FAKE, FAKE, FAKE, None) == L.LR_ERR_UNSUPPORTED
-    assert lib.lr_latent_kv_append(ctypes.byref(d), FAKE, 4096, FAKE, MIS, FAKE, FAKE, None) == L.LR_ERR_MISALIGNED
-    assert lib.lr_latent_kv_append(ctypes.byref(_kv(batch=0)), FAKE, 4096, FAKE, FAKE, FAKE, FAKE,
-                                   None) == L.LR_ERR_INVALID_ARG
+    app = lambda dd, a=FAKE, hid=4096, pos=FAKE, ws=None, wsb=0: lib.lr_latent_kv_append(  # noqa: E731
+        ctypes.byref(dd), a, hid, FAKE, pos, FAKE, FAKE, ws, wsb, None)
+    assert app(d, a=None) == L.LR_ERR_INVALID_ARG
+    assert app(d, hid=0) == L.LR_ERR_INVALID_ARG
+    assert app(d, hid=4100) == L.LR_ERR_UNSUPPORTED
+    assert app(d, hid=32768) == L.LR_ERR_UNSUPPORTED
+    assert app(d, pos=MIS) == L.LR_ERR_MISALIGNED
+    assert app(_kv(batch=0)) == L.LR_ERR_INVALID_ARG
+    # the tensor-core path's workspace: counters + a token-major fp32 row of 2 * heads * rank per token
+    n = ctypes.c_size_t(0)
+    assert lib.lr_latent_kv_append_workspace_size(ctypes.byref(d), 4096, ctypes.byref(n)) == L.LR_OK
+    assert n.value == 256 + 2 * 32 * 32 * 8 * 4
+    assert app(d, ws=FAKE, wsb=64) == L.LR_ERR_WORKSPACE
+    assert app(d, ws=MIS, wsb=1 << 20) == L.LR_ERR_MISALIGNED

@@ -90,8 +90,8 @@ def test_latent_kv_outputs(cuda_device, mode, base):
 
 
 def test_dense_and_flash_outputs(cuda_device):
-    W = dev((torch.randn(136, 264) / 16).to(torch.bfloat16))
-    x = dev(synth.make_activations(5, 264, seed=9, key=(123,)))
+    W = dev((torch.randn(136, 272) / 16).to(torch.bfloat16))
+    x = dev(synth.make_activations(5, 272, seed=9, key=(123,)))
     ybuf, y = _guarded((5, 136), torch.bfloat16)
     lr.lr_dense_linear(W, x, y=y)
     assert _guards_intact(ybuf, torch.bfloat16)

@@ -60,7 +60,9 @@ def test_reconstruct_rope_full_size_sampled(cuda_device, ctx):
     assert lr.lr_check_device_error() == 0
 
 
-def test_append_writes_only_the_new_positions(cuda_device):
+@pytest.mark.parametrize("use_ws", [True, False])
+def test_append_writes_only_the_new_positions(cuda_device, use_ws):
+    # with a workspace: tensor-core product + scatter; without: the CUDA-core GEMV
     heads, rank, hidden, ctx, batch = 32, 32, 4096, 64, 5
     pr = synth.make_latent_producer(heads, rank, hidden, seed=1)
     d = synth.make_latent_kv(batch=batch, heads=heads, ctx=ctx, seed=6)
@@ -68,7 +70,7 @@ def test_append_writes_only_the_new_positions(cuda_device):
     pos = torch.tensor([0, 17, 63, 64, -1], dtype=torch.int32)   # the last two are outside the cache
     CK, CV = dev(d["C_K"]), dev(d["C_V"])
     kv = lr.LatentKv(batch, heads, ctx, dev(d["B_K"]), dev(d["B_V"]), d["scale"])
-    lr.lr_latent_kv_append(kv, dev(pr["A_KV"]), dev(x), dev(pos), CK, CV)
+    lr.lr_latent_kv_append(kv, dev(pr["A_KV"]), dev(x), dev(pos), CK, CV, use_ws=use_ws)
     rk, rv = okv.append_latents(x, pr["A_KV"], heads, rank, d["C_K"], d["C_V"], pos.numpy())
     ck, cv = CK.cpu(), CV.cpu()
     for b in range(batch):
