@@ -640,9 +640,11 @@ def row_c3(lr, L, synth, device, d, batch, want_cpu):
     ms_e2e = time_e2e(e2e, 40)
     if batch >= TC_MIN[1]:
         passes = math.ceil(batch / 32)
-        pieces = passes * (5 if d["n_lr"] > 0 else 4)
-        note = (f"{pieces} launches: tcgen05 kind::i8 products (x A' with x D, B'^T z, W_down^T h), SwiGLU, finalize; "
-                f"every weight byte streamed once per pass of 32 tokens")
+        fused = batch <= 4   # the down projection evaluates the SwiGLU while it stages h
+        pieces = passes * ((4 if d["n_lr"] > 0 else 3) + (0 if fused else 1))
+        note = (f"{pieces} launches: tcgen05 kind::i8 products (x A' with x D, B'^T z, W_down^T h), "
+                + ("the SwiGLU evaluated while h is staged" if fused else "a SwiGLU kernel")
+                + ", finalize; every weight byte streamed once per pass of 32 tokens")
     else:
         pieces = math.ceil(batch / 2) + math.ceil(batch / 4)
         note = f"{pieces} launch(es) of the CUDA-core decode engine, each streaming its phase's weight bytes"

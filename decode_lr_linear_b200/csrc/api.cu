@@ -160,12 +160,10 @@ void tc_sizes(const HostStep* steps, int n_steps, size_t* zmax, size_t* ymax) {
     *ymax = std::max(*ymax, y);
   }
 }
-// + per-token maxima of a step's input and of its latents (int8 factors)
-constexpr size_t kTcAmaxBytes = 5 * kTcMaxPass * 4 + 96;
 size_t tc_ws_bytes(const HostStep* steps, int n_steps, int batch) {
   size_t zm, ym;
   tc_sizes(steps, n_steps, &zm, &ym);
-  return kTicketBytes + kTcAmaxBytes + (2 * zm + 2 * ym) * size_t(tc_cols(batch)) * 4;
+  return kTicketBytes + (2 * zm + 2 * ym) * size_t(tc_cols(batch)) * 4;
 }
 
 size_t chain_ws_bytes(const HostStep* steps, int n_steps, int batch, bool allow_tc = true) {
@@ -262,18 +260,12 @@ cudaError_t tc_product(TcMaps& maps, TcGemvParams& g, int sms, bool i8, cudaStre
   return launch_tc_gemv(maps, g, i8, stream);
 }
 
-// The chain on the tensor cores, per pass of up to kTcMaxPass tokens and per step:
-//   product 1: z_p += A_p x      (input: the chain input, the previous step's fp32
-//                                 accumulator, or an older step's stored output)
-//   product 2: y_p += B_p^T z_p  (fp32 z split into bf16 high and low parts)
-//   finalize:  y_p (bf16) from the accumulator; zero z and the other y set.
 // The chain on the tensor cores, per pass of up to kTcMaxPass tokens and per step s:
-//   (int8 factors: per-token max of the input)
 //   product 1: z_p += x A_p into latent set s % 2; its units first finalize step
-//              s-1 (bf16 outputs from y set (s-1) % 2) and clear y set s % 2,
-//              latent set (s-1) % 2 and the latent maxima, none of which it reads
-//   (int8 factors: per-token max of each latent)
-//   product 2: y_p += z_p B_p into y set s % 2 (units first clear the input maximum)
+//              s-1 (bf16 outputs from y set (s-1) % 2) and clear y set s % 2 and
+//              latent set (s-1) % 2, neither of which it reads
+//   product 2: y_p += z_p B_p into y set s % 2 (fp32 z as bf16 high and low
+//              parts, or int8 high and low codes for int8 factors)
 // and after the last step one finalize launch.  All accumulators are token-major
 // fp32; the input is the chain input, the previous step's y set (fp32), or an
 // older step's stored bf16 output.
@@ -281,8 +273,7 @@ lr_status_t run_chain_tc(const HostStep* steps, int n_steps, const void* x, int 
   size_t zmax, ymax;
   tc_sizes(steps, n_steps, &zmax, &ymax);
   const int cols = tc_cols(batch);
-  float* amax = reinterpret_cast<float*>(reinterpret_cast<char*>(ws) + kTicketBytes);  // [5][kTcMaxPass]
-  float* acc0 = reinterpret_cast<float*>(reinterpret_cast<char*>(ws) + kTicketBytes + kTcAmaxBytes);
+  float* acc0 = reinterpret_cast<float*>(reinterpret_cast<char*>(ws) + kTicketBytes);
   float* zacc[2] = {acc0, acc0 + zmax * cols};
   float* yacc[2] = {acc0 + 2 * zmax * cols, acc0 + (2 * zmax + ymax) * cols};
   int* err = device_error_word();
@@ -331,15 +322,6 @@ lr_status_t run_chain_tc(const HostStep* steps, int n_steps, const void* x, int 
         act_ld = src.d[h.input_proj].d_out;
       }
       cudaError_t e;
-      if (i8) {  // per-token scales of the input's int8 codes (zero on entry)
-        TcAmaxParams a;
-        std::memset(&a, 0, sizeof(a));
-        a.nsrc = 1;
-        a.nb = nb;
-        a.src[0] = TcAmaxSrc{act, act_kind, h.d[0].d_in, act_ld, amax};
-        e = launch_tc_amax(a, stream);
-        if (e != cudaSuccess) return from_cuda(e);
-      }
       // ---- product 1: z_p = x A_p ----
       TcMaps maps;
       TcGemvParams g;
@@ -356,9 +338,7 @@ lr_status_t run_chain_tc(const HostStep* steps, int n_steps, const void* x, int 
         g.pre.zero_floats[0] = ymax * cols;
         g.pre.zero[1] = zacc[(s - 1) & 1];           // consumed by step s-1's second product
         g.pre.zero_floats[1] = zmax * cols;
-        g.pre.zero[2] = amax + kTcMaxPass;           // the latent maxima of step s-1
-        g.pre.zero_floats[2] = 4 * kTcMaxPass;
-        g.pre.nz = 3;
+        g.pre.nz = 2;
       }
       size_t zoff = 0;
       for (int p = 0; p < h.n; ++p) {
@@ -367,7 +347,6 @@ lr_status_t run_chain_tc(const HostStep* steps, int n_steps, const void* x, int 
         TcSeg& sg = g.seg[p];
         sg.row_scale = i8 ? d.scale_A : nullptr;
         sg.row_scale_f16 = scale_f16;
-        sg.tok_amax = amax;
         sg.M = active(&d);
         sg.K = d.d_in;
         sg.a_mn_major = 0;
@@ -380,27 +359,9 @@ lr_status_t run_chain_tc(const HostStep* steps, int n_steps, const void* x, int 
       }
       e = tc_product(maps, g, sms, i8, stream);
       if (e != cudaSuccess) return from_cuda(e);
-      if (i8) {  // per-token scales of each projection's latent
-        TcAmaxParams a;
-        std::memset(&a, 0, sizeof(a));
-        a.nsrc = h.n;
-        a.nb = nb;
-        zoff = 0;
-        for (int p = 0; p < h.n; ++p) {
-          a.src[p] = TcAmaxSrc{z + zoff * cols, 1, active(&h.d[p]), int(tc_zld(h.d[p])), amax + (p + 1) * kTcMaxPass};
-          zoff += tc_zld(h.d[p]);
-        }
-        e = launch_tc_amax(a, stream);
-        if (e != cudaSuccess) return from_cuda(e);
-      }
       // ---- product 2: y_p = z_p B_p ----
       std::memset(&maps, 0, sizeof(maps));
       std::memset(&g.pre, 0, sizeof(g.pre));
-      if (i8) {
-        g.pre.zero[0] = amax;                        // the input maximum, read by product 1 only
-        g.pre.zero_floats[0] = kTcMaxPass;
-        g.pre.nz = 1;
-      }
       g.hilo = 1;
       g.N = std::max(16, 2 * nh);
       zoff = 0;
@@ -411,7 +372,6 @@ lr_status_t run_chain_tc(const HostStep* steps, int n_steps, const void* x, int 
         TcSeg& sg = g.seg[p];
         sg.row_scale = i8 ? d.scale_B : nullptr;
         sg.row_scale_f16 = scale_f16;
-        sg.tok_amax = amax + (p + 1) * kTcMaxPass;
         sg.M = d.d_out;
         sg.K = active(&d);
         sg.a_mn_major = 1;
@@ -426,7 +386,7 @@ lr_status_t run_chain_tc(const HostStep* steps, int n_steps, const void* x, int 
       e = tc_product(maps, g, sms, i8, stream);
       if (e != cudaSuccess) return from_cuda(e);
     }
-    // the last step: outputs (clearing its y set), its latent set, the other y set, the maxima
+    // the last step: outputs (clearing its y set), its latent set, the other y set
     const int last = n_steps - 1;
     TcFinalizeParams f;
     std::memset(&f, 0, sizeof(f));
@@ -436,9 +396,7 @@ lr_status_t run_chain_tc(const HostStep* steps, int n_steps, const void* x, int 
     f.zero_floats[0] = zmax * cols;
     f.zero[1] = yacc[(last + 1) & 1];
     f.zero_floats[1] = ymax * cols;
-    f.zero[2] = amax;
-    f.zero_floats[2] = 5 * kTcMaxPass;
-    f.nz = 3;
+    f.nz = 2;
     cudaError_t e = launch_tc_finalize(f, sms, stream);
     if (e != cudaSuccess) return from_cuda(e);
   }
@@ -620,13 +578,11 @@ lr_status_t lr_linear(const lr_factor_desc_t* desc, const void* x, const float* 
     P.y = y;
     char* w = reinterpret_cast<char*>(ws);
     P.rank_pad = int(round_up(size_t(r), 128));
-    P.z = reinterpret_cast<float*>(w);
-    w += round_up(size_t(batch) * r * 4, 256);
+    P.acc = reinterpret_cast<int32_t*>(w);
+    w += round_up(size_t(batch) * P.rank_pad * 4, 256);
     P.zq = reinterpret_cast<int8_t*>(w);
     w += round_up(size_t(round_up(batch, 128)) * P.rank_pad, 256);
     P.sz = reinterpret_cast<float*>(w);
-    w += round_up(size_t(round_up(batch, 128)) * 4, 256);
-    P.amax = reinterpret_cast<unsigned int*>(w);
     P.err = device_error_word();
     return from_cuda(launch_w8a8(P, sm_count_current(), s));
   }
@@ -738,44 +694,50 @@ static lr_status_t check_ffn(const lr_ffn_desc_t* d) {
 
 // On the tensor-core path the FFN keeps token-major fp32 accumulators: z [rank],
 // gu [2 n_lr], dd [2 n_dense], h [inter], y [hidden] per token (rows 8-float
-// aligned) for cols tokens, zero on entry and exit, and three per-token maxima.
+// aligned) for cols tokens, zero on entry and exit.
 static size_t ffn_tc_floats_per_token(const lr_ffn_desc_t* d) {
   return round_up(size_t(d->n_lr > 0 ? d->rank : 0), 8) + 2 * size_t(d->inter) + round_up(size_t(d->inter), 8) +
          size_t(d->hidden);
 }
+
+// Up to this many tokens in a pass the down projection evaluates the SwiGLU
+// while it stages h (each of its row tiles repeats it for its slice); above
+// it a SwiGLU kernel writes h once.
+constexpr int kFusedSwigluMaxTokens = 4;
 
 static size_t ffn_ws_bytes(const lr_ffn_desc_t* d, int batch) {
   const int chunk = std::min(batch, kMaxDecodeChunk);
   const int n_dense = d->inter - d->n_lr;
   size_t b = kTicketBytes + round_up(size_t(chunk) * 2 * d->n_lr * 4, 256) + round_up(size_t(chunk) * n_dense * 4, 256) +
              round_up(size_t(chunk) * d->hidden * 4, 256);
-  if (use_tc_ffn(batch))
-    b = std::max(b, kTicketBytes + kTcAmaxBytes + ffn_tc_floats_per_token(d) * size_t(tc_cols(batch)) * 4);
+  if (use_tc_ffn(batch)) b = std::max(b, kTicketBytes + ffn_tc_floats_per_token(d) * size_t(tc_cols(batch)) * 4);
   return b;
 }
 
 // The hybrid FFN on the tensor cores (int8 weights, kind::i8), per pass of up
-// to kTcMaxPass tokens:
-//   max |x|    per token (scales of x's int8 codes)
+// to kTcMaxPass tokens (every product scales its int8 activation codes per
+// token over each unit's slice of the reduction):
 //   product 1: z += A' x (low-rank latent) and dd += D x (dense gate/up), scaled per row
-//   max |z|    per token
 //   product 2: gu += B'^T z (low-rank gate/up), scaled per column of B'
-//   SwiGLU:    h = silu(g) u over both branches and max |h| per token (clears gu, dd; zeroes z)
-//   product 3: y += W_down^T h, scaled per output column
-//   finalize:  y (bf16), clearing the y accumulator; zeroes h
+//   up to kFusedSwigluMaxTokens tokens:
+//     product 3: y += W_down^T h with h = silu(g) u of both branches, evaluated
+//                while the product stages its activations; it first zeroes z
+//     finalize:  y (bf16), clearing the y accumulator; zeroes gu and dd
+//   more tokens:
+//     SwiGLU:    h = silu(g) u (clears gu, dd; zeroes z)
+//     product 3: y += W_down^T h
+//     finalize:  y (bf16), clearing the y accumulator; zeroes h
 static lr_status_t run_ffn_tc(const lr_ffn_desc_t* d, const void* x, int batch, void* y, void* ws,
                               cudaStream_t stream) {
   const int cols = tc_cols(batch);
   const int n_dense = d->inter - d->n_lr;
   const int rz = d->n_lr > 0 ? int(round_up(size_t(d->rank), 8)) : 0;
-  const int hld = int(round_up(size_t(d->inter), 8));
-  float* amax = reinterpret_cast<float*>(reinterpret_cast<char*>(ws) + kTicketBytes);  // x, z, h
-  float* zacc = reinterpret_cast<float*>(reinterpret_cast<char*>(ws) + kTicketBytes + kTcAmaxBytes);
+  float* zacc = reinterpret_cast<float*>(reinterpret_cast<char*>(ws) + kTicketBytes);
   float* gu = zacc + size_t(rz) * cols;
   float* dd = gu + size_t(2 * d->n_lr) * cols;
+  const int hld = int(round_up(size_t(d->inter), 8));
   float* h = dd + size_t(2 * n_dense) * cols;
   float* yacc = h + size_t(hld) * cols;
-  float *ax = amax, *az = amax + kTcMaxPass, *ah = amax + 2 * kTcMaxPass;
   int* err = device_error_word();
   const int sms = sm_count_current();
   const int f16 = d->scale_dtype == LR_F16 ? 1 : 0;
@@ -785,8 +747,7 @@ static lr_status_t run_ffn_tc(const lr_ffn_desc_t* d, const void* x, int batch, 
     const int N = std::max(16, 2 * nh);
     const void* xb = reinterpret_cast<const char*>(x) + size_t(b0) * d->hidden * 2;
     auto seg = [&](TcGemvParams& g, TcMaps& maps, int i, const void* W, int rows, int cols_w, int mn, int M, int K,
-                   const void* act, int act_kind, int act_ld, float* out, int out_ld, const void* rs,
-                   const float* am) -> bool {
+                   const void* act, int act_kind, int act_ld, float* out, int out_ld, const void* rs) -> bool {
       if (!weight_map(&maps.m[i], W, rows, cols_w, mn, true)) return false;
       TcSeg& sg = g.seg[i];
       sg.M = M;
@@ -799,17 +760,9 @@ static lr_status_t run_ffn_tc(const lr_ffn_desc_t* d, const void* x, int batch, 
       sg.out_ld = out_ld;
       sg.row_scale = rs;
       sg.row_scale_f16 = f16;
-      sg.tok_amax = am;
       g.nseg = i + 1;
       return true;
     };
-    TcAmaxParams am;
-    std::memset(&am, 0, sizeof(am));
-    am.nsrc = 1;
-    am.nb = nb;
-    am.src[0] = TcAmaxSrc{xb, 0, d->hidden, d->hidden, ax};
-    cudaError_t e = launch_tc_amax(am, stream);
-    if (e != cudaSuccess) return from_cuda(e);
     TcMaps maps;
     TcGemvParams g;
     std::memset(&maps, 0, sizeof(maps));
@@ -820,43 +773,53 @@ static lr_status_t run_ffn_tc(const lr_ffn_desc_t* d, const void* x, int batch, 
     g.err = err;
     int i = 0;
     if (d->n_lr > 0 &&
-        !seg(g, maps, i++, d->A, d->rank, d->hidden, 0, d->rank, d->hidden, xb, 0, d->hidden, zacc, rz, d->s_A, ax))
+        !seg(g, maps, i++, d->A, d->rank, d->hidden, 0, d->rank, d->hidden, xb, 0, d->hidden, zacc, rz, d->s_A))
       return LR_ERR_CUDA;
     if (n_dense > 0 && !seg(g, maps, i++, d->D, 2 * n_dense, d->hidden, 0, 2 * n_dense, d->hidden, xb, 0,
-                            d->hidden, dd, 2 * n_dense, d->s_D, ax))
+                            d->hidden, dd, 2 * n_dense, d->s_D))
       return LR_ERR_CUDA;
-    e = tc_product(maps, g, sms, true, stream);
+    cudaError_t e = tc_product(maps, g, sms, true, stream);
     if (e != cudaSuccess) return from_cuda(e);
     if (d->n_lr > 0) {
-      am.src[0] = TcAmaxSrc{zacc, 1, d->rank, rz, az};
-      e = launch_tc_amax(am, stream);
-      if (e != cudaSuccess) return from_cuda(e);
       std::memset(&maps, 0, sizeof(maps));
-      if (!seg(g, maps, 0, d->B, d->rank, 2 * d->n_lr, 1, 2 * d->n_lr, d->rank, zacc, 1, rz, gu, 2 * d->n_lr, d->s_B,
-               az))
+      if (!seg(g, maps, 0, d->B, d->rank, 2 * d->n_lr, 1, 2 * d->n_lr, d->rank, zacc, 1, rz, gu, 2 * d->n_lr, d->s_B))
         return LR_ERR_CUDA;
       g.nseg = 1;
       e = tc_product(maps, g, sms, true, stream);
       if (e != cudaSuccess) return from_cuda(e);
     }
-    TcSwigluParams sw;
-    std::memset(&sw, 0, sizeof(sw));
-    sw.gu = gu;
-    sw.dd = dd;
-    sw.h = h;
-    sw.h_ld = hld;
-    sw.h_amax = ah;
-    sw.n_lr = d->n_lr;
-    sw.n_dense = n_dense;
-    sw.nb = nb;
-    sw.zero = rz ? zacc : nullptr;
-    sw.zero_row = rz;
-    e = launch_tc_swiglu(sw, sms, stream);
-    if (e != cudaSuccess) return from_cuda(e);
+    const bool fused = nb <= kFusedSwigluMaxTokens;
     std::memset(&maps, 0, sizeof(maps));
-    if (!seg(g, maps, 0, d->W_down, d->inter, d->hidden, 1, d->hidden, d->inter, h, 1, hld, yacc, d->hidden,
-             d->s_down, ah))
-      return LR_ERR_CUDA;
+    if (fused) {
+      if (!seg(g, maps, 0, d->W_down, d->inter, d->hidden, 1, d->hidden, d->inter, gu, 2, 2 * d->n_lr, yacc,
+               d->hidden, d->s_down))
+        return LR_ERR_CUDA;
+      g.seg[0].act2 = dd;
+      g.seg[0].act2_ld = 2 * n_dense;
+      g.seg[0].n_lr = d->n_lr;
+      if (rz > 0) {   // the latent, read by product 2 only
+        g.pre.zero[0] = zacc;
+        g.pre.zero_floats[0] = size_t(rz) * cols;
+        g.pre.nz = 1;
+      }
+    } else {
+      TcSwigluParams sw;
+      std::memset(&sw, 0, sizeof(sw));
+      sw.gu = gu;
+      sw.dd = dd;
+      sw.h = h;
+      sw.h_ld = hld;
+      sw.n_lr = d->n_lr;
+      sw.n_dense = n_dense;
+      sw.nb = nb;
+      sw.zero = rz ? zacc : nullptr;
+      sw.zero_row = rz;
+      e = launch_tc_swiglu(sw, stream);
+      if (e != cudaSuccess) return from_cuda(e);
+      if (!seg(g, maps, 0, d->W_down, d->inter, d->hidden, 1, d->hidden, d->inter, h, 1, hld, yacc, d->hidden,
+               d->s_down))
+        return LR_ERR_CUDA;
+    }
     g.nseg = 1;
     e = tc_product(maps, g, sms, true, stream);
     if (e != cudaSuccess) return from_cuda(e);
@@ -868,11 +831,14 @@ static lr_status_t run_ffn_tc(const lr_ffn_desc_t* d, const void* x, int batch, 
     f.t[0].acc = yacc;
     f.t[0].y = reinterpret_cast<char*>(y) + size_t(b0) * d->hidden * 2;
     f.t[0].M = d->hidden;
-    f.zero[0] = h;
-    f.zero_floats[0] = size_t(hld) * cols;
-    f.zero[1] = amax;   // the per-token maxima are raised with atomicMax: zero for the next pass
-    f.zero_floats[1] = 3 * kTcMaxPass;
-    f.nz = 2;
+    if (fused) {
+      f.zero[0] = gu;   // the gate/up accumulators of both branches, read by product 3
+      f.zero_floats[0] = size_t(2 * d->inter) * cols;
+    } else {
+      f.zero[0] = h;    // read by product 3
+      f.zero_floats[0] = size_t(hld) * cols;
+    }
+    f.nz = 1;
     e = launch_tc_finalize(f, sms, stream);
     if (e != cudaSuccess) return from_cuda(e);
   }
@@ -1189,7 +1155,7 @@ lr_status_t lr_gemm_s8s32(const int8_t* A, const int8_t* B, int b_layout, int M,
   if (b_layout != 0 && b_layout != 1) return LR_ERR_INVALID_ARG;
   if ((K % 16) != 0 || (N % 16) != 0 || K >= 133144) return LR_ERR_UNSUPPORTED;
   if (!al16(A) || !al16(B) || !al16(C)) return LR_ERR_MISALIGNED;
-  return from_cuda(launch_gemm_s8s32(A, B, b_layout, M, N, K, C, device_error_word(),
+  return from_cuda(launch_gemm_s8s32(A, B, b_layout, M, N, K, C, device_error_word(), sm_count_current(),
                                      reinterpret_cast<cudaStream_t>(stream)));
 }
 

@@ -139,13 +139,19 @@ struct TcSeg {
   int M, K;           // weight rows (outputs) and reduction length
   int a_mn_major;     // 0: W stored [M, K]; 1: W stored [K, M] (its tensor map in TcMaps)
   int m_tiles, k_splits, kc, unit0;
-  const void* act;    // token-major [nb, K], row stride act_ld (a multiple of 8): act_kind 0 bf16, 1 fp32
+  // The activations, token-major [nb, K] with row stride act_ld (a multiple of 8):
+  // act_kind 0 bf16, 1 fp32; act_kind 2 the SwiGLU of the hybrid FFN, h[n][c] =
+  // silu(g) u with the interleaved gate/up pair of channel c from the fp32
+  // accumulators act [nb, 2 n_lr] (c < n_lr, row stride act_ld) or act2
+  // [nb, 2 (K - n_lr)] (the dense channels, row stride act2_ld).
+  const void* act;
   int act_kind, act_ld;
+  const float* act2;
+  int act2_ld, n_lr;
   float* out;         // token-major fp32 [nb, out_ld], out[n][m] += product
   int out_ld;
   const void* row_scale;  // int8 weights: one scale per weight row (output channel), or null
   int row_scale_f16;
-  const float* tok_amax;  // int8 weights: per-token max |act| over the whole row
 };
 struct TcFinalTarget {
   const float* acc;   // token-major fp32 [nb, M]
@@ -169,6 +175,7 @@ struct TcGemvParams {
   int nb;             // tokens
   int hilo;           // split each fp32 activation into bf16 high and low parts (rows nb.. of the operand)
   int tmem_cols;
+  int stages;         // weight ring depth (set by launch_tc_gemv)
   int* err;
   TcFinalizeParams pre;  // finalize work of the preceding step, spread over the units (after the dependency wait)
 };
@@ -176,7 +183,7 @@ struct alignas(64) TcMaps {
   CUtensorMap m[4];
 };
 int tc_gemv_kc(int K, int k_splits, bool i8);
-size_t tc_gemv_smem(int kc, int N, bool i8);
+size_t tc_gemv_smem(int kc, int N, bool i8, int stages);
 bool tc_gemv_fits(int kc, int N, bool i8);
 bool tc_make_weight_map(CUtensorMap* m, const void* W, int rows, int cols, int a_mn_major, bool i8);
 cudaError_t launch_tc_gemv(const TcMaps& maps, const TcGemvParams& p, bool i8, cudaStream_t s);
@@ -186,22 +193,11 @@ struct TcSwigluParams {
   float* dd;          // token-major [nb, 2 n_dense] of the dense channels
   float* h;           // token-major [nb, h_ld], h_ld >= n_lr + n_dense
   int h_ld;
-  float* h_amax;      // [nb] max |h| per token (fp32 bits raised with atomicMax; zero on entry)
   int n_lr, n_dense, nb;
   float* zero;        // token-major rows of zero_row floats zeroed afterwards (or null)
   int zero_row;
 };
-cudaError_t launch_tc_swiglu(const TcSwigluParams& p, int sm_count, cudaStream_t s);
-struct TcAmaxSrc {
-  const void* act;    // token-major [nb, K], row stride ld: kind 0 bf16, 1 fp32
-  int kind, K, ld;
-  float* amax;        // [nb], raised with atomicMax (zero on entry)
-};
-struct TcAmaxParams {
-  TcAmaxSrc src[4];
-  int nsrc, nb;
-};
-cudaError_t launch_tc_amax(const TcAmaxParams& p, cudaStream_t s);
+cudaError_t launch_tc_swiglu(const TcSwigluParams& p, cudaStream_t s);
 struct TcScatterParams {
   float* acc;         // token-major fp32 [nb, 2 heads rank], cleared
   void* cache_k;      // bf16 [nb, heads, ctx, rank], offset to the pass's first sequence
@@ -235,17 +231,16 @@ struct W8A8Params {
   const int8_t* Aq; const float* sA;
   const int8_t* Bq; const float* sB;
   void* y;            // bf16 [T, d_out]
-  float* z;           // [T, rank] fp32 workspace
+  int32_t* acc;       // [T, rank_pad] int32 sums of the first product (zero between calls)
   int8_t* zq;         // [T, rank_pad] int8 workspace
   float* sz;          // [T]
-  unsigned int* amax; // [T] row max |z| as fp32 bits (zero between calls)
   int rank_pad;
   int* err;           // device error word
 };
 
 size_t w8a8_workspace_bytes(int T, int rank);
 cudaError_t launch_gemm_s8s32(const int8_t* A, const int8_t* B, int b_kn, int M, int N, int K, int32_t* C,
-                              int* err, cudaStream_t s);
+                              int* err, int sm_count, cudaStream_t s);
 cudaError_t launch_w8a8(const W8A8Params& p, int sm_count, cudaStream_t s);
 
 }  // namespace lr

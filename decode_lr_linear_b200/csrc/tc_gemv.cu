@@ -16,11 +16,15 @@
 // (128-byte swizzle) through a 4-stage ring, all threads stage the unit's
 // activations once as the N x K operand (bf16, same swizzle; an fp32 source is
 // split into bf16 high and low parts in separate columns, so the product keeps
-// fp32 accuracy), warp 1 lane 0 issues tcgen05.mma kind::f16 into a TMEM
-// accumulator, and all four warps add the 128 x N partial product into an fp32
-// accumulator in L2 (red.global.add.v4.f32).  A finalize kernel turns the
-// accumulators into bf16 outputs and zeroes them.  Every wait is bounded and
-// records a device error instead of hanging.
+// fp32 accuracy; for int8 weights, two int8 codes per value with scales from
+// the slice's own per-token maxima), warp 1 lane 0 issues tcgen05.mma into a
+// TMEM accumulator, and all four warps add the 128 x N partial product into
+// an fp32 accumulator in L2.  For a few tokens the hybrid FFN's SwiGLU is
+// evaluated while its down projection stages h from the gate/up accumulators
+// (no kernel of its own); for more, a SwiGLU kernel writes h once, since every
+// tile of the down projection would repeat it.  A finalize kernel turns the accumulators into bf16
+// outputs and zeroes them.  Every wait is bounded and records a device error
+// instead of hanging.
 #include <algorithm>
 #include <cstring>
 
@@ -33,13 +37,13 @@ namespace {
 
 constexpr int kBM = 128;                 // weight rows per unit (TMEM lanes)
 constexpr int kKBytes = 128;             // k-block: one 128-byte swizzle row (64 bf16 or 128 int8)
-constexpr int kStages = 4;
-constexpr int kThreads = 128;
+constexpr int kStages = 4;                // ring depth, 3 where that keeps two CTAs per SM
+constexpr size_t kTwoPerSm = 112 * 1024;  // dynamic shared memory per CTA with two CTAs per SM
+constexpr int kThreads = 256;          // 8 warps: all stage the activations; two per TMEM lane quarter in the epilogue
 constexpr int kATile = kBM * kKBytes;    // 16 KiB
 constexpr size_t kSmemCap = 200 * 1024;
 constexpr int kMaxTokens = 64;           // operand rows (tokens, or high and low parts)
 constexpr int kSwigluChunk = 1024;       // channels per SwiGLU CTA
-constexpr int kAmaxChunk = 2048;         // row elements per max CTA
 
 // Byte offset of byte `kb` of row n in a K-major, 128-byte-swizzled operand block
 // (rows of 128 bytes; the 16-byte chunk index is XORed with row bits 0..2).
@@ -86,13 +90,36 @@ LR_DEV void load_act8(const TcSeg& g, int n, int k, int k1, float* v) {
   }
 }
 
+// kPer activations of token n from reduction index k (0 at k >= k1), any
+// source kind; k is a multiple of 8.
+template <int kPer>
+LR_DEV void fetch_act(const TcSeg& g, int n, int k, int k1, float* v) {
+  if (g.act_kind != 2) {
+#pragma unroll
+    for (int h = 0; h < kPer; h += 8) load_act8(g, n, k + h, k1, v + h);
+    return;
+  }
+  const float* gu = reinterpret_cast<const float*>(g.act) + size_t(n) * g.act_ld;
+  const float* dd = g.act2 + size_t(n) * g.act2_ld;
+#pragma unroll
+  for (int e = 0; e < kPer; ++e) {
+    const int c = k + e;
+    v[e] = 0.f;
+    if (c < k1) {
+      const float2 p = __ldcg(reinterpret_cast<const float2*>(c < g.n_lr ? gu + 2 * c : dd + 2 * (c - g.n_lr)));
+      v[e] = silu(p.x) * p.y;
+    }
+  }
+}
+
 LR_DEV void finalize_part(const TcFinalizeParams& F, int part, int parts, int t, int nt);
 
 // I8 = false: bf16 weights, kind::f16, bf16 operand rows (fp32 sources as high +
 // low parts).  I8 = true: int8 weights, kind::i8, every activation as two int8
-// codes with per-token scales s1 = max|x| / 127 over the token's whole input
-// (tok_amax, from tc_amax_kernel or the kernel that produced the input) and
-// s2 = s1 / 254: x ~ s1 hi + s2 lo with |error| <= s1 / 508.
+// codes with per-token scales s1 = max|x| / 127 over the unit's slice of the
+// token's input and s2 = s1 / 254: x ~ s1 hi + s2 lo with |error| <= s1 / 508.
+// Each unit converts its int32 partial product with its own scales before
+// adding it into the fp32 accumulator, so no scale is shared between units.
 template <bool I8>
 __global__ void __launch_bounds__(kThreads) tc_gemv_kernel(const __grid_constant__ TcMaps maps,
                                                            const __grid_constant__ TcGemvParams P) {
@@ -104,6 +131,7 @@ __global__ void __launch_bounds__(kThreads) tc_gemv_kernel(const __grid_constant
   __shared__ uint32_t tmem_slot;
   __shared__ float s_scale[2][kMaxTokens];   // I8: per-token scales of the high and low codes
   __shared__ float s_inv[2][kMaxTokens];     // and their reciprocals (codes by multiplication)
+  __shared__ unsigned int s_amax[kMaxTokens];  // I8: per-token max |x| over the slice (fp32 bits)
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;      // ring: 1024-byte aligned tiles
   unsigned char* gbase = smem_raw + (base - raw);
@@ -119,12 +147,13 @@ __global__ void __launch_bounds__(kThreads) tc_gemv_kernel(const __grid_constant
   const int nkb = (k1 - k0 + kKB - 1) / kKB;
   const int N = P.N;
   const int nh = P.hilo ? N / 2 : N;          // token rows; with high/low parts, rows nh.. hold the low parts
-  const uint32_t act = base + uint32_t(kStages) * kATile;   // nkb blocks of N rows x 128 B
-  unsigned char* act_g = gbase + size_t(kStages) * kATile;
+  const int stages = P.stages;
+  const uint32_t act = base + uint32_t(stages) * kATile;   // nkb blocks of N rows x 128 B
+  unsigned char* act_g = gbase + size_t(stages) * kATile;
   const CUtensorMap* map = &maps.m[s];
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kStages; ++i) {
+    for (int i = 0; i < stages; ++i) {
       mbar_init(&full[i], 1);
       mbar_init(&empty[i], 1);
     }
@@ -140,7 +169,7 @@ __global__ void __launch_bounds__(kThreads) tc_gemv_kernel(const __grid_constant
 
   // weights are never written by an earlier kernel: the first stages stream before the dependency wait
   auto load_stage = [&](int kb) {
-    const int st = kb % kStages;
+    const int st = kb % stages;
     const uint32_t dst = base + uint32_t(st) * kATile;
     mbar_arrive_expect_tx(&full[st], kATile);
     if (!g.a_mn_major) {
@@ -153,70 +182,144 @@ __global__ void __launch_bounds__(kThreads) tc_gemv_kernel(const __grid_constant
     }
   };
   if (warp == 0 && lane == 0)
-    for (int kb = 0; kb < min(nkb, kStages); ++kb) load_stage(kb);
+    for (int kb = 0; kb < min(nkb, stages); ++kb) load_stage(kb);
 
   // ---- the activations of this unit as the N x K operand (zero outside the data) ----
   pdl_wait();
   // the preceding step's finalize, spread over this launch's units (outputs and clearing)
   if (P.pre.nt > 0 || P.pre.nz > 0) finalize_part(P.pre, blockIdx.x, gridDim.x, threadIdx.x, kThreads);
-  if constexpr (I8) {
-    if (threadIdx.x < nh) {
-      const float a = threadIdx.x < P.nb ? g.tok_amax[threadIdx.x] : 0.f;
-      const float s1 = a > 0.f ? a / 127.f : 1.f;
-      s_scale[0][threadIdx.x] = s1;
-      s_scale[1][threadIdx.x] = s1 / 254.f;
-      s_inv[0][threadIdx.x] = 1.f / s1;
-      s_inv[1][threadIdx.x] = 254.f / s1;
-    }
-    __syncthreads();
-  }
   {
-    // chunk c: k-block kb, token n, 16 bytes of the 128-byte operand row (8 bf16 or 16 int8 codes);
-    // the reduction index varies fastest, so a thread's loads are contiguous
-    constexpr int kPer = I8 ? 16 : 8;
-    const int chunks = nkb * nh * 8;
-    for (int c = threadIdx.x; c < chunks; c += kThreads) {
-      const int kb = c / (nh * 8), rem = c % (nh * 8), n = rem / 8, kci = rem % 8;
-      const int k = k0 + kb * kKB + kci * kPer;
-      float v[kPer];
-#pragma unroll
-      for (int e = 0; e < kPer; ++e) v[e] = 0.f;
-      if (n < P.nb && k < k1) {
-        load_act8(g, n, k, k1, v);
-        if constexpr (I8) load_act8(g, n, k + 8, k1, v + 8);
-      }
-      uint32_t hi[4], lo[4];
-      if constexpr (I8) {
-        // codes by multiplication with the reciprocal scales: the result is any integer pair whose
-        // error against x stays within s2 / 2 plus rounding; the epilogue uses s1, s2 themselves
-        const float s1 = s_scale[0][n], i1 = s_inv[0][n], i2 = s_inv[1][n];
-#pragma unroll
-        for (int w = 0; w < 4; ++w) {
-          uint32_t ph = 0, pl = 0;
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float x = v[4 * w + e];
-            const float qh = fminf(fmaxf(rintf(x * i1), -127.f), 127.f);
-            const float ql = fminf(fmaxf(rintf(fmaf(-qh, s1, x) * i2), -127.f), 127.f);
-            ph |= (uint32_t(int(qh)) & 0xffu) << (8 * e);
-            pl |= (uint32_t(int(ql)) & 0xffu) << (8 * e);
-          }
-          hi[w] = ph;
-          lo[w] = pl;
-        }
-      } else {
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * e], v[2 * e + 1]);
-          hi[e] = *reinterpret_cast<const uint32_t*>(&h);
-          const float2 hf = __bfloat1622float2(h);
-          const __nv_bfloat162 l = __floats2bfloat162_rn(v[2 * e] - hf.x, v[2 * e + 1] - hf.y);
-          lo[e] = *reinterpret_cast<const uint32_t*>(&l);
-        }
-      }
+    // Token n's 16-byte piece kci of k-block kb is chunk c = (kb * nb + n) * 8 + kci
+    // (the reduction index varies fastest, so neighbouring threads load
+    // neighbouring bytes).  Only real tokens are staged: the accumulator
+    // columns of padding tokens are never read.  Pieces past k1 are zero (the
+    // weights there are zero-filled, and zero times stale bytes could be NaN).
+    // Each thread issues the loads of up to kHold pieces before it uses any.
+    constexpr int kPer = I8 ? 16 : 8;   // activations per 16-byte piece of the operand row
+    constexpr int kHold = 4;
+    const int vchunks = nkb * P.nb * 8;
+    const int step = kHold * kThreads;
+    float v[kHold][kPer];
+    auto piece = [&](int c, int& kb, int& n, int& k) {
+      kb = c / (P.nb * 8);
+      const int rem = c - kb * P.nb * 8;
+      n = rem >> 3;
+      k = k0 + kb * kKB + (rem & 7) * kPer;
+    };
+    auto store = [&](int kb, int n, int kci, const uint32_t* hi, const uint32_t* lo) {
       unsigned char* blk = act_g + size_t(kb) * N * 128;
       *reinterpret_cast<uint4*>(blk + sw128_offset(n, kci * 16)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-      if (P.hilo) *reinterpret_cast<uint4*>(blk + sw128_offset(nh + n, kci * 16)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+      if (P.hilo)
+        *reinterpret_cast<uint4*>(blk + sw128_offset(nh + n, kci * 16)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+    };
+    if constexpr (I8) {
+      if (threadIdx.x < kMaxTokens) s_amax[threadIdx.x] = 0u;
+      __syncthreads();
+      // pass 1: the slice's per-token maxima
+      for (int c0 = 0; c0 < vchunks; c0 += step) {
+#pragma unroll
+        for (int i = 0; i < kHold; ++i) {
+          const int c = c0 + i * kThreads + threadIdx.x;
+          if (c < vchunks) {
+            int kb, n, k;
+            piece(c, kb, n, k);
+            fetch_act<kPer>(g, n, k, k1, v[i]);
+          }
+        }
+#pragma unroll
+        for (int i = 0; i < kHold; ++i) {
+          const int c = c0 + i * kThreads + threadIdx.x;
+          if (c < vchunks) {
+            float m = 0.f;
+#pragma unroll
+            for (int e = 0; e < kPer; ++e) m = fmaxf(m, fabsf(v[i][e]));
+            atomicMax(&s_amax[(c % (P.nb * 8)) >> 3], __float_as_uint(m));
+          }
+        }
+      }
+      __syncthreads();
+      if (threadIdx.x < P.nb) {
+        const float a = __uint_as_float(s_amax[threadIdx.x]);
+        const float s1 = a > 0.f ? a / 127.f : 1.f;
+        s_scale[0][threadIdx.x] = s1;
+        s_scale[1][threadIdx.x] = s1 / 254.f;
+        s_inv[0][threadIdx.x] = 1.f / s1;
+        s_inv[1][threadIdx.x] = 254.f / s1;
+      }
+      __syncthreads();
+      // pass 2: int8 high and low codes; the registers still hold the pieces only when pass 1
+      // took a single round, otherwise every round reads its pieces again
+      const bool held = vchunks <= step;
+      for (int c0 = 0; c0 < vchunks; c0 += step) {
+        if (!held) {
+#pragma unroll
+          for (int i = 0; i < kHold; ++i) {
+            const int c = c0 + i * kThreads + threadIdx.x;
+            if (c < vchunks) {
+              int kb, n, k;
+              piece(c, kb, n, k);
+              fetch_act<kPer>(g, n, k, k1, v[i]);
+            }
+          }
+        }
+#pragma unroll
+        for (int i = 0; i < kHold; ++i) {
+          const int c = c0 + i * kThreads + threadIdx.x;
+          if (c < vchunks) {
+            int kb, n, k;
+            piece(c, kb, n, k);
+            // codes by multiplication with the reciprocal scales: any integer pair whose error
+            // against x stays within s2 / 2 plus rounding; the epilogue uses s1, s2 themselves
+            const float s1 = s_scale[0][n], i1 = s_inv[0][n], i2 = s_inv[1][n];
+            uint32_t hi[4], lo[4];
+#pragma unroll
+            for (int w = 0; w < 4; ++w) {
+              uint32_t ph = 0, pl = 0;
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const float x = v[i][4 * w + e];
+                const float qh = fminf(fmaxf(rintf(x * i1), -127.f), 127.f);
+                const float ql = fminf(fmaxf(rintf(fmaf(-qh, s1, x) * i2), -127.f), 127.f);
+                ph |= (uint32_t(int(qh)) & 0xffu) << (8 * e);
+                pl |= (uint32_t(int(ql)) & 0xffu) << (8 * e);
+              }
+              hi[w] = ph;
+              lo[w] = pl;
+            }
+            store(kb, n, (c & 7), hi, lo);
+          }
+        }
+      }
+    } else {
+      for (int c0 = 0; c0 < vchunks; c0 += step) {
+#pragma unroll
+        for (int i = 0; i < kHold; ++i) {
+          const int c = c0 + i * kThreads + threadIdx.x;
+          if (c < vchunks) {
+            int kb, n, k;
+            piece(c, kb, n, k);
+            fetch_act<kPer>(g, n, k, k1, v[i]);
+          }
+        }
+#pragma unroll
+        for (int i = 0; i < kHold; ++i) {
+          const int c = c0 + i * kThreads + threadIdx.x;
+          if (c < vchunks) {
+            int kb, n, k;
+            piece(c, kb, n, k);
+            uint32_t hi[4], lo[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const __nv_bfloat162 h = __floats2bfloat162_rn(v[i][2 * e], v[i][2 * e + 1]);
+              hi[e] = *reinterpret_cast<const uint32_t*>(&h);
+              const float2 hf = __bfloat1622float2(h);
+              const __nv_bfloat162 l = __floats2bfloat162_rn(v[i][2 * e] - hf.x, v[i][2 * e + 1] - hf.y);
+              lo[e] = *reinterpret_cast<const uint32_t*>(&l);
+            }
+            store(kb, n, (c & 7), hi, lo);
+          }
+        }
+      }
     }
   }
   fence_proxy_async();  // generic-proxy writes of the operand before the tensor cores read it
@@ -224,9 +327,9 @@ __global__ void __launch_bounds__(kThreads) tc_gemv_kernel(const __grid_constant
 
   if (warp == 0) {
     if (lane == 0) {
-      for (int kb = kStages; kb < nkb; ++kb) {
-        const int st = kb % kStages;
-        if (!mbar_wait_bounded(&empty[st], uint32_t(kb / kStages - 1) & 1u, P.err)) break;
+      for (int kb = stages; kb < nkb; ++kb) {
+        const int st = kb % stages;
+        if (!mbar_wait_bounded(&empty[st], uint32_t(kb / stages - 1) & 1u, P.err)) break;
         load_stage(kb);
       }
     }
@@ -236,8 +339,8 @@ __global__ void __launch_bounds__(kThreads) tc_gemv_kernel(const __grid_constant
                                 : tc::idesc_bf16(kBM, N, g.a_mn_major != 0, false);
       bool ok = true;
       for (int kb = 0; kb < nkb && ok; ++kb) {
-        const int st = kb % kStages;
-        if (!mbar_wait_bounded(&full[st], uint32_t(kb / kStages) & 1u, P.err)) {
+        const int st = kb % stages;
+        if (!mbar_wait_bounded(&full[st], uint32_t(kb / stages) & 1u, P.err)) {
           ok = false;
           break;
         }
@@ -260,15 +363,17 @@ __global__ void __launch_bounds__(kThreads) tc_gemv_kernel(const __grid_constant
   }
   __syncwarp();  // roles end: every warp converges before the warp-wide tensor-memory loads
   // ---- epilogue: lane = weight row, N accumulator columns; add into the fp32 accumulator ----
+  // warps w and w + 4 read TMEM lanes 32 (w % 4) .. + 31 and take alternate groups of 16 columns
   const bool have = mbar_wait_bounded(&accum, 0u, P.err);
   tc::fence_after();
   if (have) {
-    const int row = m0 + warp * 32 + lane;
+    const int q = warp & 3;
+    const int row = m0 + q * 32 + lane;
     const float rs = (g.row_scale && row < g.M) ? load_scale(g.row_scale, row, g.row_scale_f16 != 0) : 1.f;
-    for (int c0 = 0; c0 < nh; c0 += 16) {
+    for (int c0 = (warp >> 2) * 16; c0 < nh; c0 += 32) {
       uint32_t v[16], w[16];
-      tmem_ld16(tmem + (uint32_t(warp * 32) << 16) + uint32_t(c0), v);
-      if (P.hilo) tmem_ld16(tmem + (uint32_t(warp * 32) << 16) + uint32_t(nh + c0), w);
+      tmem_ld16(tmem + (uint32_t(q * 32) << 16) + uint32_t(c0), v);
+      if (P.hilo) tmem_ld16(tmem + (uint32_t(q * 32) << 16) + uint32_t(nh + c0), w);
       if (row < g.M) {
         // token-major accumulator: out[n * out_ld + row]; a warp's 32 rows are contiguous for each n
 #pragma unroll
@@ -339,74 +444,30 @@ __global__ void __launch_bounds__(256) tc_finalize_kernel(const __grid_constant_
   finalize_part(F, blockIdx.x, gridDim.x, threadIdx.x, blockDim.x);
 }
 
-// SwiGLU of the hybrid FFN between its tensor-core products (token-major
+// SwiGLU of the hybrid FFN between its tensor-core products, for passes of
+// more tokens than the down projection evaluates while staging (token-major
 // accumulators), grid (tokens, channel chunks): h[n][c] = silu(g) u for
 // channel c, from the gate/up pair of the low-rank channels (c < n_lr:
 // gu[n][2c], gu[n][2c+1]) or of the dense ones (dd[n][2(c - n_lr)], +1); each
-// accumulator element is read and cleared by the thread that uses it.  The
-// token's max |h| (the scale of its int8 codes in the down projection) is
-// raised with atomicMax on its fp32 bits (non-negative, zero on entry), and the
+// accumulator element is read and cleared by the thread that uses it, and the
 // chunk-0 CTA zeroes the token's latent row (consumed by the preceding product).
 __global__ void __launch_bounds__(256) tc_swiglu_kernel(const __grid_constant__ TcSwigluParams S) {
   pdl_launch_dependents();
   pdl_wait();
-  __shared__ float red[8];
   const int n = blockIdx.x;
   const int inter = S.n_lr + S.n_dense;
   float* gu = S.gu + size_t(n) * 2 * S.n_lr;
   float* dd = S.dd + size_t(n) * 2 * S.n_dense;
-  float m = 0.f;
   const int c0 = blockIdx.y * kSwigluChunk, c1 = min(inter, c0 + kSwigluChunk);
   for (int c = c0 + int(threadIdx.x); c < c1; c += blockDim.x) {
     float2* src = reinterpret_cast<float2*>(c < S.n_lr ? gu + 2 * c : dd + 2 * (c - S.n_lr));
     const float2 gv = __ldcg(src);
     __stcg(src, make_float2(0.f, 0.f));
-    const float hv = silu(gv.x) * gv.y;
-    S.h[size_t(n) * S.h_ld + c] = hv;
-    m = fmaxf(m, fabsf(hv));
-  }
-  m = warp_max(m);
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    float a = red[0];
-    for (int w = 1; w < int(blockDim.x >> 5); ++w) a = fmaxf(a, red[w]);
-    atomicMax(reinterpret_cast<int*>(S.h_amax) + n, __float_as_int(a));
+    S.h[size_t(n) * S.h_ld + c] = silu(gv.x) * gv.y;
   }
   if (S.zero && blockIdx.y == 0) {
     float* z = S.zero + size_t(n) * S.zero_row;
     for (int i = threadIdx.x; i < S.zero_row; i += blockDim.x) __stcg(z + i, 0.f);
-  }
-}
-
-// Per-token max |x| over the row of each source (token-major, bf16 or fp32):
-// grid (tokens, sources); the scale of the token's int8 codes in the next product.
-__global__ void __launch_bounds__(256) tc_amax_kernel(const __grid_constant__ TcAmaxParams A) {
-  pdl_launch_dependents();
-  pdl_wait();
-  __shared__ float red[8];
-  const int n = blockIdx.x, s = blockIdx.y;
-  const TcAmaxSrc& src = A.src[s];
-  float m = 0.f;
-  // grid z: chunks of kAmaxChunk elements of the row, combined with atomicMax (zero on entry)
-  const int kend = min(src.K, int(blockIdx.z + 1) * kAmaxChunk);
-  for (int k = int(blockIdx.z) * kAmaxChunk + threadIdx.x * 8; k < kend; k += blockDim.x * 8) {
-    float v[8];
-    TcSeg g;
-    g.act = src.act;
-    g.act_kind = src.kind;
-    g.act_ld = src.ld;
-    load_act8(g, n, k, src.K, v);
-#pragma unroll
-    for (int e = 0; e < 8; ++e) m = fmaxf(m, fabsf(v[e]));
-  }
-  m = warp_max(m);
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    float a = red[0];
-    for (int w = 1; w < int(blockDim.x >> 5); ++w) a = fmaxf(a, red[w]);
-    atomicMax(reinterpret_cast<int*>(src.amax) + n, __float_as_int(a));
   }
 }
 
@@ -442,11 +503,11 @@ int tc_gemv_kc(int K, int k_splits, bool i8) {
   return ((K + k_splits - 1) / k_splits + e - 1) / e * e;
 }
 
-size_t tc_gemv_smem(int kc, int N, bool i8) {
-  return size_t(kStages) * kATile + size_t(kc / kb_elems(i8)) * N * 128 + 1024;
+size_t tc_gemv_smem(int kc, int N, bool i8, int stages) {
+  return size_t(stages) * kATile + size_t(kc / kb_elems(i8)) * N * 128 + 1024;
 }
 
-bool tc_gemv_fits(int kc, int N, bool i8) { return N <= kMaxTokens && tc_gemv_smem(kc, N, i8) <= kSmemCap; }
+bool tc_gemv_fits(int kc, int N, bool i8) { return N <= kMaxTokens && tc_gemv_smem(kc, N, i8, kStages) <= kSmemCap; }
 
 bool tc_make_weight_map(CUtensorMap* m, const void* W, int rows, int cols, int a_mn_major, bool i8) {
   // K-major: W [rows = M, cols = K], box 128 rows x one k-block; MN-major: W [rows = K,
@@ -465,7 +526,13 @@ cudaError_t launch_tc_gemv(const TcMaps& maps, const TcGemvParams& p, bool i8, c
     kc_max = std::max(kc_max, p.seg[i].kc);
   }
   if (!tc_gemv_fits(kc_max, p.N, i8) || (i8 && !p.hilo)) return cudaErrorInvalidValue;
-  const size_t smem = tc_gemv_smem(kc_max, p.N, i8);
+  // a 4-stage ring, or 3 stages where that is what keeps two CTAs on an SM (a wide
+  // activation operand, many tokens): the second CTA hides the first one's latency
+  TcGemvParams q = p;
+  q.stages = kStages;
+  if (tc_gemv_smem(kc_max, p.N, i8, kStages) > kTwoPerSm && tc_gemv_smem(kc_max, p.N, i8, kStages - 1) <= kTwoPerSm)
+    q.stages = kStages - 1;
+  const size_t smem = tc_gemv_smem(kc_max, p.N, i8, q.stages);
   auto kern = i8 ? tc_gemv_kernel<true> : tc_gemv_kernel<false>;
   cudaError_t e = ensure_smem(kern, smem);
   if (e != cudaSuccess) return e;
@@ -479,22 +546,7 @@ cudaError_t launch_tc_gemv(const TcMaps& maps, const TcGemvParams& p, bool i8, c
   c.stream = s;
   c.attrs = attr;
   c.numAttrs = 1;
-  return cudaLaunchKernelEx(&c, kern, maps, p);
-}
-
-cudaError_t launch_tc_amax(const TcAmaxParams& p, cudaStream_t s) {
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cudaLaunchConfig_t c = {};
-  int kmax = 0;
-  for (int i = 0; i < p.nsrc; ++i) kmax = std::max(kmax, p.src[i].K);
-  c.gridDim = dim3(p.nb, p.nsrc, (kmax + kAmaxChunk - 1) / kAmaxChunk);
-  c.blockDim = dim3(256);
-  c.stream = s;
-  c.attrs = attr;
-  c.numAttrs = 1;
-  return cudaLaunchKernelEx(&c, tc_amax_kernel, p);
+  return cudaLaunchKernelEx(&c, kern, maps, q);
 }
 
 cudaError_t launch_tc_cache_scatter(const TcScatterParams& p, cudaStream_t s) {
@@ -510,7 +562,7 @@ cudaError_t launch_tc_cache_scatter(const TcScatterParams& p, cudaStream_t s) {
   return cudaLaunchKernelEx(&c, tc_cache_scatter_kernel, p);
 }
 
-cudaError_t launch_tc_swiglu(const TcSwigluParams& p, int /*sm_count*/, cudaStream_t s) {
+cudaError_t launch_tc_swiglu(const TcSwigluParams& p, cudaStream_t s) {
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;

@@ -121,8 +121,9 @@ typedef struct lr_factor_desc {
  *   tokens as N), streaming every factor once per pass of up to 32 tokens;
  *   there the latent goes through an fp32 accumulator in the workspace and
  *   enters the second product as bf16 high and low parts (bf16 factors,
- *   fp32 accuracy) or as int8 high and low codes with a per-token scale
- *   (int8 factors, error within max|z| / 64516 per element).
+ *   fp32 accuracy) or as int8 high and low codes with per-token scales
+ *   taken over each tensor-core unit's slice of the reduction (int8 factors,
+ *   error within the slice's max|z| / 64516 per element).
  * W8A8 path (x_scale != NULL; w_dtype LR_I8, scale_dtype LR_F32):
  *   x int8 [batch, d_in] with per-token scales x_scale f32 [batch] (from
  *   lr_quantize_per_token), y bf16 [batch, d_out]; int8 x int8 -> int32 tensor
@@ -132,11 +133,17 @@ typedef struct lr_factor_desc {
  *     acc2 = z_q B_q (int32);  y = bf16(fp32(fp32(acc2 * s_z[t]) * scale_B[k]))
  *   (LASER results, W8A8 setting; WSVD "Quantization-Aware Training",
  *   weights and activations quantised, e.g. W8A8).
+ *   Workspace (lr_linear_workspace_size with w8a8 = 1; rp = r rounded up
+ *   to 128, bp = batch rounded up to 128, each part rounded up to 256
+ *   bytes): the int32 sums of the first product [batch, rp] (batch * rp * 4
+ *   bytes; zero on entry and left zero: the first product adds its K-split
+ *   pieces into it), then the requantised latent int8 [bp, rp] and its
+ *   scales f32 [bp], which each call overwrites and leaves behind.
  * Weight-only limits: d_in and d_out multiples of 8 (of 16 for int8 weights)
  * and at most 32 KiB per factor row (d <= 16384 for bf16, 8192 for f32).
  * ws: workspace of at least lr_linear_workspace_size(...) bytes: 256 +
  * 8-rounded(min(batch, 8) * d_out) * 4, and for bf16 or int8 factors on the
- * tensor-core path at least 992 + (2 r8 + 2 d_out) * c * 4 with c = 8-rounded
+ * tensor-core path at least 256 + (2 r8 + 2 d_out) * c * 4 with c = 8-rounded
  * min(batch, 32) and r8 the 8-rounded active rank.  Zero on entry
  * (lr_workspace_init); every call leaves it zero.
  * Errors: LR_ERR_INVALID_ARG (null pointers, batch < 1, bad shape or rank),

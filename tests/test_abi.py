@@ -47,20 +47,23 @@ def test_linear_workspace_sizes(lib):
     assert st == L.LR_OK and n == 256 + 4096 * 4
     st, n3 = _ws(lib, _desc(), 3)
     assert st == L.LR_OK and n3 == 256 + 3 * 4096 * 4
-    # bf16 from batch 4 (tensor cores): 736 bytes of per-token maxima, two latent sets [cols, rank] and
-    # two y sets [cols, d_out], cols = 8-rounded min(batch, 32); the larger of the two paths' needs
+    # bf16 from batch 4 (tensor cores): two latent sets [cols, rank] and two y sets [cols, d_out],
+    # cols = 8-rounded min(batch, 32); the larger of the two paths' needs
     st, n16 = _ws(lib, _desc(), 16)
-    assert st == L.LR_OK and n16 == 256 + 736 + (2 * 1024 + 2 * 4096) * 16 * 4
+    assert st == L.LR_OK and n16 == 256 + (2 * 1024 + 2 * 4096) * 16 * 4
     st, n40 = _ws(lib, _desc(), 40)
-    assert st == L.LR_OK and n40 == 256 + 736 + (2 * 1024 + 2 * 4096) * 32 * 4
+    assert st == L.LR_OK and n40 == 256 + (2 * 1024 + 2 * 4096) * 32 * 4
     st, n16f = _ws(lib, _desc(w_dtype=L.LR_F32), 16)
     assert st == L.LR_OK and n16f == 256 + 8 * 4096 * 4
     st, n3s = _ws(lib, _desc(d_out=8), 3)
     assert st == L.LR_OK and n3s == 256 + 24 * 4
     st, _ = _ws(lib, _desc(w_dtype=L.LR_I8), 1)
     assert st == L.LR_ERR_INVALID_ARG  # int8 needs scales
+    # W8A8: int32 sums [batch, rp] + int8 latent [bp, rp] + f32 scales [bp] (rp, bp: 128-rounded; parts 256-rounded)
     st, n = _ws(lib, _desc(w_dtype=L.LR_I8, scale_A=FAKE, scale_B=FAKE), 2048, 1)
-    assert st == L.LR_OK and n > 2048 * 1024
+    assert st == L.LR_OK and n == 2048 * 1024 * 4 + 2048 * 1024 + 2048 * 4
+    st, n = _ws(lib, _desc(w_dtype=L.LR_I8, scale_A=FAKE, scale_B=FAKE, active_rank=200), 130, 1)
+    assert st == L.LR_OK and n == 130 * 256 * 4 + 256 * 256 + 1024
 
 
 def test_linear_validation(lib):
@@ -108,9 +111,9 @@ def test_ffn_validation_and_workspace(lib):
     n = ctypes.c_size_t(0)
     d = _ffn()
     assert lib.lr_swiglu_ffn_workspace_size(ctypes.byref(d), 1, ctypes.byref(n)) == L.LR_OK
-    # tensor-core path (every batch by default): 256 + 736 bytes, then per token (8 columns at batch 1)
+    # tensor-core path (every batch by default): 256 bytes, then per token (8 columns at batch 1)
     # z [rank], gate/up [2 inter], h [inter], y [hidden] fp32
-    assert n.value == 256 + 736 + (1536 + 2 * 11008 + 11008 + 4096) * 8 * 4
+    assert n.value == 256 + (1536 + 2 * 11008 + 11008 + 4096) * 8 * 4
     # the CUDA-core path's need: gate/up of the low-rank channels, h of the dense ones, y
     try:
         assert lib.lr_set_tensor_core_min_batch(64, 64) == L.LR_OK

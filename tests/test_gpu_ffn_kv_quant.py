@@ -38,6 +38,15 @@ def test_hybrid_ffn_llama7b(cuda_device, ffn7b, batch):
     assert err < NORMWISE_TOL, err
 
 
+def test_hybrid_ffn_long_down_slices(cuda_device):
+    # inter 20480: each unit of the down projection stages an 18-block slice of h, which at
+    # 8 tokens (SwiGLU evaluated while staging) takes more than one round of loads per pass
+    d = synth.make_hybrid_ffn(seed=2, hidden=4096, inter=20480, n_lr=16384, rank=256, rotate=False)
+    x = synth.make_activations(8, 4096, seed=2, key=(31, 8), outliers=4)
+    y = lr.lr_swiglu_ffn(_ffn_dev(d), dev(x))
+    assert normwise_rel(y, _ffn_oracle(d, x)) < NORMWISE_TOL
+
+
 @pytest.mark.parametrize("batch", [1, 5])
 def test_hybrid_ffn_cuda_core_path(cuda_device, ffn7b, batch):
     # the CUDA-core FFN kernels (the tensor cores take every batch by default)
@@ -109,7 +118,8 @@ def test_latent_kv_peaky_softmax(cuda_device):
     assert normwise_rel(o, _kv_oracle(d)) < NORMWISE_TOL
 
 
-@pytest.mark.parametrize("rows,cols", [(4, 512), (2048, 5120), (7, 13824)])
+# 40976 and 49152 columns: rows longer than the pieces a block holds in registers
+@pytest.mark.parametrize("rows,cols", [(4, 512), (2048, 5120), (7, 13824), (5, 40976), (3, 49152)])
 def test_quantize_per_token_bit_exact(cuda_device, rows, cols):
     x = synth.make_activations(rows, cols, seed=5, key=(40, rows), outliers=max(1, cols // 1000))
     xq, s = lr.lr_quantize_per_token(dev(x))

@@ -20,7 +20,8 @@ def _rand_i8(rng, shape, lo=-127, hi=127):
     return torch.from_numpy(rng.integers(lo, hi + 1, size=shape).astype(np.int8))
 
 
-@pytest.mark.parametrize("M,N,K", [(128, 256, 128), (200, 336, 272), (2048, 640, 5120), (7, 16, 16)])
+# (1100, 8192, 256): 288 tiles, so every CTA of the persistent grid takes two or more
+@pytest.mark.parametrize("M,N,K", [(128, 256, 128), (200, 336, 272), (2048, 640, 5120), (7, 16, 16), (1100, 8192, 256)])
 @pytest.mark.parametrize("b_layout", [0, 1])
 def test_gemm_s8s32_bit_exact(cuda_device, M, N, K, b_layout):
     rng = np.random.default_rng(M * 7 + N + K + b_layout)
@@ -59,7 +60,9 @@ def _pipeline(d_in, d_out, rank, T, seed):
     return p, xq, sx, q_ref, s_ref, y, res, ref64
 
 
-@pytest.mark.parametrize("d_in,d_out,rank,T", [(512, 768, 320, 256), (256, 512, 96, 130)])
+# (1024, 8192, 200, 1500): the first product split along K across CTAs, the
+# second with several tiles per CTA and a ragged last row of tiles
+@pytest.mark.parametrize("d_in,d_out,rank,T", [(512, 768, 320, 256), (256, 512, 96, 130), (1024, 8192, 200, 1500)])
 def test_w8a8_pipeline_small_bit_exact(cuda_device, d_in, d_out, rank, T):
     p, xq, sx, q_ref, s_ref, y, res, ref64 = _pipeline(d_in, d_out, rank, T, seed=1)
     assert np.array_equal(xq.cpu().numpy(), q_ref) and np.array_equal(sx.cpu().numpy(), s_ref)
