@@ -3,8 +3,10 @@
 // LASER results (W8A8 setting) and WSVD QAT section (weights and
 // activations quantised): one scale per token, s = max|x| / 127, and
 // q = clamp(rint(x / s), -127, 127).  Division and rounding are IEEE fp32
-// (__fdiv_rn, rintf: ties to even) so that the codes are reproducible bit for
-// bit; an all-zero row gets s = 1 and q = 0.
+// (the quotient correctly rounded, rint ties to even) so that the codes are
+// reproducible bit for bit; the quotient is only evaluated where a product
+// with the reciprocal cannot decide the integer (quant_code).  An all-zero
+// row gets s = 1 and q = 0.
 #include "common.cuh"
 #include "internal.h"
 
@@ -16,17 +18,16 @@ namespace {
 // is sized to the row (cols / (8 kPer) threads, rounded up to whole warps),
 // so a row needs one pass over global memory and nothing is staged in
 // shared memory.  Longer rows than kPer * kMaxThreads pieces would re-read the rest.
-constexpr int kPer = 8;
+constexpr int kPer = 4;
 constexpr int kMaxThreads = 512;
 
-LR_DEV uint2 quantize8(const uint4 v, float sc, bool zero) {
+LR_DEV uint2 quantize8(const uint4 v, float sc, float inv, bool zero) {
   float f[8];
   bf16x8_to_f32(v, f);
   uint32_t w[2] = {0u, 0u};
 #pragma unroll
   for (int e = 0; e < 8; ++e) {
-    float q = zero ? 0.f : rintf(__fdiv_rn(f[e], sc));
-    q = fminf(fmaxf(q, -127.f), 127.f);
+    const float q = zero ? 0.f : quant_code(f[e], sc, inv);
     w[e >> 2] |= (uint32_t(int(q)) & 0xffu) << (8 * (e & 3));
   }
   return make_uint2(w[0], w[1]);
@@ -68,13 +69,14 @@ __global__ void __launch_bounds__(kMaxThreads) quantize_rows_kernel(const __nv_b
   const bool zero = (sc == 0.0f);
   if (zero) sc = 1.0f;
   if (threadIdx.x == 0) s[t] = sc;
+  const float inv = __frcp_rn(sc);
   uint2* dst = reinterpret_cast<uint2*>(xq + size_t(t) * cols);
 #pragma unroll
   for (int i = 0; i < kPer; ++i) {
     const int c = threadIdx.x + i * nt;
-    if (c < nchunk) dst[c] = quantize8(v[i], sc, zero);
+    if (c < nchunk) dst[c] = quantize8(v[i], sc, inv, zero);
   }
-  for (int c = threadIdx.x + kPer * nt; c < nchunk; c += nt) dst[c] = quantize8(ld_stream16(src + c), sc, zero);
+  for (int c = threadIdx.x + kPer * nt; c < nchunk; c += nt) dst[c] = quantize8(ld_stream16(src + c), sc, inv, zero);
 }
 
 }  // namespace

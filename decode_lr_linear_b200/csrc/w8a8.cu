@@ -9,8 +9,8 @@
 //   s_z  = max|z| / 127, z_q = clamp(rint(z / s_z))               (requant)
 //   acc2 = z_q B_q                   (tcgen05.mma kind::i8)
 //   y    = bf16(fp32(fp32(acc2 * s_z[t]) * s_B[k]))                (epilogue)
-// Every fp32 step is one IEEE operation (__fmul_rn, __fdiv_rn, rintf), so the
-// codes match an exact emulation bit for bit.
+// Every fp32 step is one IEEE operation (__fmul_rn, the correctly rounded
+// quotient, rintf), so the codes match an exact emulation bit for bit.
 //
 // GEMM kernel: persistent, one CTA per SM, 128 x 256 output tiles.  Warp 0
 // issues TMA loads of 128-byte-swizzled operand tiles into a 4-stage
@@ -325,13 +325,15 @@ __global__ void __launch_bounds__(kThreads, 1) w8a8_gemm_kernel(const __grid_con
 }
 
 // Per-token requantisation of the latent, from the int32 sums of the first
-// product (row stride rank_pad): z_j = fp32(fp32(acc_j * s_x) * s_A[j]), s_z = max_j |z_j| / 127 (1
-// for a zero row), z_q = clamp(rint(z / s_z), -127, 127); columns r ..
-// rank_pad-1 of z_q are zero.  The sums are reset to zero for the next call.
-// One CTA per token; the first kHeld values of each thread stay in registers
-// between the row maximum and the quantisation.
+// product (row stride rank_pad): z_j = fp32(fp32(acc_j * s_x) * s_A[j]), s_z =
+// max_j |z_j| / 127 (1 for a zero row), z_q = clamp(rint(z / s_z), -127, 127);
+// columns r .. rank_pad-1 of z_q are zero (their sums are zero: the first
+// product never writes them).  The sums are reset to zero for the next call.
+// One CTA per token, four columns per access (16-byte loads of the sums, four
+// codes per store); the first kHeldGroups groups of each thread stay in
+// registers between the row maximum and the quantisation.
 constexpr int kReqThreads = 256;
-constexpr int kHeld = 8;
+constexpr int kHeldGroups = 4;
 
 __global__ void __launch_bounds__(kReqThreads) requant_kernel(int32_t* __restrict__ acc, const float* __restrict__ sx,
                                                               const float* __restrict__ sA, int r, int rank_pad,
@@ -341,17 +343,42 @@ __global__ void __launch_bounds__(kReqThreads) requant_kernel(int32_t* __restric
   pdl_launch_dependents();
   pdl_wait();
   int32_t* ar = acc + size_t(t) * rank_pad;
+  const int ng = rank_pad >> 2;
   const float sr = sx[t];
-  float z[kHeld];
+  // z of the four columns of group g (scales past r are not read: their sums are zero)
+  auto zgroup = [&](int g, float* z) {
+    const int4 a = *reinterpret_cast<const int4*>(ar + 4 * g);
+    const int j = 4 * g;
+    float s4[4];
+    if (j + 4 <= r) {
+      const float4 f = *reinterpret_cast<const float4*>(sA + j);
+      s4[0] = f.x; s4[1] = f.y; s4[2] = f.z; s4[3] = f.w;
+    } else {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) s4[e] = j + e < r ? sA[j + e] : 0.f;
+    }
+    z[0] = __fmul_rn(__fmul_rn(__int2float_rn(a.x), sr), s4[0]);
+    z[1] = __fmul_rn(__fmul_rn(__int2float_rn(a.y), sr), s4[1]);
+    z[2] = __fmul_rn(__fmul_rn(__int2float_rn(a.z), sr), s4[2]);
+    z[3] = __fmul_rn(__fmul_rn(__int2float_rn(a.w), sr), s4[3]);
+  };
+  float z[kHeldGroups][4];
   float m = 0.f;
 #pragma unroll
-  for (int i = 0; i < kHeld; ++i) {
-    const int j = threadIdx.x + i * kReqThreads;
-    z[i] = j < r ? __fmul_rn(__fmul_rn(__int2float_rn(ar[j]), sr), sA[j]) : 0.f;
-    m = fmaxf(m, fabsf(z[i]));
+  for (int i = 0; i < kHeldGroups; ++i) {
+    const int g = threadIdx.x + i * kReqThreads;
+    if (g < ng) {
+      zgroup(g, z[i]);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) m = fmaxf(m, fabsf(z[i][e]));
+    }
   }
-  for (int j = threadIdx.x + kHeld * kReqThreads; j < r; j += kReqThreads)
-    m = fmaxf(m, fabsf(__fmul_rn(__fmul_rn(__int2float_rn(ar[j]), sr), sA[j])));
+  for (int g = threadIdx.x + kHeldGroups * kReqThreads; g < ng; g += kReqThreads) {
+    float w[4];
+    zgroup(g, w);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) m = fmaxf(m, fabsf(w[e]));
+  }
   m = warp_max(m);
   if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
   __syncthreads();
@@ -362,24 +389,28 @@ __global__ void __launch_bounds__(kReqThreads) requant_kernel(int32_t* __restric
   const bool zero = sc == 0.0f;
   if (zero) sc = 1.0f;
   if (threadIdx.x == 0) sz[t] = sc;
-  int8_t* qr = zq + size_t(t) * rank_pad;
-  auto code = [&](float v) -> int8_t {
-    const float c = zero ? 0.f : fminf(fmaxf(rintf(__fdiv_rn(v, sc)), -127.f), 127.f);
-    return int8_t(int(c));
+  uint32_t* qr = reinterpret_cast<uint32_t*>(zq + size_t(t) * rank_pad);
+  const float inv = __frcp_rn(sc);
+  auto put = [&](int g, const float* w) {
+    uint32_t word = 0;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float c = zero ? 0.f : quant_code(w[e], sc, inv);
+      word |= (uint32_t(int(c)) & 0xffu) << (8 * e);
+    }
+    qr[g] = word;
+    *reinterpret_cast<int4*>(ar + 4 * g) = make_int4(0, 0, 0, 0);
   };
 #pragma unroll
-  for (int i = 0; i < kHeld; ++i) {
-    const int j = threadIdx.x + i * kReqThreads;
-    if (j < r) {
-      qr[j] = code(z[i]);
-      ar[j] = 0;
-    }
+  for (int i = 0; i < kHeldGroups; ++i) {
+    const int g = threadIdx.x + i * kReqThreads;
+    if (g < ng) put(g, z[i]);
   }
-  for (int j = threadIdx.x + kHeld * kReqThreads; j < r; j += kReqThreads) {
-    qr[j] = code(__fmul_rn(__fmul_rn(__int2float_rn(ar[j]), sr), sA[j]));
-    ar[j] = 0;
+  for (int g = threadIdx.x + kHeldGroups * kReqThreads; g < ng; g += kReqThreads) {
+    float w[4];
+    zgroup(g, w);
+    put(g, w);
   }
-  for (int j = r + threadIdx.x; j < rank_pad; j += kReqThreads) qr[j] = 0;
 }
 
 // Persistent grid: one CTA per SM at most (the shared-memory ring keeps it

@@ -128,6 +128,22 @@ def test_quantize_per_token_bit_exact(cuda_device, rows, cols):
     assert np.array_equal(xq.cpu().numpy(), q_ref)
 
 
+def test_quantize_dense_ties(cuda_device):
+    # max 63.5 gives s = 0.5 exactly, so every multiple of 0.25 divides to an exact
+    # half-integer (a tie, rounded to even); the other rows mix in scales that are
+    # not powers of two
+    rng = np.random.default_rng(11)
+    x = torch.from_numpy(rng.integers(-254, 255, size=(64, 2048)).astype(np.float32) * 0.25)
+    x[:, 0] = 63.5
+    x[32:] *= 1.171875   # (rounded to bf16 below) s no longer a power of two
+    x = x.to(torch.bfloat16)
+    xq, s = lr.lr_quantize_per_token(dev(x))
+    q_ref, s_ref = ow8.quantize_per_token(x)
+    assert np.array_equal(s.cpu().numpy(), s_ref)
+    assert np.array_equal(xq.cpu().numpy(), q_ref)
+    assert s[0].item() == 0.5
+
+
 def test_quantize_zero_row_and_ties(cuda_device):
     x = torch.zeros(3, 32, dtype=torch.bfloat16)
     x[1, :8] = torch.tensor([127.0, 2.5, 3.5, -2.5, -0.5, 0.5, 1.5, -127.0])
