@@ -9,6 +9,7 @@
 // row gets s = 1 and q = 0.
 #include "common.cuh"
 #include "internal.h"
+#include "quant.cuh"
 
 namespace lr {
 namespace {

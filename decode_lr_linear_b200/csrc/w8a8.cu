@@ -34,6 +34,7 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "quant.cuh"
 #include "tc.cuh"
 
 namespace lr {
