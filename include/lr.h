@@ -189,8 +189,8 @@ LR_API lr_status_t lr_linear_grouped_workspace_size(const lr_factor_desc_t* desc
  * scale_dtype; any batch >= 1 (one launch per 8 rows or fewer, depending on
  * the widest row); at most LR_MAX_CHAIN steps.
  * bf16 and int8 factors from batch 4 run on the tensor cores instead (as
- * lr_linear: two launches per step and pass of up to 32 tokens, four with
- * int8 factors, plus one at the end; there the
+ * lr_linear: two launches per step and pass of up to 32 tokens, plus one at
+ * the end; there the
  * step right before is read at fp32 from its accumulator and an older step
  * from its stored output).
  * On the CUDA-core path, one persistent CTA per SM (all resident: checked before the
