@@ -84,6 +84,31 @@ def test_append_writes_only_the_new_positions(cuda_device, use_ws):
         assert torch.equal(cv[b][:, keep], d["C_V"][b][:, keep])
 
 
+def test_append_repeated_on_one_workspace(cuda_device):
+    # three appends through the same workspace: every call writes the right latents, and the
+    # workspace (the product's accumulator) is all zero again afterwards
+    heads, rank, hidden, ctx, batch = 32, 32, 4096, 64, 3
+    pr = synth.make_latent_producer(heads, rank, hidden, seed=4)
+    d = synth.make_latent_kv(batch=batch, heads=heads, ctx=ctx, seed=8)
+    kv = lr.LatentKv(batch, heads, ctx, dev(d["B_K"]), dev(d["B_V"]), d["scale"])
+    CK, CV = dev(d["C_K"]), dev(d["C_V"])
+    ws = lr.workspace(lr.lr_latent_kv_append_workspace_size(kv, hidden), CK.device)
+    ck_ref, cv_ref = d["C_K"].clone(), d["C_V"].clone()
+    for call in range(3):
+        x = synth.make_activations(batch, hidden, seed=4, key=(41, call))
+        pos = torch.tensor([call, 10 + call, 30 + 2 * call], dtype=torch.int32)
+        lr.lr_latent_kv_append(kv, dev(pr["A_KV"]), dev(x), dev(pos), CK, CV, ws=ws)
+        rk, rv = okv.append_latents(x, pr["A_KV"], heads, rank, ck_ref, cv_ref, pos.numpy())
+        for b in range(batch):
+            p = int(pos[b])
+            assert normwise_rel(CK.cpu()[b, :, p], rk[b, :, p]) < NORMWISE_TOL
+            assert normwise_rel(CV.cpu()[b, :, p], rv[b, :, p]) < NORMWISE_TOL
+        ck_ref, cv_ref = CK.cpu(), CV.cpu()
+    torch.cuda.synchronize()
+    assert int(ws.abs().max()) == 0
+    assert lr.lr_check_device_error() == 0
+
+
 def test_decode_step_append_then_rotated_attention(cuda_device):
     # one decode step of a layer's attention: write the new token's latents, then attend with rotation
     heads, rank, hidden, ctx, batch, base = 32, 32, 4096, 2048, 4, 10000.0
