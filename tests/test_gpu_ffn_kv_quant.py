@@ -40,7 +40,7 @@ def test_hybrid_ffn_llama7b(cuda_device, ffn7b, batch):
 
 def test_hybrid_ffn_long_down_slices(cuda_device):
     # inter 20480: each unit of the down projection stages an 18-block slice of h, which at
-    # 8 tokens (SwiGLU evaluated while staging) takes more than one round of loads per pass
+    # 8 tokens takes more than one round of loads per pass (pieces read again for the codes)
     d = synth.make_hybrid_ffn(seed=2, hidden=4096, inter=20480, n_lr=16384, rank=256, rotate=False)
     x = synth.make_activations(8, 4096, seed=2, key=(31, 8), outliers=4)
     y = lr.lr_swiglu_ffn(_ffn_dev(d), dev(x))
